@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the verification hot path on B200.
+
+Workload (per GPU): batched chain verification of B=64 sequences with K=8
+drafts over a V=128256 bf16 vocabulary (targets N(0, 2^2) plus a Zipf(1.1)
+log-prior over ids, drafts = target + N(0, 1), T = 1), followed by the
+paged-KV commit of a+1 rows per sequence (block 16, contexts U[512, 4096],
+128 KiB of K/V per token, hidden rows of 4096 bf16). One step = row
+statistics + accept/residual decide + commit, through the C ABI. Each step
+verifies a fresh Philox round and commits against the same committed prefix,
+so it rolls the previous round back and grows again: the pool stays bounded
+and every step does the same kind of work.
+
+Prints one JSON line (rank 0). ``--impl reference`` times the fp64 oracle on
+the host cores instead (the reference arm of this build).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "verified tokens/s and achieved HBM GB/s vs peak (B=64,K=8,V=128256 bf16)"
+B, K, V = 64, 8, 128256
+KV_BYTES_PER_TOKEN = 32 * 2 * 8 * 128 * 2       # layers x {K,V} x heads x dim x bf16
+HID_BYTES_PER_TOKEN = 4096 * 2
+LOGIT_BYTES = B * (2 * K + 1) * V * 2           # every target and draft row once
+WORKLOAD = ("batched chain verification + paged commit: B=64, K=8, V=128256 bf16 logits "
+            "(N(0,4) + Zipf(1.1) log-prior targets, drafts +N(0,1), T=1), block 16, "
+            "contexts U[512,4096], 128 KiB K/V + 8 KiB hidden per token")
+NCU_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+ROW_STATS_SOURCES = ["row_stats.cu", "common.cuh", "kernels.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# Distributed plumbing (one process per GPU, no collective on the data path)
+# ----------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def reduce(self, x: float, op: str) -> float:
+        if not self.pg:
+            return x
+        dev = "cuda" if torch.cuda.is_available() and self.pg.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX if op == "max" else self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 7:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def row_stats_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "speculative_decoding_verification_89_b200", "csrc")
+    for f in ROW_STATS_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic():
+    """DRAM bytes per launch of the row-statistics kernel from the committed
+    ncu summary, or None if absent or taken on different kernel source."""
+    try:
+        with open(NCU_TRAFFIC) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != row_stats_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# The oracle on the host (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def run_oracle_steps(prob_host, tables, seq_lens, free_stack, free_top, seqs, n_steps,
+                     rnd0=0):
+    """n_steps oracle steps; step s verifies sequence seqs[s % len] at round
+    rnd0 + s // len and commits its rows. Returns (tokens, seconds)."""
+    from oracle.commit import commit_paged
+    from oracle.verify import verify_chain
+    tok = 0
+    t0 = time.perf_counter()
+    for s in range(n_steps):
+        b = seqs[s % len(seqs)]
+        r = verify_chain(prob_host["tgt"][b:b + 1], prob_host["drf"][b:b + 1],
+                         prob_host["draft"][b:b + 1], prob_host["T"][b:b + 1], 2,
+                         prob_host["sid"][b:b + 1], rnd0 + s // len(seqs))[0]
+        keep = np.array([r.accepted + 1])
+        c = commit_paged(tables[b:b + 1], seq_lens[b:b + 1], seq_lens[b:b + 1], keep,
+                         free_stack, free_top, 16, len(free_stack), K + 1)
+        assert c.status == 0
+        tok += r.accepted + 1
+    return tok, time.perf_counter() - t0
+
+
+def host_problem(prob, state):
+    to64 = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
+    return ({"tgt": to64(prob.tgt), "drf": to64(prob.drf),
+             "draft": prob.draft_tok.cpu().numpy(), "T": prob.temperature.cpu().numpy(),
+             "sid": prob.seq_id.cpu().numpy()},
+            state.tables.cpu().numpy(), state.seq_lens.cpu().numpy(),
+            state.free_stack.cpu().numpy(), int(state.free_top.cpu()[0]))
+
+
+def cpu_baseline(prob, state, budget_s=12.0):
+    hp, tables, lens, stack, top = host_problem(prob, state)
+    tok1, t1 = run_oracle_steps(hp, tables, lens, stack, top, [0], 1)
+    n = max(2, min(4 * B, int(budget_s / max(t1, 1e-3))))
+    tok, sec = run_oracle_steps(hp, tables, lens, stack, top, list(range(B)), n)
+    return {"value": tok / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} sequence-rounds of the same workload (chain verify + commit, "
+                      f"fp64 numpy, single thread), {sec:.1f} s"}
+
+
+def spot_check(prob, acc_round0):
+    """Oracle vs GPU on two sequences of round 0 (both as run in the bench)."""
+    from oracle.verify import verify_chain
+    to64 = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
+    ok = True
+    for b in (0, B - 1):
+        r = verify_chain(to64(prob.tgt[b:b + 1]), to64(prob.drf[b:b + 1]),
+                         prob.draft_tok[b:b + 1].cpu().numpy(),
+                         prob.temperature[b:b + 1].cpu().numpy(), prob.seed,
+                         prob.seq_id[b:b + 1].cpu().numpy(), 0)[0]
+        if r.accepted != int(acc_round0[b]):
+            ok = ok and min(d.margin for d in r.decisions) < 1e-6
+    return "ok" if ok else "MISMATCH"
+
+
+# ----------------------------------------------------------------------------
+# Our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, dist):
+    from speculative_decoding_verification_89_b200 import capi
+    from speculative_decoding_verification_89_b200 import workloads as W
+
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    prob = W.chain_batch(device=dev, seed=2 + 1000 * dist.rank, seq_id_base=B * dist.rank)
+    state, bufs = W.commit_setup(B, K, device=dev, seed=2 + dist.rank)
+    base = state.seq_lens.clone()
+    total = args.warmup + args.steps
+    hist = torch.zeros((total, B), dtype=torch.int32, device=dev)
+    out_tok = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = capi.workspace(B, K, V, torch.bfloat16, device=dev)
+    tgt, drf, T, sid, dt = prob.tgt, prob.drf, prob.temperature, prob.seq_id, prob.draft_tok
+
+    def row_stats():
+        capi.spec_chain_row_stats(tgt, drf, T, status, ws, stream=stream)
+
+    def decide_commit(i):
+        capi.spec_chain_decide(tgt, drf, dt, T, prob.seed, sid, i, hist[i], out_tok, status, ws,
+                               stream=stream)
+        capi.spec_commit_paged(state.tables, state.seq_lens, base, hist[i], 1, state.free_stack,
+                               state.free_top, K + 1, status, block_size=16,
+                               kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
+                               hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
+                               hid_off=bufs.hid_off, stream=stream)
+
+    clocks = Clocks(dist.local)
+    clocks.start()
+    for i in range(args.warmup):
+        row_stats()
+        decide_commit(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for s in range(args.steps):
+        i = args.warmup + s
+        ev[s][0].record(stream)
+        row_stats()
+        ev[s][1].record(stream)
+        decide_commit(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    st = int(status.item())
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {capi.spec_status_string(st)}")
+    ms = e0.elapsed_time(e1)
+    ms_max = dist.reduce(ms, "max")
+    acc = hist[args.warmup:].cpu().numpy()
+    tokens = float((acc + 1).sum())
+    tokens_all = dist.reduce(tokens, "sum")
+    rs_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    commit_bytes = tokens * 2 * (KV_BYTES_PER_TOKEN + HID_BYTES_PER_TOKEN)
+    step_bytes = LOGIT_BYTES * args.steps + commit_bytes
+    bytes_all = dist.reduce(step_bytes, "sum")
+
+    peak, peak_kind = measured_peak()
+    achieved = LOGIT_BYTES / (rs_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": tokens_all / (ms_max * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "logits_dtype": "bf16", "batch_per_gpu": B,
+                   "drafts": K, "vocab": V, "l2": "inputs 279 MB per step > 126 MB L2; no flush",
+                   "parallelism": f"replicas x{dist.world} (independent sequences per GPU)"},
+        "hbm_gbs": bytes_all / (ms_max * 1e-3) / 1e9,
+        "hbm_frac_of_8tbs": bytes_all / (ms_max * 1e-3) / 8e12,
+        "hbm_frac_of_measured": bytes_all / (ms_max * 1e-3) / 1e9 / peak,
+        "mean_accepted": float(acc.mean()),
+        "roofline": {"bound": "hbm", "kernel": "row_stats_kernel (bf16, chain rows)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": ncu_traffic(), "algorithmic_bytes_per_launch": LOGIT_BYTES,
+                     "launch_ms": rs_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, prob, state, bufs, base, dev, dist)
+    if dist.world == 1 and dist.rank == 0:
+        result["parity_spot_check"] = spot_check(prob, hist[0].cpu().numpy())
+        if not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(prob, state)
+    return result
+
+
+def run_e2e(args, prob, state, bufs, base, dev, dist):
+    """Same step through the public API with pinned host inputs: each step
+    copies its logits, drafts, temperatures, ids and staged K/V + hidden rows
+    host->device and reads accept lengths and tokens back."""
+    from speculative_decoding_verification_89_b200 import capi
+    steps = max(3, min(args.steps, 100))
+    host = {k: v.cpu().pin_memory() for k, v in
+            dict(tgt=prob.tgt, drf=prob.drf, dt=prob.draft_tok, T=prob.temperature,
+                 sid=prob.seq_id, kv=bufs.kv_stage, hid=bufs.hid_stage).items()}
+    d = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    out = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    acc_h = torch.empty((steps, B), dtype=torch.int32).pin_memory()
+    out_h = torch.empty((steps, B, K + 1), dtype=torch.int32).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = capi.workspace(B, K, V, torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = acc.numel() * 4 + out.numel() * 4
+
+    def step(i):
+        for k in host:
+            d[k].copy_(host[k], non_blocking=True)
+        capi.spec_verify_chain(d["tgt"], d["drf"], d["dt"], d["T"], prob.seed, d["sid"], i, acc,
+                               out, status, ws, stream=stream)
+        capi.spec_commit_paged(state.tables, state.seq_lens, base, acc, 1, state.free_stack,
+                               state.free_top, K + 1, status, block_size=16,
+                               kv_stage=d["kv"], kv_pool=bufs.kv_pool, hid_stage=d["hid"],
+                               hid_out=bufs.hid_out, hid_off=bufs.hid_off, stream=stream)
+        acc_h[i].copy_(acc, non_blocking=True)
+        out_h[i].copy_(out, non_blocking=True)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = dist.reduce(e0.elapsed_time(e1), "max")
+    tokens = dist.reduce(float((acc_h.numpy() + 1).sum()), "sum")
+    if int(status.item()) != 0:
+        raise RuntimeError("device status during e2e run")
+    return {"value": tokens / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ----------------------------------------------------------------------------
+# Reference arm: the oracle on the host cores
+# ----------------------------------------------------------------------------
+def run_reference(args, dist):
+    from speculative_decoding_verification_89_b200 import workloads as W
+    prob = W.chain_batch(device="cpu")
+    state, _ = W.commit_setup(B, K, device="cpu", with_kv=False)
+    hp, tables, lens, stack, top = host_problem(prob, state)
+    # One step = one sequence-round; bounded so the whole run takes minutes.
+    _, t1 = run_oracle_steps(hp, tables, lens, stack, top, [0], 1)
+    steps = max(3, min(args.steps, int(120.0 / max(t1, 1e-3))))
+    warm = max(1, min(args.warmup, 3))
+    run_oracle_steps(hp, tables, lens, stack, top, list(range(B)), warm)
+    tok, sec = run_oracle_steps(hp, tables, lens, stack, top, list(range(B)), steps, rnd0=warm)
+    value = tok / sec
+    sample = (f"{steps} sequence-rounds (one sequence's chain verify + commit per step) of the "
+              f"B=64 K=8 V=128256 workload, fp64 numpy oracle, single thread")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": dist.world, "steps": steps, "warmup": warm, "ms_per_step": sec * 1e3 / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "logits_dtype": "bf16"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    dist = Dist()
+    if args.impl == "reference":
+        if dist.rank == 0:
+            print(json.dumps(run_reference(args, dist)), flush=True)
+        return 0
+    dist.init("nccl")
+    try:
+        res = run_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

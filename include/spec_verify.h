@@ -1,0 +1,237 @@
+/*
+ * spec_verify.h -- C ABI of libspecverify: batched lossless speculative-
+ * sampling verification, two-stage (L_d -> L_i -> L_f) verification over a
+ * window, and the paged-KV commit that follows it, on NVIDIA B200 (sm_100a).
+ *
+ * Where the operations come from
+ *   [HS]  "HiSpec: Hierarchical Speculative Decoding for LLMs", gist.science
+ *         summary of arXiv 2510.01336: section 2 "Methodik" -- Kernmechanismus
+ *         (the exits L_d, L_i ~ 1/4 depth, L_f) and the bullets "Verlustfreie
+ *         Garantie" (two-stage lossless check), "Dynamische
+ *         Verifizierungsrichtlinie" (window of N_i = 4), "Wiederverwendung von
+ *         KV-Cache und versteckten Zustaenden" (buffer, then drop rejected
+ *         entries) and "Unterstuetzung fuer Batch-Inferenz" (paged attention,
+ *         block tables, per-sequence acceptance without padding).
+ *   [SSD] "Speculative Speculative Decoding", gist.science summary of arXiv
+ *         2603.03251, Technische Zusammenfassung section 2 item 1 (an outcome
+ *         is the accepted count plus a bonus token) and section 3.B (residual
+ *         distribution proportional to the target-minus-draft difference).
+ * The pages print no formulas. The rules implemented are the standard
+ * speculative-sampling rules they appeal to: with p = softmax(l_target / T)
+ * and q = softmax(l_draft / T), draft x_j is accepted iff u_j * q_j(x_j) <
+ * p_j(x_j); at the first rejection a the token is drawn from
+ * normalize(max(0, p_a - q_a)) (from p_a if that mass is zero); if all K are
+ * accepted a bonus token is drawn from p_K. A draw with weights w and uniform
+ * u' takes the smallest v with sum_{t<=v} w_t > u' * sum_t w_t. T == 0 is the
+ * greedy path: accept iff x_j == argmax l_target_j (ties: smallest id), emit
+ * the argmax.
+ *
+ * Randomness: Philox4x32-10 (Salmon et al., SC'11), key = (seed & 0xffffffff,
+ * seed >> 32), counter = (seq_id[b], round, position, stage); lane 0 is the
+ * accept uniform, lane 1 the draw uniform; u = (2*(x >> 9) + 1) * 2^-24.
+ * Stage 1 = chain verification and the first stage; stage 2 = second stage.
+ *
+ * Conventions for every call
+ *   - Pointers are DEVICE memory owned by the caller unless a comment says
+ *     otherwise; the library allocates nothing and keeps no state between
+ *     calls. Work is queued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream); no call synchronises the host.
+ *   - Return value: SPEC_OK when the work was queued. Argument errors are
+ *     found on the host before anything is launched (SPEC_EINVAL,
+ *     SPEC_EWORKSPACE); a failed launch returns SPEC_ECUDA.
+ *   - `dev_status` (device int32) records conditions only the device can see.
+ *     It is sticky: kernels only ever store an error code into it, and only
+ *     while it still holds SPEC_OK (first error wins). The caller sets it to
+ *     SPEC_OK (0) and reads it when it wants. A commit does nothing while it
+ *     holds an error.
+ *   - Logit rows must start on 16-byte boundaries: the base pointers are
+ *     16-byte aligned and the row stride times the element size is a
+ *     multiple of 16 bytes. V itself may be any value >= 1.
+ *   - Calls on different streams must use different workspaces.
+ */
+#ifndef SPEC_VERIFY_H
+#define SPEC_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPEC_OK = 0,
+  SPEC_EINVAL = -1,      /* bad argument (host) / bad value (device, commit) */
+  SPEC_ECUDA = -2,       /* a CUDA launch or API call failed                 */
+  SPEC_EWORKSPACE = -3,  /* workspace missing, misaligned or too small       */
+  SPEC_ENOBLOCKS = -4,   /* device: the free-block pool cannot cover a commit */
+  SPEC_ETIMEOUT = -5,    /* device: a bounded wait ran out                   */
+  SPEC_EDEVICE = -6      /* device: invalid input value in a verification
+                            (draft id outside [0,V), temperature negative or
+                            not finite, a row with no finite maximum, window
+                            length out of range); the sequence's outputs are
+                            set to -1 and the others are still computed      */
+} spec_status;
+
+typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
+
+/* Limits checked on the host. */
+#define SPEC_MAX_K 256           /* drafts per sequence per call      */
+#define SPEC_MAX_V (1 << 22)     /* vocabulary size                   */
+
+/* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
+ * chain call, Ni > 0 a two-stage call. Returns 0 for invalid sizes. */
+size_t spec_workspace_bytes(int B, int K, int V, int dtype, int Ni);
+
+/* Static English text for a status code (host memory, never freed). */
+const char* spec_status_string(int status);
+
+/* ---------------------------------------------------------------------------
+ * Chain verification ([HS] Kernmechanismus with one verifying exit; [SSD] 2.1)
+ *
+ * tgt   : target logits [B, K+1, V]; row (b, j) starts at element
+ *         (b*(K+1) + j) * ld_tgt. Row j is the target law of slot j; row K
+ *         gives the bonus token.
+ * drf   : draft logits  [B, K, V];   row (b, j) starts at (b*K + j) * ld_drf.
+ *         Not read for sequences with temperature 0.
+ * dtype : SPEC_F32 or SPEC_BF16 (both tensors).
+ * draft_tok   : int32 [B, K] drafted token ids.
+ * temperature : float [B]: 0 (greedy) or within [1e-6, 1e6]; anything else
+ *               marks the sequence invalid (SPEC_EDEVICE).
+ * seed, seq_id (int32 [B]), round : Philox key and counter fields.
+ * accept_len  : out int32 [B], a_b in [0, K] (-1 if the sequence is invalid).
+ * out_tok     : out int32 [B, K+1]: drafts 0..a-1, then the drawn token at a,
+ *               then -1.
+ * diag        : optional out double [B, 4K+2] (NULL to skip): natural-log
+ *               partition ln sum exp(l/T) of target rows 0..K, of draft rows
+ *               0..K-1, p_j(x_j) for j < K, q_j(x_j) for j < K, and the mass
+ *               Z of the final draw (sum max(0, p_a - q_a), or sum p_K for the
+ *               bonus). NaN for greedy sequences.
+ * ws, ws_bytes: workspace of at least spec_workspace_bytes(B, K, V, dtype, 0)
+ *               bytes, 256-byte aligned. No initial contents are needed.
+ * Equivalent to spec_chain_row_stats followed by spec_chain_decide.
+ * ------------------------------------------------------------------------- */
+int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf,
+                      int64_t ld_drf, int dtype, int B, int K, int V,
+                      const int32_t* draft_tok, const float* temperature,
+                      uint64_t seed, const int32_t* seq_id, uint32_t round,
+                      int32_t* accept_len, int32_t* out_tok, double* diag,
+                      int32_t* dev_status, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* First half of spec_verify_chain: per-row softmax statistics (running max,
+ * sum of exponentials, first argmax) over every target and draft row, split
+ * over vocabulary tiles, written into the workspace. Same arguments. */
+int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf,
+                         int64_t ld_drf, int dtype, int B, int K, int V,
+                         const float* temperature, int32_t* dev_status,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Second half: combines the workspace statistics, runs the accept test on all
+ * K positions, finds the first rejection and draws the resampled or bonus
+ * token (re-reading only rows a of the target and draft). The logits,
+ * temperatures and workspace must be those of the preceding
+ * spec_chain_row_stats call. */
+int spec_chain_decide(const void* tgt, int64_t ld_tgt, const void* drf,
+                      int64_t ld_drf, int dtype, int B, int K, int V,
+                      const int32_t* draft_tok, const float* temperature,
+                      uint64_t seed, const int32_t* seq_id, uint32_t round,
+                      int32_t* accept_len, int32_t* out_tok, double* diag,
+                      int32_t* dev_status, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Two-stage verification, one round ([HS] Verlustfreie Garantie and
+ * Dynamische Verifizierungsrichtlinie).
+ *
+ * lg_d, lg_i, lg_f : logits of the exits L_d, L_i, L_f, each [B, S, V] with
+ *         S = Ni + K + 1; row (b, s) starts at element (b*S + s) * ld. Rows
+ *         are indexed by slot since the last commit: slot s is the law of the
+ *         s-th token after the committed prefix. The caller writes rows for
+ *         slots >= win_len[b] before each call and leaves earlier slots
+ *         unchanged within a window cycle.
+ * Ni    : window size (>= 1). K: drafts per round (>= 1).
+ * draft_tok : int32 [B, K], drafts for slots win_len[b] .. win_len[b]+K-1.
+ * temperature, seed, seq_id, round : as for chain verification; stage one
+ *         uses stage tag 1 and stage two stage tag 2, position = slot.
+ * win_len : in/out int32 [B], tokens tentatively accepted in the current
+ *         cycle (0 <= win_len < Ni on entry).
+ * win_tok : in/out int32 [B, Ni+K], the window's tokens.
+ * win_stat: in/out double [B, Ni+K, 2]: for each window slot, the largest raw
+ *         logit m of its L_i row and ln sum_v exp((l_v - m)/T), buffered so
+ *         stage two does not recompute them (the row's log-partition is
+ *         m/T + the second value). NaN for greedy sequences.
+ * Stage one checks the drafts against L_i (draft law L_d) at slots
+ * w..w+K; its a1 accepted drafts and its drawn token join the window. If the
+ * window then holds >= Ni tokens, stage two checks them against L_f (draft
+ * law: L_i at each slot; bonus row: L_f at slot |W|), commits a2 + 1 tokens
+ * and empties the window.
+ * acc1    : out int32 [B] stage-one accepted count (-1 if invalid).
+ * acc2    : out int32 [B] stage-two accepted count, -1 if stage two did not run.
+ * commit_tok : out int32 [B, Ni+K+1] committed tokens then -1.
+ * commit_n   : out int32 [B] number of committed tokens (0 if none).
+ * diag    : optional out double [B, 4K + 3S + 1]: the chain layout for stage
+ *         one, then ln-partition of L_f slots 0..S-1, p_f(tok_s) and
+ *         q_i(tok_s) for s < S-1, and Z of stage two; NaN where not computed.
+ * ws      : spec_workspace_bytes(B, K, V, dtype, Ni) bytes.
+ * ------------------------------------------------------------------------- */
+int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f,
+                     int64_t ld, int dtype, int B, int K, int V, int Ni,
+                     const int32_t* draft_tok, const float* temperature,
+                     uint64_t seed, const int32_t* seq_id, uint32_t round,
+                     int32_t* win_len, int32_t* win_tok, double* win_stat,
+                     int32_t* acc1, int32_t* acc2, int32_t* commit_tok,
+                     int32_t* commit_n, double* diag, int32_t* dev_status,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Paged-KV commit / rollback and pruning of buffered rows ([HS] KV-Cache
+ * reuse and batch-inference bullets).
+ *
+ * block_tables : in/out int32 [B, max_blocks]; a sequence of length n owns
+ *         entries 0 .. ceil(n / block_size) - 1.
+ * seq_lens     : in/out int32 [B] current lengths.
+ * base_len     : int32 [B] committed length before this round (<= seq_lens);
+ *                NULL means base_len = seq_lens (grow only).
+ * keep, keep_add : rows kept per sequence are keep[b] + keep_add (so a chain
+ *         verification's accept_len with keep_add = 1 keeps a + 1 rows);
+ *         must lie in [0, Kp1].
+ * New length len' = base_len + kept. Entries no longer covered are freed
+ * (sequences ascending, each table's tail in ascending index, pushed on
+ * free_stack), then missing entries are allocated (sequences ascending,
+ * popped from the top of the stack).
+ * free_stack   : in/out int32 [num_blocks]; free_top: in/out device int32,
+ *                number of valid entries (top of stack = free_stack[top-1]).
+ * kv_stage : [B, Kp1, layers, 2, kv_heads, head_dim] 2-byte elements (the
+ *            K and V rows staged for each verified token); kv_pool:
+ *            [num_blocks, layers, 2, block_size, kv_heads, head_dim]. Kept row
+ *            i of sequence b goes to position base_len[b] + i. Both NULL for a
+ *            table-only commit. kv_heads*head_dim*2 must be a multiple of 16.
+ * hid_stage: [B, Kp1, hidden] 2-byte elements; hid_out: [sum kept, hidden],
+ *            sequences packed in order; hid_off: out int32 [B+1] exclusive
+ *            scan of the kept counts (may be given without the hidden
+ *            buffers). hidden*2 must be a multiple of 16. NULL to skip.
+ * Every check (kept count, base_len, table entries and popped ids inside
+ * [0, num_blocks), stack capacity, pool size) is made before anything is
+ * changed; on failure *dev_status gets SPEC_EINVAL or SPEC_ENOBLOCKS and no
+ * table, length, stack or buffer is modified.
+ * ------------------------------------------------------------------------- */
+int spec_commit_paged(int B, int block_size, int max_blocks,
+                      int32_t* block_tables, int32_t* seq_lens,
+                      const int32_t* base_len, const int32_t* keep,
+                      int keep_add, int32_t* free_stack, int32_t* free_top,
+                      int num_blocks, int Kp1, const void* kv_stage,
+                      void* kv_pool, int layers, int kv_heads, int head_dim,
+                      const void* hid_stage, void* hid_out, int32_t* hid_off,
+                      int hidden, int32_t* dev_status, void* stream);
+
+/* Diagnostic: the device Philox. For i < n, counter = ctr[4i .. 4i+3]
+ * (device uint32), key from `seed`; writes the two uniforms (accept lane,
+ * draw lane) to out[2i], out[2i+1] (device float). */
+int spec_philox_uniforms(uint64_t seed, const uint32_t* ctr, int n,
+                         float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPEC_VERIFY_H */

@@ -1,0 +1,296 @@
+// C ABI of libspecverify: argument checks on the host, workspace carving and
+// the launch sequence of each call. Declarations and the contract of every
+// entry point are in include/spec_verify.h.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace specv;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+int elem_size(int dtype) { return dtype == SPEC_BF16 ? 2 : 4; }
+int stat_tiles(int V, int dtype) {
+  const int ept = kTileBytes / elem_size(dtype);
+  return (V + ept - 1) / ept;
+}
+
+struct Layout {
+  size_t part, rsum, counters, total;
+};
+
+// Workspace: tile partials for the largest row set, residual tile sums and
+// the per-sequence arrival counters, each 256-byte aligned.
+bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
+  if (B < 0 || K < 0 || K > SPEC_MAX_K || V < 1 || V > SPEC_MAX_V) return false;
+  if (dtype != SPEC_F32 && dtype != SPEC_BF16) return false;
+  if (Ni < 0 || Ni > SPEC_MAX_K) return false;
+  const long long per = Ni > 0 ? (long long)std::max(2 * K + 1, Ni + K + 1) : 2LL * K + 1;
+  const long long rows = (long long)B * per;
+  if (rows > (1LL << 30)) return false;
+  L->part = 0;
+  const size_t part_bytes = align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
+  L->rsum = part_bytes;
+  const size_t rsum_bytes = align_up((size_t)B * residual_tiles(V) * sizeof(double));
+  L->counters = L->rsum + rsum_bytes;
+  L->total = L->counters + align_up((size_t)std::max(B, 1) * sizeof(int));
+  return true;
+}
+
+bool rows_ok(const void* p, int64_t ld, int V, int dtype) {
+  if (!p || !aligned(p, 16)) return false;
+  if (ld < V) return false;
+  return ((ld * elem_size(dtype)) % 16) == 0;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA; }
+
+struct ChainCheck {
+  Layout L;
+  int rc;
+};
+
+ChainCheck check_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                       int dtype, int B, int K, int V, const float* temperature, void* ws,
+                       size_t ws_bytes) {
+  ChainCheck c{};
+  c.rc = SPEC_EINVAL;
+  if (!layout(B, K, V, dtype, 0, &c.L)) return c;
+  if (B == 0) { c.rc = SPEC_OK; return c; }
+  if (!rows_ok(tgt, ld_tgt, V, dtype) || !temperature) return c;
+  if (K > 0 && !rows_ok(drf, ld_drf, V, dtype)) return c;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < c.L.total) { c.rc = SPEC_EWORKSPACE; return c; }
+  c.rc = SPEC_OK;
+  return c;
+}
+
+DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_tok,
+                         const float* temperature, uint64_t seed, const int32_t* seq_id,
+                         uint32_t round, double* diag, int32_t* dev_status, void* ws,
+                         const Layout& L) {
+  DecideCommon c;
+  c.dtype = dtype;
+  c.B = B;
+  c.K = K;
+  c.V = V;
+  c.ntiles = stat_tiles(V, dtype);
+  c.draft_tok = draft_tok;
+  c.temperature = temperature;
+  c.seed = seed;
+  c.seq_id = seq_id;
+  c.round = round;
+  c.part = reinterpret_cast<const Partial*>((char*)ws + L.part);
+  c.rsum = reinterpret_cast<double*>((char*)ws + L.rsum);
+  c.counters = reinterpret_cast<int*>((char*)ws + L.counters);
+  c.nsplit = decide_split(B, V);
+  c.diag = diag;
+  c.status = dev_status;
+  return c;
+}
+
+}  // namespace
+
+#pragma GCC visibility push(default)
+extern "C" {
+
+size_t spec_workspace_bytes(int B, int K, int V, int dtype, int Ni) {
+  Layout L;
+  if (!layout(B, K, V, dtype, Ni, &L)) return 0;
+  return L.total;
+}
+
+const char* spec_status_string(int status) {
+  switch (status) {
+    case SPEC_OK: return "ok";
+    case SPEC_EINVAL: return "invalid argument or value";
+    case SPEC_ECUDA: return "CUDA launch or API error";
+    case SPEC_EWORKSPACE: return "workspace missing, misaligned or too small";
+    case SPEC_ENOBLOCKS: return "free-block pool cannot cover the commit";
+    case SPEC_ETIMEOUT: return "a bounded device wait ran out";
+    case SPEC_EDEVICE: return "invalid input value found on the device";
+    default: return "unknown status";
+  }
+}
+
+int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                         int dtype, int B, int K, int V, const float* temperature,
+                         int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
+                                    ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  const int es = elem_size(dtype);
+  ChainRows rows;
+  rows.tgt = (const unsigned char*)tgt;
+  rows.drf = (const unsigned char*)drf;
+  rows.ld_tgt = ld_tgt * es;
+  rows.ld_drf = ld_drf * es;
+  rows.temperature = temperature;
+  rows.K = K;
+  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V,
+                                      reinterpret_cast<Partial*>((char*)ws + ck.L.part),
+                                      reinterpret_cast<int*>((char*)ws + ck.L.counters), B,
+                                      dev_status, (cudaStream_t)stream));
+}
+
+int spec_chain_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                      int B, int K, int V, const int32_t* draft_tok, const float* temperature,
+                      uint64_t seed, const int32_t* seq_id, uint32_t round, int32_t* accept_len,
+                      int32_t* out_tok, double* diag, int32_t* dev_status, void* ws,
+                      size_t ws_bytes, void* stream) {
+  const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
+                                    ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!seq_id || !accept_len || !out_tok || (K > 0 && !draft_tok)) return SPEC_EINVAL;
+  const int es = elem_size(dtype);
+  ChainDecideArgs a;
+  a.c = common_args(dtype, B, K, V, draft_tok, temperature, seed, seq_id, round, diag, dev_status,
+                    ws, ck.L);
+  a.tgt = (const unsigned char*)tgt;
+  a.drf = (const unsigned char*)drf;
+  a.ld_tgt = ld_tgt * es;
+  a.ld_drf = ld_drf * es;
+  a.accept_len = accept_len;
+  a.out_tok = out_tok;
+  return cuda_status(launch_chain_decide(a, (cudaStream_t)stream));
+}
+
+int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                      int B, int K, int V, const int32_t* draft_tok, const float* temperature,
+                      uint64_t seed, const int32_t* seq_id, uint32_t round, int32_t* accept_len,
+                      int32_t* out_tok, double* diag, int32_t* dev_status, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (!seq_id || !accept_len || !out_tok || (K > 0 && !draft_tok)) {
+    Layout L;
+    if (layout(B, K, V, dtype, 0, &L) && B == 0) return SPEC_OK;
+    return SPEC_EINVAL;
+  }
+  int rc = spec_chain_row_stats(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, dev_status,
+                                ws, ws_bytes, stream);
+  if (rc != SPEC_OK) return rc;
+  return spec_chain_decide(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok, temperature, seed,
+                           seq_id, round, accept_len, out_tok, diag, dev_status, ws, ws_bytes,
+                           stream);
+}
+
+int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64_t ld, int dtype,
+                     int B, int K, int V, int Ni, const int32_t* draft_tok,
+                     const float* temperature, uint64_t seed, const int32_t* seq_id,
+                     uint32_t round, int32_t* win_len, int32_t* win_tok, double* win_stat,
+                     int32_t* acc1, int32_t* acc2, int32_t* commit_tok, int32_t* commit_n,
+                     double* diag, int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  if (K < 1 || Ni < 1 || !layout(B, K, V, dtype, Ni, &L)) return SPEC_EINVAL;
+  if (B == 0) return SPEC_OK;
+  if (!rows_ok(lg_d, ld, V, dtype) || !rows_ok(lg_i, ld, V, dtype) || !rows_ok(lg_f, ld, V, dtype))
+    return SPEC_EINVAL;
+  if (!draft_tok || !temperature || !seq_id || !win_len || !win_tok || !win_stat || !acc1 ||
+      !acc2 || !commit_tok || !commit_n)
+    return SPEC_EINVAL;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < L.total) return SPEC_EWORKSPACE;
+  const int es = elem_size(dtype);
+  const int S = Ni + K + 1;
+  cudaStream_t st = (cudaStream_t)stream;
+  Partial* part = reinterpret_cast<Partial*>((char*)ws + L.part);
+  int* counters = reinterpret_cast<int*>((char*)ws + L.counters);
+
+  HierDecideArgs a;
+  a.c = common_args(dtype, B, K, V, draft_tok, temperature, seed, seq_id, round, diag, dev_status,
+                    ws, L);
+  a.lg_d = (const unsigned char*)lg_d;
+  a.lg_i = (const unsigned char*)lg_i;
+  a.lg_f = (const unsigned char*)lg_f;
+  a.ld = ld * es;
+  a.S = S;
+  a.Ni = Ni;
+  a.win_len = win_len;
+  a.win_tok = win_tok;
+  a.win_stat = win_stat;
+  a.acc1 = acc1;
+  a.acc2 = acc2;
+  a.commit_tok = commit_tok;
+  a.commit_n = commit_n;
+
+  Hier1Rows r1;
+  r1.lg_i = a.lg_i;
+  r1.lg_d = a.lg_d;
+  r1.ld = a.ld;
+  r1.temperature = temperature;
+  r1.win_len = win_len;
+  r1.K = K;
+  r1.S = S;
+  r1.Ni = Ni;
+  cudaError_t e = launch_row_stats(dtype, r1, B * (2 * K + 1), V, part, counters, B, dev_status, st);
+  if (e == cudaSuccess) e = launch_hier1_decide(a, st);
+  Hier2Rows r2;
+  r2.lg_f = a.lg_f;
+  r2.ld = a.ld;
+  r2.temperature = temperature;
+  r2.win_len = win_len;
+  r2.acc1 = acc1;
+  r2.S = S;
+  r2.Ni = Ni;
+  if (e == cudaSuccess) e = launch_row_stats(dtype, r2, B * S, V, part, counters, B, dev_status, st);
+  if (e == cudaSuccess) e = launch_hier2_decide(a, st);
+  return cuda_status(e);
+}
+
+int spec_commit_paged(int B, int block_size, int max_blocks, int32_t* block_tables,
+                      int32_t* seq_lens, const int32_t* base_len, const int32_t* keep, int keep_add,
+                      int32_t* free_stack, int32_t* free_top, int num_blocks, int Kp1,
+                      const void* kv_stage, void* kv_pool, int layers, int kv_heads, int head_dim,
+                      const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden,
+                      int32_t* dev_status, void* stream) {
+  if (B < 0 || block_size < 1 || max_blocks < 0 || num_blocks < 0 || Kp1 < 0) return SPEC_EINVAL;
+  if (B == 0) return SPEC_OK;
+  if (!block_tables || !seq_lens || !keep || !free_stack || !free_top) return SPEC_EINVAL;
+  if ((long long)B * Kp1 > (1LL << 31) - 1) return SPEC_EINVAL;
+  CommitArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if ((kv_stage == nullptr) != (kv_pool == nullptr)) return SPEC_EINVAL;
+  if (kv_stage) {
+    if (layers < 1 || kv_heads < 1 || head_dim < 1) return SPEC_EINVAL;
+    const long long seg = 2LL * kv_heads * head_dim;
+    if (seg % 16 != 0 || seg > (1 << 30)) return SPEC_EINVAL;
+    if (!aligned(kv_stage, 16) || !aligned(kv_pool, 16)) return SPEC_EINVAL;
+    a.layers = layers;
+    a.seg_bytes = (int)seg;
+  }
+  if ((hid_stage == nullptr) != (hid_out == nullptr)) return SPEC_EINVAL;
+  if (hid_stage) {
+    if (hidden < 1 || (2LL * hidden) % 16 != 0 || !hid_off) return SPEC_EINVAL;
+    if (!aligned(hid_stage, 16) || !aligned(hid_out, 16)) return SPEC_EINVAL;
+    a.hid_bytes = 2 * hidden;
+  }
+  a.B = B;
+  a.block_size = block_size;
+  a.max_blocks = max_blocks;
+  a.num_blocks = num_blocks;
+  a.Kp1 = Kp1;
+  a.keep_add = keep_add;
+  a.tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.base_len = base_len;
+  a.keep = keep;
+  a.free_stack = free_stack;
+  a.free_top = free_top;
+  a.kv_stage = (const unsigned char*)kv_stage;
+  a.kv_pool = (unsigned char*)kv_pool;
+  a.hid_stage = (const unsigned char*)hid_stage;
+  a.hid_out = (unsigned char*)hid_out;
+  a.hid_off = hid_off;
+  a.status = dev_status;
+  return cuda_status(launch_commit(a, (cudaStream_t)stream));
+}
+
+int spec_philox_uniforms(uint64_t seed, const uint32_t* ctr, int n, float* out, void* stream) {
+  if (n < 0 || (n > 0 && (!ctr || !out))) return SPEC_EINVAL;
+  return cuda_status(launch_philox(seed, ctr, n, out, (cudaStream_t)stream));
+}
+
+}  // extern "C"
+#pragma GCC visibility pop

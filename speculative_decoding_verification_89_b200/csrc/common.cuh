@@ -1,0 +1,195 @@
+// Device helpers shared by the kernels of libspecverify (sm_100a).
+//
+// Philox4x32-10: J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw,
+// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11 -- S-P network with the
+// 4x32 multipliers and Weyl key increments of its table 2, ten rounds.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/spec_verify.h"
+
+namespace specv {
+
+// ----------------------------------------------------------------------------
+// Constants and small structs
+// ----------------------------------------------------------------------------
+constexpr double kLog2e = 1.4426950408889634073599246810018921;  // 1/ln 2
+constexpr double kLn2 = 0.6931471805599453094172321214581766;
+
+// Row-statistics tiles: 8 KiB of one row, staged by one bulk copy.
+constexpr int kTileBytes = 8192;
+constexpr int kRsWarps = 8;      // warps per row-statistics CTA
+constexpr int kRsStages = 4;     // per-warp ring depth
+constexpr int kRsSmem = kRsWarps * kRsStages * kTileBytes + kRsWarps * kRsStages * 8;
+
+// Residual tiles: 32 lanes x 8 elements.
+constexpr int kResTile = 256;
+constexpr int kDecideThreads = 256;
+constexpr int kMaxSplit = 32;    // CTAs sharing one residual row pair
+
+// Per (row, tile) statistics: the tile's largest raw logit m, its first index,
+// and s = sum over the tile of 2^((l - m) * c), c = log2(e) / T.
+struct Partial {
+  float m;
+  int idx;
+  double s;
+};
+
+template <typename T> struct Elem;
+template <> struct Elem<float> { static constexpr int kDtype = SPEC_F32; };
+template <> struct Elem<__nv_bfloat16> { static constexpr int kDtype = SPEC_BF16; };
+
+// Temperature scale c = log2(e) / T split as c_hi + c_lo (two floats) so the
+// fp32 hot loop carries ~48 bits of the scale. c_hi is rounded toward zero
+// and kept strictly below c, so c_lo > 0 and (-inf) * c_lo stays -inf.
+struct Scale {
+  float hi, lo;
+  double d;
+};
+__device__ __forceinline__ Scale make_scale(float T) {
+  Scale s;
+  s.d = kLog2e / (double)T;
+  s.hi = __double2float_rz(s.d);
+  if ((double)s.hi == s.d) s.hi = nextafterf(s.hi, 0.0f);
+  s.lo = (float)(s.d - (double)s.hi);
+  return s;
+}
+
+// Accepted temperatures: 0 (greedy) or 1e-6 <= T <= 1e6.
+constexpr float kTempMin = 1.0e-6f, kTempMax = 1.0e6f;
+__device__ __forceinline__ bool temp_valid(float T) {
+  return T == 0.0f || (T >= kTempMin && T <= kTempMax);  // false for NaN
+}
+
+// ----------------------------------------------------------------------------
+// Element access
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float load_elem(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p) {
+  unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p));
+  return __uint_as_float(((unsigned)h) << 16);
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 2^x with the hardware approximation (flushes subnormal results to zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ----------------------------------------------------------------------------
+// Philox4x32-10 and the uniform map
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) { k0 += W0; k1 += W1; }
+    const uint32_t lo0 = M0 * c.x, hi0 = __umulhi(M0, c.x);
+    const uint32_t lo1 = M1 * c.z, hi1 = __umulhi(M1, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// (2*(x >> 9) + 1) * 2^-24: odd multiple of 2^-24 in (0, 1), exact in fp32.
+__device__ __forceinline__ float to_uniform(uint32_t x) {
+  return (float)(2u * (x >> 9) + 1u) * 5.9604644775390625e-08f;
+}
+
+__device__ __forceinline__ float2 spec_uniforms(uint64_t seed, uint32_t seq, uint32_t rnd,
+                                                uint32_t pos, uint32_t stage) {
+  uint4 r = philox4x32_10(make_uint4(seq, rnd, pos, stage), (uint32_t)seed,
+                          (uint32_t)(seed >> 32));
+  return make_float2(to_uniform(r.x), to_uniform(r.y));
+}
+
+// ----------------------------------------------------------------------------
+// Status word: first error wins.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void set_status(int32_t* st, int code) {
+  if (st) atomicCAS(reinterpret_cast<int*>(st), 0, code);
+}
+
+// ----------------------------------------------------------------------------
+// mbarrier + 1-D bulk copy (TMA without a tensor map, no multicast)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for a barrier phase, at most `limit_ns` nanoseconds. Returns false on
+// timeout (the caller records SPEC_ETIMEOUT and winds down).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// ----------------------------------------------------------------------------
+// Warp reductions
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// (max value, smallest index among equal maxima); NaN never wins.
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+  }
+}
+
+}  // namespace specv

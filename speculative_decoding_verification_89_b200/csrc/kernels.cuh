@@ -1,0 +1,164 @@
+// Internal interface between the C ABI and the kernels of libspecverify.
+#pragma once
+
+#include "common.cuh"
+
+namespace specv {
+
+// A logit row as the row-statistics kernel sees it.
+struct RowRef {
+  const unsigned char* ptr;  // first element of the row
+  float chi, clo;            // temperature scale (valid when !greedy)
+  bool valid;                // statistics wanted
+  bool greedy;               // argmax only (temperature 0)
+};
+
+__device__ __forceinline__ RowRef make_row(const unsigned char* ptr, float T, bool want) {
+  RowRef r;
+  r.ptr = ptr;
+  r.valid = want && temp_valid(T);
+  r.greedy = (T == 0.0f);
+  r.chi = r.clo = 0.0f;
+  if (r.valid && !r.greedy) {
+    const Scale s = make_scale(T);
+    r.chi = s.hi;
+    r.clo = s.lo;
+  }
+  return r;
+}
+
+// Chain verification rows, grouped by sequence: for sequence b, rows
+// b*(2K+1) + j are target row j (j <= K) and then draft row j - K - 1.
+struct ChainRows {
+  const unsigned char* tgt;
+  const unsigned char* drf;
+  long long ld_tgt, ld_drf;  // row strides in bytes
+  const float* temperature;
+  int K;
+  __device__ __forceinline__ RowRef get(int r) const {
+    const int per = 2 * K + 1, b = r / per, j = r - b * per;
+    const float T = temperature[b];
+    if (j <= K) return make_row(tgt + ((long long)b * (K + 1) + j) * ld_tgt, T, true);
+    return make_row(drf + ((long long)b * K + (j - K - 1)) * ld_drf, T, T != 0.0f);
+  }
+};
+
+// Stage one of the two-stage check: per sequence, L_i rows at slots
+// w .. w+K, then L_d rows at slots w .. w+K-1 (w = window length).
+struct Hier1Rows {
+  const unsigned char* lg_i;
+  const unsigned char* lg_d;
+  long long ld;  // bytes
+  const float* temperature;
+  const int32_t* win_len;
+  int K, S, Ni;
+  __device__ __forceinline__ RowRef get(int r) const {
+    const int per = 2 * K + 1, b = r / per, j = r - b * per;
+    const float T = temperature[b];
+    const int w = win_len[b];
+    const bool ok = (w >= 0 && w < Ni);
+    if (j <= K)
+      return make_row(lg_i + ((long long)b * S + (ok ? w : 0) + j) * ld, T, ok);
+    return make_row(lg_d + ((long long)b * S + (ok ? w : 0) + (j - K - 1)) * ld, T,
+                    ok && T != 0.0f);
+  }
+};
+
+// Stage two: L_f rows at slots 0 .. W of sequences whose window holds
+// W >= Ni tokens after stage one (rows b*S + s).
+struct Hier2Rows {
+  const unsigned char* lg_f;
+  long long ld;
+  const float* temperature;
+  const int32_t* win_len;
+  const int32_t* acc1;
+  int S, Ni;
+  __device__ __forceinline__ RowRef get(int r) const {
+    const int b = r / S, s = r - b * S;
+    const int W = win_len[b];
+    const bool fire = acc1[b] >= 0 && W >= Ni && W < S && s <= W;
+    return make_row(lg_f + (long long)r * ld, temperature[b], fire);
+  }
+};
+
+template <typename Rows>
+cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, Partial* part,
+                             int* zero_words, int nzero, int32_t* status, cudaStream_t st);
+
+// ----------------------------------------------------------------------------
+// Decide kernels (accept test, first rejection, residual / bonus draw)
+// ----------------------------------------------------------------------------
+struct DecideCommon {
+  int dtype, B, K, V, ntiles;      // ntiles: row-statistics tiles per row
+  const int32_t* draft_tok;
+  const float* temperature;
+  uint64_t seed;
+  const int32_t* seq_id;
+  uint32_t round;
+  const Partial* part;
+  double* rsum;                    // [B, nrt] residual tile sums
+  int* counters;                   // [B] arrival counters (zeroed by row stats)
+  int nsplit;                      // CTAs per sequence for the residual pass
+  double* diag;
+  int32_t* status;
+};
+
+struct ChainDecideArgs {
+  DecideCommon c;
+  const unsigned char* tgt;
+  const unsigned char* drf;
+  long long ld_tgt, ld_drf;        // bytes
+  int32_t* accept_len;
+  int32_t* out_tok;
+};
+
+struct HierDecideArgs {
+  DecideCommon c;
+  const unsigned char* lg_d;
+  const unsigned char* lg_i;
+  const unsigned char* lg_f;
+  long long ld;                    // bytes
+  int S, Ni;
+  int32_t* win_len;
+  int32_t* win_tok;
+  double* win_stat;                // [B, Ni+K, 2]: (row max, ln sum exp((l-max)/T))
+  int32_t* acc1;
+  int32_t* acc2;
+  int32_t* commit_tok;
+  int32_t* commit_n;
+};
+
+cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st);
+cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st);
+cudaError_t launch_hier2_decide(const HierDecideArgs& a, cudaStream_t st);
+int decide_split(int B, int V);   // CTAs per sequence for the residual pass
+__host__ __device__ __forceinline__ int residual_tiles(int V) {  // kResTile tiles per row
+  return (V + kResTile - 1) / kResTile;
+}
+
+// ----------------------------------------------------------------------------
+// Paged commit
+// ----------------------------------------------------------------------------
+struct CommitArgs {
+  int B, block_size, max_blocks, num_blocks, Kp1, keep_add;
+  int32_t* tables;
+  int32_t* seq_lens;
+  const int32_t* base_len;
+  const int32_t* keep;
+  int32_t* free_stack;
+  int32_t* free_top;
+  const unsigned char* kv_stage;
+  unsigned char* kv_pool;
+  int layers, seg_bytes;           // seg_bytes = kv_heads * head_dim * 2
+  const unsigned char* hid_stage;
+  unsigned char* hid_out;
+  int32_t* hid_off;
+  int hid_bytes;                   // hidden * 2
+  int32_t* status;
+};
+
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
+
+cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
+
+}  // namespace specv

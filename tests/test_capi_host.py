@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point declared in include/spec_verify.h, sizes workspaces, names
+status codes, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from speculative_decoding_verification_89_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spec_verify.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(spec_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = build_mod.build()
+    return ctypes.CDLL(path)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "spec_verify_chain" in names and "spec_commit_paged" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in spec_verify.h but not exported"
+
+
+def test_binding_covers_the_header():
+    from speculative_decoding_verification_89_b200 import capi
+    assert set(_declared()) <= set(capi.EXPORTED)
+
+
+def test_workspace_bytes(lib):
+    f = lib.spec_workspace_bytes
+    f.restype = ctypes.c_size_t
+    n = f(64, 8, 128256, 1, 0)
+    tiles = (128256 + 4095) // 4096
+    assert n >= 64 * 17 * tiles * 16 and n % 256 == 0
+    assert f(256, 2, 151936, 0, 4) > f(256, 2, 151936, 0, 0)   # S = 7 > 2K+1 = 5
+    assert f(1, 300, 1024, 0, 0) == 0          # K above the limit
+    assert f(1, 4, 0, 0, 0) == 0               # empty vocabulary
+    assert f(1, 4, 10, 7, 0) == 0              # unknown dtype
+
+
+def test_status_strings(lib):
+    f = lib.spec_status_string
+    f.restype = ctypes.c_char_p
+    for code in range(0, -7, -1):
+        assert f(code) and f(code) != b"unknown status"
+    assert f(-99) == b"unknown status"
+
+
+def test_host_argument_errors_launch_nothing(lib):
+    P = ctypes.c_void_p
+    f = lib.spec_verify_chain
+    f.restype = ctypes.c_int
+    f.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int, P, P, ctypes.c_uint64, P, ctypes.c_uint32,
+                  P, P, P, P, P, ctypes.c_size_t, P]
+    fake = P(0x10000)          # never dereferenced: checks fail first
+    odd = P(0x10008)           # not 16-byte aligned
+    base = [fake, 1024, fake, 1024, 0, 4, 3, 1024, fake, fake, 0, fake, 0, fake, fake,
+            None, None, fake, 1 << 30, None]
+    assert f(*base[:5], 0, *base[6:]) == 0           # B = 0: nothing to do
+    bad = list(base); bad[0] = None
+    assert f(*bad) == -1                            # null logits
+    bad = list(base); bad[0] = odd
+    assert f(*bad) == -1                            # misaligned rows
+    bad = list(base); bad[1] = 1000
+    assert f(*bad) == -1                            # stride below V
+    bad = list(base); bad[1] = 1026
+    assert f(*bad) == -1                            # row stride not 16-byte multiple
+    bad = list(base); bad[4] = 5
+    assert f(*bad) == -1                            # dtype
+    bad = list(base); bad[6] = 300
+    assert f(*bad) == -1                            # K too large
+    bad = list(base); bad[17] = None
+    assert f(*bad) == -3                            # no workspace
+    bad = list(base); bad[18] = 16
+    assert f(*bad) == -3                            # workspace too small
+    bad = list(base); bad[13] = None
+    assert f(*bad) == -1                            # no accept_len output
+
+
+def test_commit_host_argument_errors(lib):
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    f = lib.spec_commit_paged
+    f.restype = I
+    f.argtypes = [I, I, I, P, P, P, P, I, P, P, I, I, P, P, I, I, I, P, P, P, I, P, P]
+    fake = P(0x10000)
+    args = [4, 16, 8, fake, fake, None, fake, 1, fake, fake, 64, 9, fake, fake, 32, 8, 128,
+            None, None, None, 0, None, None]
+    bad = list(args); bad[1] = 0
+    assert f(*bad) == -1                  # block size
+    bad = list(args); bad[13] = None
+    assert f(*bad) == -1                  # stage without pool
+    bad = list(args); bad[15] = 1; bad[16] = 3
+    assert f(*bad) == -1                  # segment not a multiple of 16 bytes
+    bad = list(args); bad[17] = fake; bad[18] = fake; bad[20] = 4096
+    assert f(*bad) == -1                  # hidden rows without offsets
+    bad = list(args); bad[3] = None
+    assert f(*bad) == -1                  # no tables
