@@ -225,6 +225,10 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
                       const void* hid_stage, void* hid_out, int32_t* hid_off,
                       int hidden, int32_t* dev_status, void* stream);
 
+/* Diagnostic: text of the last CUDA error behind a SPEC_ECUDA return on the
+ * calling thread ("no error" if none). Static storage. */
+const char* spec_last_cuda_error(void);
+
 /* Diagnostic: the device Philox. For i < n, counter = ctr[4i .. 4i+3]
  * (device uint32), key from `seed`; writes the two uniforms (accept lane,
  * draw lane) to out[2i], out[2i+1] (device float). */

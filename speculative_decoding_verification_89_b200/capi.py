@@ -43,6 +43,7 @@ _SIGS = {
     "spec_commit_paged": (_i, [_i, _i, _i, _p, _p, _p, _p, _i, _p, _p, _i, _i, _p, _p,
                                _i, _i, _i, _p, _p, _p, _i, _p, _p]),
     "spec_philox_uniforms": (_i, [_u64, _p, _i, _p, _p]),
+    "spec_last_cuda_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -54,7 +55,10 @@ EXPORTED = tuple(_SIGS)
 
 class SpecError(RuntimeError):
     def __init__(self, fn, code):
-        super().__init__(f"{fn}: {spec_status_string(code)} ({code})")
+        msg = f"{fn}: {spec_status_string(code)} ({code})"
+        if code == SPEC_ECUDA:
+            msg += f": {_lib.spec_last_cuda_error().decode()}"
+        super().__init__(msg)
         self.code = code
 
 

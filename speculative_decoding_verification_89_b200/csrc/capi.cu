@@ -32,7 +32,7 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   if (Ni < 0 || Ni > SPEC_MAX_K) return false;
   const long long per = Ni > 0 ? (long long)std::max(2 * K + 1, Ni + K + 1) : 2LL * K + 1;
   const long long rows = (long long)B * per;
-  if (rows > (1LL << 30)) return false;
+  if (rows * stat_tiles(V, dtype) >= (1LL << 31)) return false;  // 32-bit item indices
   L->part = 0;
   const size_t part_bytes = align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
   L->rsum = part_bytes;
@@ -48,7 +48,13 @@ bool rows_ok(const void* p, int64_t ld, int V, int dtype) {
   return ((ld * elem_size(dtype)) % 16) == 0;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA; }
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SPEC_OK;
+  g_last_cuda = e;
+  return SPEC_ECUDA;
+}
 
 struct ChainCheck {
   Layout L;
@@ -248,7 +254,8 @@ int spec_commit_paged(int B, int block_size, int max_blocks, int32_t* block_tabl
   if (B < 0 || block_size < 1 || max_blocks < 0 || num_blocks < 0 || Kp1 < 0) return SPEC_EINVAL;
   if (B == 0) return SPEC_OK;
   if (!block_tables || !seq_lens || !keep || !free_stack || !free_top) return SPEC_EINVAL;
-  if ((long long)B * Kp1 > (1LL << 31) - 1) return SPEC_EINVAL;
+  if ((long long)B * Kp1 > (1LL << 31) - 1 || (long long)B * max_blocks > (1LL << 31) - 1)
+    return SPEC_EINVAL;
   CommitArgs a;
   std::memset(&a, 0, sizeof(a));
   if ((kv_stage == nullptr) != (kv_pool == nullptr)) return SPEC_EINVAL;
@@ -286,6 +293,8 @@ int spec_commit_paged(int B, int block_size, int max_blocks, int32_t* block_tabl
   a.status = dev_status;
   return cuda_status(launch_commit(a, (cudaStream_t)stream));
 }
+
+const char* spec_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 
 int spec_philox_uniforms(uint64_t seed, const uint32_t* ctr, int n, float* out, void* stream) {
   if (n < 0 || (n > 0 && (!ctr || !out))) return SPEC_EINVAL;

@@ -64,10 +64,21 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
   __syncthreads();
   if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;  // sticky error
   const int bs = a.block_size;
+  // Every covered table entry must be a valid block id: one coalesced pass
+  // over the flattened [B, max_blocks] table by the whole CTA.
+  int bad = 0;
+  const int nent = a.B * a.max_blocks;  // < 2^31, checked on the host
+  for (int e = threadIdx.x; e < nent; e += blockDim.x) {
+    const int b = e / a.max_blocks, i = e - b * a.max_blocks;
+    if (i < ceil_div(max(a.seq_lens[b], 0), bs)) {
+      const int x = a.tables[e];
+      if (x < 0 || x >= a.num_blocks) bad = 1;
+    }
+  }
   // Each thread owns a contiguous run of sequences.
   const int per = ceil_div(a.B, blockDim.x);
   const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
-  int nfree = 0, nalloc = 0, nkept = 0, bad = 0;
+  int nfree = 0, nalloc = 0, nkept = 0;
   for (int b = b0; b < b1; ++b) {
     const int old_len = a.seq_lens[b];
     const int base = a.base_len ? a.base_len[b] : old_len;
@@ -75,9 +86,6 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
     if (kept < 0 || kept > a.Kp1 || base < 0 || base > old_len || old_len < 0) { bad = 1; continue; }
     const int nb_old = ceil_div(old_len, bs), nb_new = ceil_div(base + kept, bs);
     if (nb_old > a.max_blocks || nb_new > a.max_blocks) { bad = 1; continue; }
-    const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-    for (int i = 0; i < nb_old; ++i)
-      if (tab[i] < 0 || tab[i] >= a.num_blocks) bad = 1;
     nfree += max(0, nb_old - nb_new);
     nalloc += max(0, nb_new - nb_old);
     nkept += kept;

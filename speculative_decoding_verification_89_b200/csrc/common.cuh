@@ -19,11 +19,23 @@ namespace specv {
 constexpr double kLog2e = 1.4426950408889634073599246810018921;  // 1/ln 2
 constexpr double kLn2 = 0.6931471805599453094172321214581766;
 
-// Row-statistics tiles: 8 KiB of one row, staged by one bulk copy.
-constexpr int kTileBytes = 8192;
-constexpr int kRsWarps = 8;      // warps per row-statistics CTA
-constexpr int kRsStages = 4;     // per-warp ring depth
+// Row-statistics tiles: kTileBytes of one row, staged by one bulk copy into a
+// per-warp ring of kRsStages buffers; one CTA of kRsWarps warps per SM.
+#ifndef SPEC_RS_TILE
+#define SPEC_RS_TILE 8192
+#endif
+#ifndef SPEC_RS_WARPS
+#define SPEC_RS_WARPS 8
+#endif
+#ifndef SPEC_RS_STAGES
+#define SPEC_RS_STAGES 3
+#endif
+constexpr int kTileBytes = SPEC_RS_TILE;
+constexpr int kRsWarps = SPEC_RS_WARPS;
+constexpr int kRsStages = SPEC_RS_STAGES;
 constexpr int kRsSmem = kRsWarps * kRsStages * kTileBytes + kRsWarps * kRsStages * 8;
+static_assert(kRsSmem <= 227 * 1024, "row-statistics ring exceeds shared memory");
+static_assert(kTileBytes % 512 == 0, "a tile is a whole number of warp-wide 16-byte vectors");
 
 // Residual tiles: 32 lanes x 8 elements.
 constexpr int kResTile = 256;
@@ -31,7 +43,8 @@ constexpr int kDecideThreads = 256;
 constexpr int kMaxSplit = 32;    // CTAs sharing one residual row pair
 
 // Per (row, tile) statistics: the tile's largest raw logit m, its first index,
-// and s = sum over the tile of 2^((l - m) * c), c = log2(e) / T.
+// and s = sum over the tile of 2^(l*c - M), c = log2(e) / T, with the exact
+// fp32 shift M = fl(m * c_hi) (c_hi from make_scale; M is recomputed from m).
 struct Partial {
   float m;
   int idx;

@@ -29,21 +29,23 @@ constexpr int kUnroll = 4;  // residual tiles in flight per warp
 
 int decide_split(int B, int V) {
   const int nrt = residual_tiles(V);
-  int s = (2 * 148 + B - 1) / B;
+  int s = (4 * 148 + B - 1) / B;  // about four CTAs per SM over the whole grid
   if (s > kMaxSplit) s = kMaxSplit;
   if (s > nrt) s = nrt;
   return s < 1 ? 1 : s;
 }
 
-// Statistics of one row: raw max m, L = log2 sum 2^((l - m) c), first argmax.
+// Statistics of one row: raw max m, the exact shift M = fl(m * c_hi) and
+// L = log2 sum_v 2^(l_v*c - M), so log2 p(v) = l_v*c - (M + L); first argmax.
 struct RowStat {
-  double m, L;
+  double m, M, L;
   int amax;
   bool ok;
 };
 
 // Warp-cooperative combine of a row's tile partials.
-__device__ RowStat combine_row(const Partial* p, int ntiles, bool greedy, double cd, int lane) {
+__device__ RowStat combine_row(const Partial* p, int ntiles, bool greedy, const Scale& sc,
+                               int lane) {
   float mv = -INFINITY;
   int mi = INT_MAX;
   for (int t = lane; t < ntiles; t += 32) {
@@ -54,13 +56,15 @@ __device__ RowStat combine_row(const Partial* p, int ntiles, bool greedy, double
   RowStat r;
   r.m = mv;
   r.amax = mi;
+  r.M = 0.0;
   r.L = 0.0;
   r.ok = (mv > -INFINITY && mv < INFINITY);
   if (r.ok && !greedy) {
+    r.M = (double)__fmul_rn(mv, sc.hi);
     double s = 0.0;
     for (int t = lane; t < ntiles; t += 32) {
       const Partial q = p[t];
-      if (q.s != 0.0) s += q.s * exp2(((double)q.m - (double)mv) * cd);
+      if (q.s != 0.0) s += q.s * exp2((double)__fmul_rn(q.m, sc.hi) - r.M);
     }
     s = warp_sum_d(s);
     r.ok = (s > 0.0 && s < INFINITY);
@@ -99,23 +103,26 @@ __device__ __forceinline__ void load8<float>(const float* row, int e0, int V, fl
   }
 }
 
-// Probability of a logit under row statistics (m, L): 2^((x - m) c - L),
-// with c = chi + clo and L = Lhi + Llo.
+// Probability of a logit x of a row with log2-partition Lt = M + L:
+// 2^(x*c - Lt), c = chi + clo, Lt = Lhi + Llo; the product x*chi - Lhi is
+// rounded once relative to the (small) result.
 struct ProbCoef {
-  float m, chi, clo, Lhi, Llo;
+  float chi, clo, nLhi, nLlo;
 };
-__device__ __forceinline__ ProbCoef make_coef(const RowStat& r, const Scale& s) {
+__device__ __forceinline__ ProbCoef make_coef(double Lt, const Scale& s) {
   ProbCoef k;
-  k.m = (float)r.m;  // exact: r.m is a float logit
   k.chi = s.hi;
   k.clo = s.lo;
-  k.Lhi = (float)r.L;
-  k.Llo = (float)(r.L - (double)k.Lhi);
+  const float hi = (float)Lt;
+  k.nLhi = -hi;
+  k.nLlo = -(float)(Lt - (double)hi);
   return k;
 }
-__device__ __forceinline__ float prob(float x, const ProbCoef& k) {
-  const float d = x - k.m;
-  return ex2(fmaf(d, k.chi, fmaf(d, k.clo, -k.Llo)) - k.Lhi);
+__device__ __forceinline__ float2 prob2(float2 x, const ProbCoef& k) {
+  float2 t = __ffma2_rn(x, make_float2(k.chi, k.chi), make_float2(k.nLhi, k.nLhi));
+  t = __ffma2_rn(x, make_float2(k.clo, k.clo), t);
+  t = __fadd2_rn(t, make_float2(k.nLlo, k.nLlo));
+  return make_float2(ex2(t.x), ex2(t.y));
 }
 
 // Weights w = max(0, p - q) (or p when there is no draft row) of 8 elements.
@@ -128,17 +135,28 @@ __device__ __forceinline__ void weights8(const T* prow, const T* qrow, int e0, i
     float xq[8];
     load8<T>(qrow, e0, V, xq);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = fmaxf(prob(xp[e], kp) - prob(xq[e], kq), 0.0f);
+    for (int e = 0; e < 8; e += 2) {
+      const float2 p = prob2(make_float2(xp[e], xp[e + 1]), kp);
+      const float2 q = prob2(make_float2(xq[e], xq[e + 1]), kq);
+      w[e] = fmaxf(p.x - q.x, 0.0f);
+      w[e + 1] = fmaxf(p.y - q.y, 0.0f);
+    }
   } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = prob(xp[e], kp);
+    for (int e = 0; e < 8; e += 2) {
+      const float2 p = prob2(make_float2(xp[e], xp[e + 1]), kp);
+      w[e] = p.x;
+      w[e + 1] = p.y;
+    }
   }
 }
+// A lane's 8 weights summed pairwise in fp32 (error ~ 3 ulp of the small
+// sum), then widened; tiles and lanes combine in fp64.
 __device__ __forceinline__ double lane_sum8(const float w[8]) {
-  double s = 0.0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) s += (double)w[e];
-  return s;
+  const float2 a = __fadd2_rn(make_float2(w[0], w[1]), make_float2(w[2], w[3]));
+  const float2 b = __fadd2_rn(make_float2(w[4], w[5]), make_float2(w[6], w[7]));
+  const float2 c = __fadd2_rn(a, b);
+  return (double)(c.x + c.y);
 }
 
 // Tile sums of the weights over residual tiles [t0, t1) (one CTA's share).
@@ -177,13 +195,16 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
   __shared__ double s_Z;
   __shared__ int s_tile, s_tok;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double* sh_sum = sh_pre + nrt;  // second half of the dynamic buffer
+  for (int t = threadIdx.x; t < nrt; t += blockDim.x) sh_sum[t] = __ldcg(tsum_g + t);
+  __syncthreads();
   // Exclusive prefix over tiles in a fixed order (warp 0: each lane owns a
   // contiguous run of tiles).
   if (warp == 0) {
     const int per = (nrt + 31) / 32;
     const int a = min(nrt, lane * per), b = min(nrt, a + per);
     double run = 0.0;
-    for (int t = a; t < b; ++t) run += __ldcg(tsum_g + t);
+    for (int t = a; t < b; ++t) run += sh_sum[t];
     double incl = run;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -194,7 +215,7 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
     if (lane == 0) c = 0.0;
     for (int t = a; t < b; ++t) {
       sh_pre[t] = c;
-      c += __ldcg(tsum_g + t);
+      c += sh_sum[t];
     }
     if (lane == 31) s_Z = incl;
     if (lane == 0) s_tile = -1;
@@ -206,7 +227,7 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
   const double target = (double)u * Z;
   // The last tile with mass whose prefix does not exceed the target.
   for (int t = threadIdx.x; t < nrt; t += blockDim.x)
-    if (sh_pre[t] <= target && __ldcg(tsum_g + t) > 0.0) atomicMax(&s_tile, t);
+    if (sh_pre[t] <= target && sh_sum[t] > 0.0) atomicMax(&s_tile, t);
   __syncthreads();
   const int tile = s_tile < 0 ? 0 : s_tile;  // s_tile >= 0 whenever Z > 0
   if (warp == 0) {
@@ -285,7 +306,7 @@ __device__ bool draw_token(const DecideCommon& c, int b, int sp, const T* prow, 
 // Shared per-sequence state
 // ---------------------------------------------------------------------------
 struct SeqShared {
-  double m[kMaxRows], L[kMaxRows];
+  double m[kMaxRows], M[kMaxRows], L[kMaxRows];
   int amax[kMaxRows];
   int ok[kMaxRows];
   int a, bad, last, tok;
@@ -294,15 +315,21 @@ struct SeqShared {
 
 // Combine all rows of a sequence into shared memory (warp per row).
 __device__ void combine_rows(SeqShared& sh, const Partial* part, int row0, int nrows_seq,
-                             int ntiles, const bool* want, bool greedy, double cd) {
+                             int ntiles, const bool* want, bool greedy, const Scale& sc) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int r = warp; r < nrows_seq; r += kWarps) {
     if (!want[r]) {
-      if (lane == 0) { sh.ok[r] = 1; sh.m[r] = 0; sh.L[r] = 0; sh.amax[r] = -1; }
+      if (lane == 0) { sh.ok[r] = 1; sh.m[r] = 0; sh.M[r] = 0; sh.L[r] = 0; sh.amax[r] = -1; }
       continue;
     }
-    const RowStat s = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, cd, lane);
-    if (lane == 0) { sh.m[r] = s.m; sh.L[r] = s.L; sh.amax[r] = s.amax; sh.ok[r] = s.ok; }
+    const RowStat s = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, sc, lane);
+    if (lane == 0) {
+      sh.m[r] = s.m;
+      sh.M[r] = s.M;
+      sh.L[r] = s.L;
+      sh.amax[r] = s.amax;
+      sh.ok[r] = s.ok;
+    }
   }
 }
 
@@ -312,13 +339,14 @@ __device__ __forceinline__ const T* row_ptr(const unsigned char* base, long long
   return reinterpret_cast<const T*>(base + row * ld_bytes);
 }
 
-// One speculative check on n positions. Target row j: tp(j) with stats sh[tr(j)];
-// draft law of position j: stats (dm(j), dL(j)) and row dp(j). Returns a in
-// warp 0 via sh.a; sh.bad set if a draft id is out of range.
+// One speculative check on n positions. Target row j: tp(j) with log2
+// partition sh.M + sh.L at index tr0 + j; draft law of position j: row dp(j)
+// with log2 partition dlt(j). Returns a via sh.a (warp 0); sh.bad is set if a
+// draft id is out of range.
 template <typename T, typename TP, typename DP, typename DS>
 __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const DecideCommon& c,
-                            int b, float Tb, bool greedy, double cd, const int32_t* drafts,
-                            TP tp, DP dp, DS dstat, int tr0, double* diag_p, double* diag_q) {
+                            int b, bool greedy, double cd, const int32_t* drafts, TP tp, DP dp,
+                            DS dstat, int tr0, double* diag_p, double* diag_q) {
   const int lane = threadIdx.x & 31;
   int a = n, bad = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
@@ -331,10 +359,8 @@ __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const Dec
       } else if (greedy) {
         acc = (x == sh.amax[tr0 + j]);
       } else {
-        const double lp = ((double)load_elem(tp(j) + x) - sh.m[tr0 + j]) * cd - sh.L[tr0 + j];
-        double dm, dL;
-        dstat(j, dm, dL);
-        const double lq = ((double)load_elem(dp(j) + x) - dm) * cd - dL;
+        const double lp = (double)load_elem(tp(j) + x) * cd - (sh.M[tr0 + j] + sh.L[tr0 + j]);
+        const double lq = (double)load_elem(dp(j) + x) * cd - dstat(j);
         const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(pos0 + j),
                                       (uint32_t)stage).x;
         acc = (double)u < exp2(lp - lq);
@@ -380,17 +406,17 @@ __global__ void __launch_bounds__(kDecideThreads)
   };
   if (!tvalid) { if (sp == 0) fail(); return; }
 
-  combine_rows(sh, c.part, b * per, per, c.ntiles, want, greedy, cd);
+  combine_rows(sh, c.part, b * per, per, c.ntiles, want, greedy, sc);
   __syncthreads();
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   const unsigned char* tgt = A.tgt;
   const unsigned char* drf = A.drf;
   auto tp = [&](int j) { return row_ptr<T>(tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
   auto dp = [&](int j) { return row_ptr<T>(drf, A.ld_drf, (long long)b * K + j); };
-  auto ds = [&](int j, double& m, double& L) { m = sh.m[K + 1 + j]; L = sh.L[K + 1 + j]; };
+  auto ds = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
   if (threadIdx.x < 32) {
     const bool dg = diag && sp == 0 && !greedy;
-    accept_scan<T>(sh, K, 0, 1, c, b, Tb, greedy, cd, drafts, tp, dp, ds, 0,
+    accept_scan<T>(sh, K, 0, 1, c, b, greedy, cd, drafts, tp, dp, ds, 0,
                    dg ? diag + 2 * K + 1 : nullptr, dg ? diag + 3 * K + 1 : nullptr);
   }
   __syncthreads();
@@ -406,9 +432,8 @@ __global__ void __launch_bounds__(kDecideThreads)
   } else {
     const T* prow = tp(a);
     const T* qrow = a < K ? dp(a) : nullptr;
-    RowStat rp{sh.m[a], sh.L[a], 0, true};
-    RowStat rq{a < K ? sh.m[K + 1 + a] : 0.0, a < K ? sh.L[K + 1 + a] : 0.0, 0, true};
-    const ProbCoef kp = make_coef(rp, sc), kq = make_coef(rq, sc);
+    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sc);
+    const ProbCoef kq = make_coef(a < K ? ds(a) : 0.0, sc);
     const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 1u).y;
     if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
   }
@@ -419,7 +444,7 @@ __global__ void __launch_bounds__(kDecideThreads)
   if (diag) {
     for (int j = threadIdx.x; j < per; j += blockDim.x)
       diag[j] = greedy ? __longlong_as_double(0x7ff8000000000000ll)
-                       : (sh.m[j] * cd + sh.L[j]) * kLn2;
+                       : (sh.M[j] + sh.L[j]) * kLn2;
     if (greedy)
       for (int j = threadIdx.x; j < 2 * K; j += blockDim.x)
         diag[per + j] = __longlong_as_double(0x7ff8000000000000ll);
@@ -429,17 +454,19 @@ __global__ void __launch_bounds__(kDecideThreads)
 
 cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st) {
   const int nrt = residual_tiles(a.c.V);
-  const size_t smem = (size_t)nrt * sizeof(double);
+  const size_t smem = 2 * (size_t)nrt * sizeof(double);
   dim3 grid(a.c.nsplit, a.c.B);
   if (a.c.dtype == SPEC_BF16) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(chain_decide_kernel<__nv_bfloat16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(chain_decide_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return cudaGetLastError();
     chain_decide_kernel<__nv_bfloat16><<<grid, kDecideThreads, smem, st>>>(a);
   } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(chain_decide_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(chain_decide_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return cudaGetLastError();
     chain_decide_kernel<float><<<grid, kDecideThreads, smem, st>>>(a);
   }
   return cudaGetLastError();
@@ -490,16 +517,16 @@ __global__ void __launch_bounds__(kDecideThreads)
   for (int r = threadIdx.x; r < per; r += blockDim.x) want[r] = (r <= K) || !greedy;
   __syncthreads();
 
-  combine_rows(sh, c.part, b * per, per, c.ntiles, want, greedy, cd);
+  combine_rows(sh, c.part, b * per, per, c.ntiles, want, greedy, sc);
   __syncthreads();
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   const long long row0 = (long long)b * S + w;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, row0 + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_d, A.ld, row0 + j); };
-  auto ds = [&](int j, double& m, double& L) { m = sh.m[K + 1 + j]; L = sh.L[K + 1 + j]; };
+  auto ds = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
   if (threadIdx.x < 32) {
     const bool dg = diag && sp == 0 && !greedy;
-    accept_scan<T>(sh, K, w, 1, c, b, Tb, greedy, cd, drafts, tp, dp, ds, 0,
+    accept_scan<T>(sh, K, w, 1, c, b, greedy, cd, drafts, tp, dp, ds, 0,
                    dg ? diag + 2 * K + 1 : nullptr, dg ? diag + 3 * K + 1 : nullptr);
   }
   __syncthreads();
@@ -517,9 +544,8 @@ __global__ void __launch_bounds__(kDecideThreads)
   } else {
     const T* prow = tp(a);
     const T* qrow = a < K ? dp(a) : nullptr;
-    RowStat rp{sh.m[a], sh.L[a], 0, true};
-    RowStat rq{a < K ? sh.m[K + 1 + a] : 0.0, a < K ? sh.L[K + 1 + a] : 0.0, 0, true};
-    const ProbCoef kp = make_coef(rp, sc), kq = make_coef(rq, sc);
+    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sc);
+    const ProbCoef kq = make_coef(a < K ? ds(a) : 0.0, sc);
     const float u =
         spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(w + a), 1u).y;
     if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
@@ -529,7 +555,8 @@ __global__ void __launch_bounds__(kDecideThreads)
     const size_t slot = (size_t)b * WC + w + j;
     A.win_tok[slot] = j < a ? drafts[j] : tok;
     A.win_stat[2 * slot] = greedy ? __longlong_as_double(kNaNBits) : sh.m[j];
-    A.win_stat[2 * slot + 1] = greedy ? __longlong_as_double(kNaNBits) : sh.L[j] * kLn2;
+    A.win_stat[2 * slot + 1] =
+        greedy ? __longlong_as_double(kNaNBits) : (sh.M[j] + sh.L[j] - sh.m[j] * cd) * kLn2;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -537,7 +564,7 @@ __global__ void __launch_bounds__(kDecideThreads)
     A.acc1[b] = a;
   }
   if (diag && !greedy) {
-    for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.m[j] * cd + sh.L[j]) * kLn2;
+    for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
     if (threadIdx.x == 0) diag[4 * K + 1] = Z;
   }
 }
@@ -567,16 +594,16 @@ __global__ void __launch_bounds__(kDecideThreads)
   for (int r = threadIdx.x; r < S; r += blockDim.x) want[r] = (r <= W);
   __syncthreads();
 
-  combine_rows(sh, c.part, b * S, W + 1, c.ntiles, want, greedy, cd);
+  combine_rows(sh, c.part, b * S, W + 1, c.ntiles, want, greedy, sc);
   __syncthreads();
   const int32_t* wtok = A.win_tok + (size_t)b * WC;
   const double* wst = A.win_stat + (size_t)b * WC * 2;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_f, A.ld, (long long)b * S + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, (long long)b * S + j); };
-  auto ds = [&](int j, double& m, double& L) { m = wst[2 * j]; L = wst[2 * j + 1] * kLog2e; };
+  auto ds = [&](int j) { return wst[2 * j] * cd + wst[2 * j + 1] * kLog2e; };
   if (threadIdx.x < 32) {
     const bool dg = diag && sp == 0 && !greedy;
-    accept_scan<T>(sh, W, 0, 2, c, b, Tb, greedy, cd, wtok, tp, dp, ds, 0,
+    accept_scan<T>(sh, W, 0, 2, c, b, greedy, cd, wtok, tp, dp, ds, 0,
                    dg ? diag + S : nullptr, dg ? diag + 2 * S - 1 : nullptr);
   }
   __syncthreads();
@@ -594,11 +621,8 @@ __global__ void __launch_bounds__(kDecideThreads)
   } else {
     const T* prow = tp(a);
     const T* qrow = a < W ? dp(a) : nullptr;
-    double qm = 0.0, qL = 0.0;
-    if (a < W) ds(a, qm, qL);
-    RowStat rp{sh.m[a], sh.L[a], 0, true};
-    RowStat rq{qm, qL, 0, true};
-    const ProbCoef kp = make_coef(rp, sc), kq = make_coef(rq, sc);
+    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sc);
+    const ProbCoef kq = make_coef(a < W ? ds(a) : 0.0, sc);
     const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 2u).y;
     if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
   }
@@ -611,7 +635,7 @@ __global__ void __launch_bounds__(kDecideThreads)
     A.win_len[b] = 0;
   }
   if (diag && !greedy) {
-    for (int j = threadIdx.x; j <= W; j += blockDim.x) diag[j] = (sh.m[j] * cd + sh.L[j]) * kLn2;
+    for (int j = threadIdx.x; j <= W; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
     if (threadIdx.x == 0) diag[3 * S - 2] = Z;
   }
 }
@@ -620,24 +644,28 @@ template <typename K1, typename K2>
 static cudaError_t launch_decide(K1 kb, K2 kf, int dtype, dim3 grid, size_t smem,
                                  const HierDecideArgs& a, cudaStream_t st) {
   if (dtype == SPEC_BF16) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+      return cudaGetLastError();
     kb<<<grid, kDecideThreads, smem, st>>>(a);
   } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+      return cudaGetLastError();
     kf<<<grid, kDecideThreads, smem, st>>>(a);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)residual_tiles(a.c.V) * sizeof(double);
+  const size_t smem = 2 * (size_t)residual_tiles(a.c.V) * sizeof(double);
   return launch_decide(hier1_decide_kernel<__nv_bfloat16>, hier1_decide_kernel<float>, a.c.dtype,
                        dim3(a.c.nsplit, a.c.B), smem, a, st);
 }
 cudaError_t launch_hier2_decide(const HierDecideArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)residual_tiles(a.c.V) * sizeof(double);
+  const size_t smem = 2 * (size_t)residual_tiles(a.c.V) * sizeof(double);
   return launch_decide(hier2_decide_kernel<__nv_bfloat16>, hier2_decide_kernel<float>, a.c.dtype,
                        dim3(a.c.nsplit, a.c.B), smem, a, st);
 }

@@ -8,22 +8,15 @@ namespace specv {
 // A logit row as the row-statistics kernel sees it.
 struct RowRef {
   const unsigned char* ptr;  // first element of the row
-  float chi, clo;            // temperature scale (valid when !greedy)
-  bool valid;                // statistics wanted
-  bool greedy;               // argmax only (temperature 0)
+  float T;                   // temperature of its sequence
+  bool valid;                // statistics wanted (and temperature valid)
 };
 
 __device__ __forceinline__ RowRef make_row(const unsigned char* ptr, float T, bool want) {
   RowRef r;
   r.ptr = ptr;
+  r.T = T;
   r.valid = want && temp_valid(T);
-  r.greedy = (T == 0.0f);
-  r.chi = r.clo = 0.0f;
-  if (r.valid && !r.greedy) {
-    const Scale s = make_scale(T);
-    r.chi = s.hi;
-    r.clo = s.lo;
-  }
   return r;
 }
 
@@ -37,7 +30,7 @@ struct ChainRows {
   int K;
   __device__ __forceinline__ RowRef get(int r) const {
     const int per = 2 * K + 1, b = r / per, j = r - b * per;
-    const float T = temperature[b];
+    const float T = __ldg(temperature + b);
     if (j <= K) return make_row(tgt + ((long long)b * (K + 1) + j) * ld_tgt, T, true);
     return make_row(drf + ((long long)b * K + (j - K - 1)) * ld_drf, T, T != 0.0f);
   }
@@ -54,7 +47,7 @@ struct Hier1Rows {
   int K, S, Ni;
   __device__ __forceinline__ RowRef get(int r) const {
     const int per = 2 * K + 1, b = r / per, j = r - b * per;
-    const float T = temperature[b];
+    const float T = __ldg(temperature + b);
     const int w = win_len[b];
     const bool ok = (w >= 0 && w < Ni);
     if (j <= K)
@@ -77,7 +70,7 @@ struct Hier2Rows {
     const int b = r / S, s = r - b * S;
     const int W = win_len[b];
     const bool fire = acc1[b] >= 0 && W >= Ni && W < S && s <= W;
-    return make_row(lg_f + (long long)r * ld, temperature[b], fire);
+    return make_row(lg_f + (long long)r * ld, __ldg(temperature + b), fire);
   }
 };
 

@@ -46,25 +46,60 @@ __device__ __forceinline__ float vec_elem(uint4 w, int e, float*) {
   return __uint_as_float(word);
 }
 
-// sum_e 2^((x_e - m) * c) over one vector; pairwise inside the vector.
-__device__ __forceinline__ float term(float x, float m, float chi, float clo) {
+// Sum over one 16-byte vector of 2^(x*c - M) with c = chi + clo and M an
+// exact fp32 shift: two packed FP32x2 FMAs per element pair form the
+// exponent (the product x*chi - M is rounded once, relative to the small
+// result), one MUFU ex2 per element, packed adds pairwise inside the vector.
+__device__ __forceinline__ float2 expo2(float2 x, float2 chi, float2 clo, float2 nM) {
+  return __ffma2_rn(x, clo, __ffma2_rn(x, chi, nM));
+}
+__device__ __forceinline__ float2 ex2x2(float2 a) { return make_float2(ex2(a.x), ex2(a.y)); }
+
+__device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, float2 nM,
+                                             __nv_bfloat16*) {
+  const float2 e0 = ex2x2(expo2(make_float2(bf_lo(w.x), bf_hi(w.x)), chi, clo, nM));
+  const float2 e1 = ex2x2(expo2(make_float2(bf_lo(w.y), bf_hi(w.y)), chi, clo, nM));
+  const float2 e2 = ex2x2(expo2(make_float2(bf_lo(w.z), bf_hi(w.z)), chi, clo, nM));
+  const float2 e3 = ex2x2(expo2(make_float2(bf_lo(w.w), bf_hi(w.w)), chi, clo, nM));
+  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
+}
+__device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, float2 nM, float*) {
+  const float2 e0 =
+      ex2x2(expo2(make_float2(__uint_as_float(w.x), __uint_as_float(w.y)), chi, clo, nM));
+  const float2 e1 =
+      ex2x2(expo2(make_float2(__uint_as_float(w.z), __uint_as_float(w.w)), chi, clo, nM));
+  return __fadd2_rn(e0, e1);
+}
+// Scalar form of one term (tail elements).
+__device__ __forceinline__ float term(float x, float chi, float clo, float nM) {
+  return ex2(fmaf(x, clo, fmaf(x, chi, nM)));
+}
+
+// Slow form for |M| >= 2^26, where 2^(m*c - M) itself could overflow:
+// x*c - M = (x - m)*c + (m*chi - M) + m*clo with the product residual exact.
+__device__ __forceinline__ float term_far(float x, float m, float chi, float clo, float rr) {
   const float d = x - m;
-  return ex2(fmaf(d, chi, d * clo));
+  return ex2(fmaf(d, chi, fmaf(d, clo, rr)));
 }
-__device__ __forceinline__ float vec_expsum(uint4 w, float m, float chi, float clo,
-                                            __nv_bfloat16*) {
-  const float e0 = term(bf_lo(w.x), m, chi, clo), e1 = term(bf_hi(w.x), m, chi, clo);
-  const float e2 = term(bf_lo(w.y), m, chi, clo), e3 = term(bf_hi(w.y), m, chi, clo);
-  const float e4 = term(bf_lo(w.z), m, chi, clo), e5 = term(bf_hi(w.z), m, chi, clo);
-  const float e6 = term(bf_lo(w.w), m, chi, clo), e7 = term(bf_hi(w.w), m, chi, clo);
-  return ((e0 + e1) + (e2 + e3)) + ((e4 + e5) + (e6 + e7));
+template <typename T>
+__device__ __forceinline__ float vec_expsum_far(uint4 w, float m, float chi, float clo, float rr);
+template <>
+__device__ __forceinline__ float vec_expsum_far<__nv_bfloat16>(uint4 w, float m, float chi,
+                                                              float clo, float rr) {
+  float s = 0.0f;
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    s += term_far(bf_lo(ws[q]), m, chi, clo, rr) + term_far(bf_hi(ws[q]), m, chi, clo, rr);
+  return s;
 }
-__device__ __forceinline__ float vec_expsum(uint4 w, float m, float chi, float clo, float*) {
-  const float e0 = term(__uint_as_float(w.x), m, chi, clo);
-  const float e1 = term(__uint_as_float(w.y), m, chi, clo);
-  const float e2 = term(__uint_as_float(w.z), m, chi, clo);
-  const float e3 = term(__uint_as_float(w.w), m, chi, clo);
-  return (e0 + e1) + (e2 + e3);
+template <>
+__device__ __forceinline__ float vec_expsum_far<float>(uint4 w, float m, float chi, float clo,
+                                                      float rr) {
+  return (term_far(__uint_as_float(w.x), m, chi, clo, rr) +
+          term_far(__uint_as_float(w.y), m, chi, clo, rr)) +
+         (term_far(__uint_as_float(w.z), m, chi, clo, rr) +
+          term_far(__uint_as_float(w.w), m, chi, clo, rr));
 }
 
 template <typename T, typename Rows>
@@ -91,38 +126,47 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   __syncwarp();
 
   const int ntiles = (V + kEpt - 1) / kEpt;
-  const long long nitems = (long long)nrows * ntiles;
-  const long long gw = (long long)blockIdx.x * kRsWarps + warp;
-  const long long nw = (long long)gridDim.x * kRsWarps;
+  const int gw = blockIdx.x * kRsWarps + warp;
+  const int nw = gridDim.x * kRsWarps;
+  const int dr = nw / ntiles, dt = nw - dr * ntiles;
 
-  auto next_valid = [&](long long it) -> long long {
-    for (; it < nitems; it += nw)
-      if (rows.get((int)(it / ntiles)).valid) return it;
-    return nitems;
+  // Item cursors (row, tile) advanced by nw items at a time, skipping rows
+  // that need no statistics.
+  struct Cursor {
+    int r, t;
   };
-  auto issue = [&](int s, long long it) {
-    const int r = (int)(it / ntiles), t = (int)(it - (long long)r * ntiles);
-    const RowRef ref = rows.get(r);
-    const int nel = min(kEpt, V - t * kEpt);
+  auto advance = [&](Cursor& c) {
+    c.t += dt;
+    c.r += dr;
+    if (c.t >= ntiles) { c.t -= ntiles; ++c.r; }
+  };
+  auto settle = [&](Cursor& c) {
+    while (c.r < nrows && !rows.get(c.r).valid) advance(c);
+  };
+  auto issue = [&](int s, const Cursor& c) {
+    const RowRef ref = rows.get(c.r);
+    const int nel = min(kEpt, V - c.t * kEpt);
     const uint32_t bytes = ((uint32_t)nel * sizeof(T)) & ~15u;
     mbar_arrive_expect_tx(&bars[s], bytes);
-    if (bytes) bulk_g2s(wbuf + s * kTileBytes, ref.ptr + (size_t)t * kTileBytes, bytes, &bars[s]);
+    if (bytes) bulk_g2s(wbuf + s * kTileBytes, ref.ptr + (size_t)c.t * kTileBytes, bytes, &bars[s]);
   };
 
-  long long prod = next_valid(gw);
+  Cursor prod{gw / ntiles, gw % ntiles};
+  settle(prod);
   int inflight = 0;
-  for (int s = 0; s < kRsStages && prod < nitems; ++s) {
+  for (int s = 0; s < kRsStages && prod.r < nrows; ++s) {
     if (lane == 0) issue(s, prod);
     ++inflight;
-    prod = next_valid(prod + nw);
+    advance(prod);
+    settle(prod);
   }
-  long long cons = next_valid(gw);
+  Cursor cons{gw / ntiles, gw % ntiles};
+  settle(cons);
   uint32_t phase = 0;
   bool timed_out = false;
-  int k = 0;
+  int s = 0;  // stage of the item being consumed
 
-  for (; cons < nitems; ++k) {
-    const int s = k & (kRsStages - 1);
+  for (; cons.r < nrows; s = (s + 1 == kRsStages) ? 0 : s + 1) {
     const bool ok = mbar_wait_bounded(&bars[s], (phase >> s) & 1u, kWaitLimitNs);
     if (__any_sync(0xffffffffu, !ok)) {
       timed_out = true;
@@ -131,8 +175,15 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     phase ^= 1u << s;
     --inflight;
 
-    const int r = (int)(cons / ntiles), t = (int)(cons - (long long)r * ntiles);
+    const int r = cons.r, t = cons.t;
     const RowRef ref = rows.get(r);
+    const bool greedy = (ref.T == 0.0f);
+    float chi = 0.0f, clo = 0.0f;
+    if (!greedy) {
+      const Scale sc = make_scale(ref.T);
+      chi = sc.hi;
+      clo = sc.lo;
+    }
     const int nel = min(kEpt, V - t * kEpt);
     const int nvec = (int)(((uint32_t)nel * sizeof(T)) >> 4);
     const int ntail = nel - nvec * kVec;
@@ -165,16 +216,31 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     warp_argmax(best, bidx);
 
     double ssum = 0.0;
-    if (!ref.greedy && best > -INFINITY && best < INFINITY) {
-      // Pass 2: sum of 2^((l - m) c) with m the tile maximum.
-      float acc = 0.0f;
+    if (!greedy && best > -INFINITY && best < INFINITY) {
+      // Pass 2: sum of 2^(l*c - M) with the exact fp32 shift M = fl(m*chi).
+      const float M = __fmul_rn(best, chi);
+      if (fabsf(M) < 67108864.0f) {  // 2^26: 2^(m*c - M) <= 2^2
+        const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
+        const float2 nM2 = make_float2(-M, -M);
+        float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int i = 0; i < kVpl; ++i) {
-        const int v = lane + 32 * i;
-        if (v < nvec) acc += vec_expsum(buf[v], best, ref.chi, ref.clo, (T*)nullptr);
+        for (int i = 0; i < kVpl; ++i) {
+          const int v = lane + 32 * i;
+          if (v < nvec) acc = __fadd2_rn(acc, vec_expsum(buf[v], chi2, clo2, nM2, (T*)nullptr));
+        }
+        float a = acc.x + acc.y;
+        if (lane < ntail) a += term(tailx, chi, clo, -M);
+        ssum = warp_sum_d((double)a);
+      } else {
+        const float rr = fmaf(best, chi, -M) + best * clo;
+        float a = 0.0f;
+        for (int i = 0; i < kVpl; ++i) {
+          const int v = lane + 32 * i;
+          if (v < nvec) a += vec_expsum_far<T>(buf[v], best, chi, clo, rr);
+        }
+        if (lane < ntail) a += term_far(tailx, best, chi, clo, rr);
+        ssum = warp_sum_d((double)a);
       }
-      if (lane < ntail) acc += term(tailx, best, ref.chi, ref.clo);
-      ssum = warp_sum_d((double)acc);
     }
     if (lane == 0) {
       Partial p;
@@ -186,24 +252,26 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
 
     // Every lane is done with stage s; refill it.
     __syncwarp();
-    if (prod < nitems) {
+    if (prod.r < nrows) {
       if (lane == 0) {
         fence_proxy_async_smem();
         issue(s, prod);
       }
       ++inflight;
-      prod = next_valid(prod + nw);
+      advance(prod);
+      settle(prod);
     }
-    cons = next_valid(cons + nw);
+    advance(cons);
+    settle(cons);
   }
 
   if (timed_out) {
     if (lane == 0) set_status(status, SPEC_ETIMEOUT);
     // Let copies still in flight land before the CTA's shared memory goes:
-    // stages k, k+1, ... hold the `inflight` copies not yet consumed.
+    // stages s, s+1, ... hold the `inflight` copies not yet consumed.
     for (int j = 0; j < inflight; ++j) {
-      const int s = (k + j) & (kRsStages - 1);
-      mbar_wait_bounded(&bars[s], (phase >> s) & 1u, kWaitLimitNs);
+      const int q = (s + j) % kRsStages;
+      mbar_wait_bounded(&bars[q], (phase >> q) & 1u, kWaitLimitNs);
     }
   }
 }
@@ -229,11 +297,15 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
   static bool smem_set = false;  // once per instantiation (same on every B200)
   if (!smem_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmem);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // do not leave the error pending for later calls
+      return e;
+    }
     smem_set = true;
   }
   constexpr int kEpt = kTileBytes / (int)sizeof(T);
   const long long items = (long long)nrows * ((V + kEpt - 1) / kEpt);
+  if (items >= (1LL << 31)) return cudaErrorInvalidValue;
   long long grid = rs_grid();
   const long long need = (items + kRsWarps - 1) / kRsWarps;
   if (grid > need) grid = need;

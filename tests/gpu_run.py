@@ -8,6 +8,19 @@ import torch
 from oracle.verify import verify_chain
 
 
+def padded(t):
+    """Copy of a [B, n, V] logits tensor whose rows start on 16-byte
+    boundaries (row stride rounded up), returned as the [B, n, V] view."""
+    B, n, V = t.shape
+    mult = 16 // t.element_size()
+    ld = (V + mult - 1) // mult * mult
+    if ld == V:
+        return t
+    big = torch.zeros((B, n, ld), dtype=t.dtype, device=t.device)
+    big[:, :, :V] = t
+    return big[:, :, :V]
+
+
 def to_np(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
@@ -15,8 +28,8 @@ def to_np(t):
 def run_chain_gpu(prob, diag=True, split=False):
     from speculative_decoding_verification_89_b200 import capi
     dev = torch.device("cuda")
-    tgt = prob.tgt.to(dev)
-    drf = prob.drf.to(dev)
+    tgt = padded(prob.tgt.to(dev))
+    drf = padded(prob.drf.to(dev))
     B, Kp1, V = tgt.shape
     K = Kp1 - 1
     dt = prob.draft_tok.to(dev).contiguous()

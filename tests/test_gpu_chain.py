@@ -119,6 +119,22 @@ def test_chain_invalid_values_flag_only_their_sequence():
         compare_check(f"seq{b}", ref[b], int(acc[b]), list(out[b, :acc[b] + 1]), tally)
 
 
+def test_chain_unaligned_rows_rejected_on_host():
+    """Rows that do not start on 16-byte boundaries are refused before any
+    launch (the row statistics stage them with bulk copies)."""
+    from speculative_decoding_verification_89_b200 import capi
+    prob = W.chain_problem(2, 2, 1001, torch.bfloat16, seed=1)
+    tgt, drf = prob.tgt.cuda(), prob.drf.cuda()   # row stride 2002 bytes
+    ws = capi.workspace(2, 2, 1001, torch.bfloat16)
+    acc = torch.empty(2, dtype=torch.int32, device="cuda")
+    out = torch.empty((2, 3), dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(capi.SpecError) as e:
+        capi.spec_verify_chain(tgt, drf, prob.draft_tok.cuda(), prob.temperature.cuda(), 0,
+                               prob.seq_id.cuda(), 0, acc, out, st, ws)
+    assert e.value.code == capi.SPEC_EINVAL
+
+
 def test_chain_padded_rows():
     B, K, V, ld = 3, 4, 3000, 3008
     base = W.chain_problem(B, K, ld, torch.bfloat16, seed=8, temperature=1.1)

@@ -106,9 +106,8 @@ def test_failures_leave_state_untouched():
     state = W.paged_state([5, 12, 3], 4, 4, 10)
     Kp1 = 5
     cases = [
-        (torch.tensor([5, 6, 3]), torch.tensor([5, 0, 4]), -1),    # keep > K+1
+        (torch.tensor([5, 6, 3]), torch.tensor([6, 0, 4]), -1),    # keep > K+1
         (torch.tensor([6, 6, 3]), torch.tensor([3, 0, 4]), -1),    # base beyond length
-        (torch.tensor([5, 12, 3]), torch.tensor([4, 4, 4]), -4),   # pool exhausted
     ]
     for base, keep, code in cases:
         gpu, status, _ = _gpu_commit(state, base.int(), keep.int(), 0, Kp1)
@@ -116,6 +115,14 @@ def test_failures_leave_state_untouched():
         assert torch.equal(gpu.tables, state.tables) and torch.equal(gpu.seq_lens, state.seq_lens)
         assert torch.equal(gpu.free_stack, state.free_stack)
         assert torch.equal(gpu.free_top, state.free_top)
+    # pool exhausted: two blocks needed, one free, nothing freed
+    tight = W.paged_state([5, 12, 3], 4, 4, 7)
+    gpu, status, _ = _gpu_commit(tight, torch.tensor([5, 12, 3]).int(),
+                                 torch.tensor([4, 0, 5]).int(), 0, Kp1)
+    assert status == -4
+    for a, b in ((gpu.tables, tight.tables), (gpu.seq_lens, tight.seq_lens),
+                 (gpu.free_stack, tight.free_stack), (gpu.free_top, tight.free_top)):
+        assert torch.equal(a, b)
     # a pending error blocks the commit entirely
     gpu, status, _ = _gpu_commit(state, None, torch.tensor([1, 1, 1], dtype=torch.int32), 0,
                                  Kp1, status=-6)

@@ -1,0 +1,272 @@
+"""Two-stage (L_d -> L_i -> L_f) verification on the GPU against the oracle,
+through the C ABI, plus the engine loop with paged commit / rollback and the
+block-table invariants every round."""
+import numpy as np
+import pytest
+import torch
+
+from oracle.commit import check_invariants, commit_paged
+from oracle.philox import PhiloxUniforms, STAGE_ONE, STAGE_TWO
+from oracle.verify import verify_hier_seq
+from speculative_decoding_verification_89_b200 import workloads as W
+from tests.gpu_run import padded
+from tests.parity import Tally, close, compare_check
+
+pytestmark = pytest.mark.gpu
+
+
+class HierRunner:
+    """Device state of the window and outputs for B sequences."""
+
+    def __init__(self, B, K, Ni, V, dtype, dev="cuda"):
+        from speculative_decoding_verification_89_b200 import capi
+        self.capi = capi
+        self.B, self.K, self.Ni, self.S = B, K, Ni, Ni + K + 1
+        WC = Ni + K
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.win_len = torch.zeros(B, **i32)
+        self.win_tok = torch.full((B, WC), -1, **i32)
+        self.win_stat = torch.zeros((B, WC, 2), dtype=torch.float64, device=dev)
+        self.acc1 = torch.empty(B, **i32)
+        self.acc2 = torch.empty(B, **i32)
+        self.ctok = torch.empty((B, WC + 1), **i32)
+        self.cn = torch.empty(B, **i32)
+        self.status = torch.zeros(1, **i32)
+        self.diag = torch.empty((B, 4 * K + 3 * self.S + 1), dtype=torch.float64, device=dev)
+        self.ws = capi.workspace(B, K, V, dtype, Ni=Ni, device=dev)
+
+    def step(self, lg_d, lg_i, lg_f, drafts, T, seed, seq_id, rnd):
+        lg_d, lg_i, lg_f = padded(lg_d), padded(lg_i), padded(lg_f)
+        self.capi.spec_verify_hier(lg_d, lg_i, lg_f, self.Ni, drafts, T, seed, seq_id, rnd,
+                                   self.win_len, self.win_tok, self.win_stat, self.acc1,
+                                   self.acc2, self.ctok, self.cn, self.status, self.ws,
+                                   diag=self.diag)
+
+    def host(self):
+        torch.cuda.synchronize()
+        return {k: getattr(self, k).cpu().numpy() for k in
+                ("win_len", "win_tok", "acc1", "acc2", "ctok", "cn", "diag")} | \
+               {"status": int(self.status.item())}
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _check_seq(tag, r, h, b, w, K, S, T, tally):
+    """Compare one sequence's round (oracle HierResult r, window length w
+    before the round) with the GPU state h. Returns the window the oracle
+    continues from, or None after an excused near-margin divergence (the
+    caller then follows the GPU)."""
+    a1 = int(h["acc1"][b])
+    # Stage-one output stays readable in win_tok[w .. w+a1] even when stage
+    # two has emptied the window (only win_len is reset).
+    toks1 = [int(x) for x in h["win_tok"][b, w:w + a1 + 1]]
+    if not compare_check(f"{tag}/s1", r.stage1, a1, toks1, tally):
+        return None
+    fired = int(h["acc2"][b]) >= 0
+    assert fired == (r.stage2 is not None), (tag, "stage two firing")
+    d = h["diag"][b]
+    if T > 0:
+        for j in range(K + 1):
+            assert close(d[j], r.stage1.lse_target[j], floor=1.0), (tag, "lse_i", j)
+        for j in range(K):
+            assert close(d[K + 1 + j], r.stage1.lse_draft[j], floor=1.0), (tag, "lse_d", j)
+            if r.stage1.p_draft_tok[j] > 1e-290:
+                assert close(d[2 * K + 1 + j], r.stage1.p_draft_tok[j]), (tag, "p_i", j)
+            if r.stage1.q_draft_tok[j] > 1e-290:
+                assert close(d[3 * K + 1 + j], r.stage1.q_draft_tok[j]), (tag, "q_d", j)
+        assert close(d[4 * K + 1], r.stage1.residual_mass), (tag, "Z1")
+    if not fired:
+        return list(r.window)
+    a2 = int(h["acc2"][b])
+    n = int(h["cn"][b])
+    if not compare_check(f"{tag}/s2", r.stage2, a2, [int(x) for x in h["ctok"][b, :n]], tally):
+        return None
+    assert int(h["win_len"][b]) == 0
+    if T > 0:
+        o = 4 * K + 2
+        for j, v in enumerate(r.stage2.lse_target):
+            assert close(d[o + j], v, floor=1.0), (tag, "lse_f", j)
+        for j, v in enumerate(r.stage2.p_draft_tok):
+            if v > 1e-290:
+                assert close(d[o + S + j], v), (tag, "p_f", j)
+        for j, v in enumerate(r.stage2.q_draft_tok):
+            if v > 1e-290:
+                assert close(d[o + 2 * S - 1 + j], v), (tag, "q_i", j)
+        assert close(d[o + 3 * S - 2], r.stage2.residual_mass), (tag, "Z2")
+    return []
+
+
+def _run_rounds(B, K, Ni, V, dtype, rounds, T, seed, make_logits, sample, tally, tag):
+    """Rounds of two-stage verification; rows for slots >= win_len are
+    redrawn every round, earlier slots kept (the call's contract)."""
+    dev = "cuda"
+    S = Ni + K + 1
+    runner = HierRunner(B, K, Ni, V, dtype)
+    seq_id = torch.arange(B, dtype=torch.int32, device=dev)
+    Td = T.to(dev)
+    lg = None
+    windows = {b: [] for b in sample}
+    for r in range(rounds):
+        fresh = make_logits(r)
+        if lg is None:
+            lg = [x.clone() for x in fresh]
+        else:
+            w = runner.win_len.view(B, 1, 1)
+            keep_old = torch.arange(S, device=dev).view(1, S, 1) < w
+            lg = [torch.where(keep_old, old, new) for old, new in zip(lg, fresh)]
+        w_before = runner.win_len.cpu()
+        drafts = W.window_drafts(lg[0], runner.win_len, K, Td, W.generator(seed + 7 * r, dev))
+        runner.step(lg[0], lg[1], lg[2], drafts, Td, seed, seq_id, r)
+        h = runner.host()
+        assert h["status"] == 0, h["status"]
+        host_rows = {b: [_np(x[b]) for x in lg] for b in sample}
+        dr = drafts.cpu().numpy()
+        for b in sample:
+            Tb = float(T[b])
+            res = verify_hier_seq(host_rows[b][0], host_rows[b][1], host_rows[b][2], dr[b], Tb,
+                                  windows[b], Ni, PhiloxUniforms(seed, b, r, STAGE_ONE),
+                                  PhiloxUniforms(seed, b, r, STAGE_TWO))
+            assert int(w_before[b]) == len(windows[b])
+            nxt = _check_seq(f"{tag}/r{r}/b{b}", res, h, b, int(w_before[b]), K, S, Tb, tally)
+            if nxt is None:   # excused near-margin divergence: follow the GPU
+                nxt = [int(x) for x in h["win_tok"][b, :int(h["win_len"][b])]]
+            windows[b] = nxt
+            assert int(h["win_len"][b]) == len(nxt)
+            assert [int(x) for x in h["win_tok"][b, :len(nxt)]] == nxt
+    return runner
+
+
+def test_hier_peaked_rounds():
+    """B=8, K=4, N_i=4, V=32000 bf16, peaked rows (+6 on 5 %), T=0.7 with
+    sequence 0 greedy, Philox seed 1; 24 rounds."""
+    base = W.hier_peaked()
+    B, K, Ni, V = 8, 4, 4, 32000
+    tally = Tally()
+
+    def make(r):
+        if r == 0:
+            return [base.lg_d.cuda(), base.lg_i.cuda(), base.lg_f.cuda()]
+        gen = W.generator(1000 + r, "cuda")
+        return list(W.hier_logits(B, 9, V, torch.bfloat16, gen, "cuda", final_std=2.5,
+                                  inter_noise=0.7, draft_noise=1.5, boost_p=0.05, boost=6.0))
+
+    _run_rounds(B, K, Ni, V, torch.bfloat16, 24, base.temperature, 1, make, range(B), tally,
+                "peaked")
+    tally.check_share()
+
+
+@pytest.mark.parametrize("K,Ni,V,dtype", [(1, 1, 300, torch.float32), (3, 2, 5000, torch.bfloat16),
+                                          (2, 5, 4099, torch.float32), (6, 3, 777, torch.bfloat16)])
+def test_hier_shapes(K, Ni, V, dtype):
+    B = 5
+    T = torch.tensor([1.0, 0.0, 0.6, 2.0, 0.9])
+    S = Ni + K + 1
+    tally = Tally()
+
+    def make(r):
+        gen = W.generator(77 + r, "cuda")
+        return list(W.hier_logits(B, S, V, dtype, gen, "cuda", final_std=2.0, inter_noise=0.6,
+                                  draft_noise=1.2))
+
+    _run_rounds(B, K, Ni, V, dtype, 10, T, 9, make, range(B), tally, f"K{K}N{Ni}V{V}")
+    tally.check_share()
+
+
+def test_hier_mixed_full_size():
+    """B=256, K=4, N_i=4, V=151936 fp32, T ~ U(0, 1.2] with 51 greedy
+    sequences, l_i = l_f + N(0, .5^2), l_d = l_f + N(0, 2^2), Philox seed 3;
+    3 rounds, oracle on 40 sampled sequences (greedy ones included)."""
+    prob = W.hier_mixed(device="cuda")
+    B, K, Ni, V = 256, 4, 4, 151936
+    T = prob.temperature.cpu()
+    greedy = [b for b in range(B) if float(T[b]) == 0.0][:8]
+    sample = sorted(set(list(range(0, B, 8)) + greedy))
+    tally = Tally()
+
+    def make(r):
+        if r == 0:
+            return [prob.lg_d, prob.lg_i, prob.lg_f]
+        gen = W.generator(3000 + r, "cuda")
+        return list(W.hier_logits(B, 9, V, torch.float32, gen, "cuda", final_std=2.0,
+                                  inter_noise=0.5, draft_noise=2.0))
+
+    _run_rounds(B, K, Ni, V, torch.float32, 3, prob.temperature, 3, make, sample, tally, "mixed")
+    tally.check_share()
+
+
+def test_engine_loop_with_paged_commit():
+    """64 sequences x 256 rounds, K = N_i = 4, V=32000 bf16, per-round logits
+    from a generator seeded by (4, round); each round reserves the cycle's
+    slots in the block tables, verifies, then commits the committed tokens
+    and rolls the reservation back (block 16, pool of 65536 blocks, start
+    lengths U[128, 2048]); invariants on every table every round, table
+    parity with the oracle every round, verification parity on 8 sampled
+    sequences."""
+    from speculative_decoding_verification_89_b200 import capi
+    B, K, Ni, V, rounds = 64, 4, 4, 32000, 256
+    S = Ni + K + 1
+    dev = "cuda"
+    ctx = W.context_lengths(B, 128, 2048, seed=4)
+    max_blocks = (max(ctx) + rounds * S + S) // 16 + 2
+    state = W.paged_state(ctx, 16, max_blocks, 65536, device=dev)
+    committed = state.seq_lens.clone()
+    T = torch.ones(B)
+    Td = T.to(dev)
+    sample = list(range(0, B, 8))
+    runner = HierRunner(B, K, Ni, V, torch.bfloat16)
+    seq_id = torch.arange(B, dtype=torch.int32, device=dev)
+    windows = {b: [] for b in sample}
+    tally = Tally()
+    lg = None
+    full = torch.full((B,), S, dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    for r in range(rounds):
+        (ld, li, lf), _ = W.engine_round_logits(B, S, V, r, dev)
+        if lg is None:
+            lg = [ld, li, lf]
+        else:
+            keep_old = torch.arange(S, device=dev).view(1, S, 1) < runner.win_len.view(B, 1, 1)
+            lg = [torch.where(keep_old, o, n) for o, n in zip(lg, (ld, li, lf))]
+        # Reserve the cycle's slots past the committed prefix.
+        capi.spec_commit_paged(state.tables, state.seq_lens, committed, full, 0,
+                               state.free_stack, state.free_top, S, st, block_size=16)
+        w_before = runner.win_len.cpu()
+        drafts = W.window_drafts(lg[0], runner.win_len, K, Td, W.generator(40 + r, dev))
+        runner.step(lg[0], lg[1], lg[2], drafts, Td, 4, seq_id, r)
+        h = runner.host()
+        assert h["status"] == 0
+        # Commit what stage two committed; roll the rest of the reservation back.
+        before = W.PagedState(state.tables.cpu(), state.seq_lens.cpu(),
+                              state.free_stack.cpu(), state.free_top.cpu(), 16)
+        capi.spec_commit_paged(state.tables, state.seq_lens, committed, runner.cn, 0,
+                               state.free_stack, state.free_top, S, st, block_size=16)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        ref = commit_paged(before.tables.numpy(), before.seq_lens.numpy(),
+                           committed.cpu().numpy(), h["cn"], before.free_stack.numpy(),
+                           int(before.free_top[0]), 16, 65536, S)
+        lens = state.seq_lens.cpu().numpy()
+        tabs = state.tables.cpu().numpy()
+        stack = state.free_stack.cpu().numpy()
+        top = int(state.free_top.cpu()[0])
+        assert list(lens) == list(ref.seq_lens) and top == ref.free_top
+        assert np.array_equal(stack[:top], ref.free_stack[:top])
+        for b in range(B):
+            nb = (int(lens[b]) + 15) // 16
+            assert np.array_equal(tabs[b, :nb], ref.tables[b, :nb])
+        assert check_invariants(tabs, lens, stack, top, 16, 65536) == []
+        assert list(lens) == list(committed.cpu().numpy() + h["cn"])
+        committed = state.seq_lens.clone()
+        host_rows = {b: [_np(x[b]) for x in lg] for b in sample}
+        dr = drafts.cpu().numpy()
+        for b in sample:
+            res = verify_hier_seq(host_rows[b][0], host_rows[b][1], host_rows[b][2], dr[b], 1.0,
+                                  windows[b], Ni, PhiloxUniforms(4, b, r, STAGE_ONE),
+                                  PhiloxUniforms(4, b, r, STAGE_TWO))
+            nxt = _check_seq(f"loop/r{r}/b{b}", res, h, b, int(w_before[b]), K, S, 1.0, tally)
+            if nxt is None:
+                nxt = [int(x) for x in h["win_tok"][b, :int(h["win_len"][b])]]
+            windows[b] = nxt
+    tally.check_share()

@@ -155,3 +155,17 @@ def test_empirical_acceptance_with_philox():
     mean = 1.0 - _tv(p, q)
     sd = np.sqrt(mean * (1 - mean) / n)
     assert abs(acc / n - mean) < 5 * sd
+
+
+def test_log_partition_is_logsumexp():
+    """The oracle's row log-partition equals scipy's logsumexp(l / T),
+    including rows with masked (-inf) entries and extreme temperatures."""
+    import scipy.special
+    from oracle.verify import log_partition
+    rng = np.random.default_rng(33)
+    for T in (1e-3, 0.7, 1.0, 50.0):
+        for _ in range(10):
+            l = rng.normal(0, 3, size=257)
+            l[rng.integers(0, 257, size=5)] = -np.inf
+            want = scipy.special.logsumexp(l / T)
+            assert abs(log_partition(l, T) - want) <= 1e-13 * max(1.0, abs(want))
