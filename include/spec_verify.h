@@ -47,7 +47,8 @@
  *   - Logit rows must start on 16-byte boundaries: the base pointers are
  *     16-byte aligned and the row stride times the element size is a
  *     multiple of 16 bytes. V itself may be any value >= 1.
- *   - Calls on different streams must use different workspaces.
+ *   - Calls on different streams must use different workspaces; calls that
+ *     share one workspace must not overlap on the GPU.
  */
 #ifndef SPEC_VERIFY_H
 #define SPEC_VERIFY_H
@@ -78,6 +79,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 /* Limits checked on the host. */
 #define SPEC_MAX_K 256           /* drafts per sequence per call      */
 #define SPEC_MAX_V (1 << 22)     /* vocabulary size                   */
+#define SPEC_MAX_COMMIT_B 32768  /* sequences per paged commit        */
 
 /* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
  * chain call, Ni > 0 a two-stage call. Returns 0 for invalid sizes. */
@@ -108,7 +110,10 @@ const char* spec_status_string(int status);
  *               Z of the final draw (sum max(0, p_a - q_a), or sum p_K for the
  *               bonus). NaN for greedy sequences.
  * ws, ws_bytes: workspace of at least spec_workspace_bytes(B, K, V, dtype, 0)
- *               bytes, 256-byte aligned. No initial contents are needed.
+ *               bytes, 256-byte aligned, zero-filled before its first use (it
+ *               holds self-resetting arrival counters that every completed
+ *               call leaves at zero; zero it again after a device error or
+ *               before using it for other sizes).
  * Equivalent to spec_chain_row_stats followed by spec_chain_decide.
  * ------------------------------------------------------------------------- */
 int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf,

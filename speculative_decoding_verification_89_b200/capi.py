@@ -107,11 +107,12 @@ def spec_status_string(code):
 
 
 def workspace(B, K, V, dtype, Ni=0, device="cuda"):
-    """A workspace tensor of the size a call needs (256-byte aligned)."""
+    """A zero-filled workspace tensor of the size a call needs (256-byte
+    aligned by the allocator)."""
     n = spec_workspace_bytes(B, K, V, dtype, Ni)
     if n == 0:
         raise ValueError("invalid sizes")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def spec_verify_chain(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,

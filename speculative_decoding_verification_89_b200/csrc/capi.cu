@@ -21,7 +21,8 @@ int stat_tiles(int V, int dtype) {
 }
 
 struct Layout {
-  size_t part, rsum, counters, total;
+  size_t part, fin, dec, rsum, counters, total;
+  long long rows;
 };
 
 // Workspace: tile partials for the largest row set, residual tile sums and
@@ -33,12 +34,14 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   const long long per = Ni > 0 ? (long long)std::max(2 * K + 1, Ni + K + 1) : 2LL * K + 1;
   const long long rows = (long long)B * per;
   if (rows * stat_tiles(V, dtype) >= (1LL << 31)) return false;  // 32-bit item indices
-  L->part = 0;
-  const size_t part_bytes = align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
-  L->rsum = part_bytes;
-  const size_t rsum_bytes = align_up((size_t)B * residual_tiles(V) * sizeof(double));
-  L->counters = L->rsum + rsum_bytes;
-  L->total = L->counters + align_up((size_t)std::max(B, 1) * sizeof(int));
+  // Counters first, so a workspace zeroed once keeps them zero across calls.
+  L->rows = rows;
+  L->counters = 0;
+  L->dec = align_up((size_t)std::max(B, 1) * sizeof(int));
+  L->fin = L->dec + align_up((size_t)std::max(B, 1) * sizeof(SeqDecision));
+  L->part = L->fin + align_up((size_t)rows * sizeof(RowFinal));
+  L->rsum = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
+  L->total = L->rsum + align_up((size_t)B * residual_tiles(V) * sizeof(double));
   return true;
 }
 
@@ -75,6 +78,14 @@ ChainCheck check_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t
   return c;
 }
 
+RsBuffers rs_buffers(void* ws, const Layout& L, int B) {
+  RsBuffers b;
+  b.part = reinterpret_cast<Partial*>((char*)ws + L.part);
+  b.seq_cnt = reinterpret_cast<int*>((char*)ws + L.counters);
+  b.nseq = B;
+  return b;
+}
+
 DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_tok,
                          const float* temperature, uint64_t seed, const int32_t* seq_id,
                          uint32_t round, double* diag, int32_t* dev_status, void* ws,
@@ -84,13 +95,15 @@ DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_to
   c.B = B;
   c.K = K;
   c.V = V;
-  c.ntiles = stat_tiles(V, dtype);
   c.draft_tok = draft_tok;
   c.temperature = temperature;
   c.seed = seed;
   c.seq_id = seq_id;
   c.round = round;
   c.part = reinterpret_cast<const Partial*>((char*)ws + L.part);
+  c.ntiles = stat_tiles(V, dtype);
+  c.fin = reinterpret_cast<RowFinal*>((char*)ws + L.fin);
+  c.dec = reinterpret_cast<SeqDecision*>((char*)ws + L.dec);
   c.rsum = reinterpret_cast<double*>((char*)ws + L.rsum);
   c.counters = reinterpret_cast<int*>((char*)ws + L.counters);
   c.nsplit = decide_split(B, V);
@@ -137,9 +150,7 @@ int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64
   rows.ld_drf = ld_drf * es;
   rows.temperature = temperature;
   rows.K = K;
-  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V,
-                                      reinterpret_cast<Partial*>((char*)ws + ck.L.part),
-                                      reinterpret_cast<int*>((char*)ws + ck.L.counters), B,
+  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, ck.L, B),
                                       dev_status, (cudaStream_t)stream));
 }
 
@@ -201,8 +212,7 @@ int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64
   const int es = elem_size(dtype);
   const int S = Ni + K + 1;
   cudaStream_t st = (cudaStream_t)stream;
-  Partial* part = reinterpret_cast<Partial*>((char*)ws + L.part);
-  int* counters = reinterpret_cast<int*>((char*)ws + L.counters);
+  const RsBuffers rsb = rs_buffers(ws, L, B);
 
   HierDecideArgs a;
   a.c = common_args(dtype, B, K, V, draft_tok, temperature, seed, seq_id, round, diag, dev_status,
@@ -230,7 +240,7 @@ int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64
   r1.K = K;
   r1.S = S;
   r1.Ni = Ni;
-  cudaError_t e = launch_row_stats(dtype, r1, B * (2 * K + 1), V, part, counters, B, dev_status, st);
+  cudaError_t e = launch_row_stats(dtype, r1, B * (2 * K + 1), V, rsb, dev_status, st);
   if (e == cudaSuccess) e = launch_hier1_decide(a, st);
   Hier2Rows r2;
   r2.lg_f = a.lg_f;
@@ -240,7 +250,7 @@ int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64
   r2.acc1 = acc1;
   r2.S = S;
   r2.Ni = Ni;
-  if (e == cudaSuccess) e = launch_row_stats(dtype, r2, B * S, V, part, counters, B, dev_status, st);
+  if (e == cudaSuccess) e = launch_row_stats(dtype, r2, B * S, V, rsb, dev_status, st);
   if (e == cudaSuccess) e = launch_hier2_decide(a, st);
   return cuda_status(e);
 }
@@ -251,7 +261,9 @@ int spec_commit_paged(int B, int block_size, int max_blocks, int32_t* block_tabl
                       const void* kv_stage, void* kv_pool, int layers, int kv_heads, int head_dim,
                       const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden,
                       int32_t* dev_status, void* stream) {
-  if (B < 0 || block_size < 1 || max_blocks < 0 || num_blocks < 0 || Kp1 < 0) return SPEC_EINVAL;
+  if (B < 0 || B > SPEC_MAX_COMMIT_B || block_size < 1 || max_blocks < 0 || num_blocks < 0 ||
+      Kp1 < 0)
+    return SPEC_EINVAL;
   if (B == 0) return SPEC_OK;
   if (!block_tables || !seq_lens || !keep || !free_stack || !free_top) return SPEC_EINVAL;
   if ((long long)B * Kp1 > (1LL << 31) - 1 || (long long)B * max_blocks > (1LL << 31) - 1)

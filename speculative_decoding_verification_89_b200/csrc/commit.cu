@@ -59,20 +59,34 @@ __device__ int block_excl_scan(int v, int* total) {
 }
 
 __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a) {
+  grid_dependency_wait();
+  extern __shared__ int s_nb[];  // [B] blocks covered before the commit
   __shared__ int s_bad, s_code;
   if (threadIdx.x == 0) { s_bad = 0; s_code = 0; }
   __syncthreads();
   if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;  // sticky error
   const int bs = a.block_size;
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) s_nb[b] = ceil_div(max(a.seq_lens[b], 0), bs);
+  __syncthreads();
   // Every covered table entry must be a valid block id: one coalesced pass
-  // over the flattened [B, max_blocks] table by the whole CTA.
+  // over the flattened [B, max_blocks] table, loads batched per thread.
   int bad = 0;
   const int nent = a.B * a.max_blocks;  // < 2^31, checked on the host
-  for (int e = threadIdx.x; e < nent; e += blockDim.x) {
-    const int b = e / a.max_blocks, i = e - b * a.max_blocks;
-    if (i < ceil_div(max(a.seq_lens[b], 0), bs)) {
-      const int x = a.tables[e];
-      if (x < 0 || x >= a.num_blocks) bad = 1;
+  constexpr int kBatch = 8;
+  for (int e0 = threadIdx.x; e0 < nent; e0 += kBatch * blockDim.x) {
+    int v[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int e = e0 + k * blockDim.x;
+      v[k] = e < nent ? a.tables[e] : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int e = e0 + k * blockDim.x;
+      if (e < nent) {
+        const int b = e / a.max_blocks, i = e - b * a.max_blocks;
+        if (i < s_nb[b] && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
+      }
     }
   }
   // Each thread owns a contiguous run of sequences.
@@ -154,57 +168,68 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
   }
 }
 
-// Copy of kept token rows: grid (B * Kp1, kCopyParts).
+// Copy of kept token rows: a grid-stride loop over (token, part) items; the
+// staged K/V segments of a token are split into kCopyParts parts.
 __global__ void __launch_bounds__(kCopyThreads) commit_copy_kernel(CommitArgs a) {
+  grid_dependency_wait();
   if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;
-  const int b = blockIdx.x / a.Kp1, i = blockIdx.x - b * a.Kp1, part = blockIdx.y;
-  const int kept = a.keep[b] + a.keep_add;
-  if (i >= kept) return;
-  const int pos = a.seq_lens[b] - kept + i;  // base_len + i
-  if (a.kv_stage) {
-    const int blk = a.tables[(size_t)b * a.max_blocks + pos / a.block_size];
-    const int slot = pos % a.block_size;
-    const int nseg = a.layers * 2;
-    const int segs_per = (nseg + kCopyParts - 1) / kCopyParts;
-    const int s0 = part * segs_per, s1 = min(nseg, s0 + segs_per);
-    const int vps = a.seg_bytes / 16;  // vectors per segment
-    const long long nvec = (long long)max(0, s1 - s0) * vps;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        a.kv_stage + (((size_t)b * a.Kp1 + i) * nseg + s0) * (size_t)a.seg_bytes);
-    for (long long v0 = threadIdx.x; v0 < nvec; v0 += (long long)blockDim.x * 4) {
-      uint4 r[4];
+  const int nitems = a.B * a.Kp1 * kCopyParts;
+  const int nseg = a.layers * 2;
+  const int segs_per = (nseg + kCopyParts - 1) / kCopyParts;
+  const int vps = a.seg_bytes / 16;  // vectors per segment
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int tok = item / kCopyParts, part = item - tok * kCopyParts;
+    const int b = tok / a.Kp1, i = tok - b * a.Kp1;
+    const int kept = a.keep[b] + a.keep_add;
+    if (i >= kept) continue;
+    const int pos = a.seq_lens[b] - kept + i;  // base_len + i
+    if (a.kv_stage) {
+      const int blk = a.tables[(size_t)b * a.max_blocks + pos / a.block_size];
+      const int slot = pos % a.block_size;
+      const int s0 = part * segs_per, s1 = min(nseg, s0 + segs_per);
+      const int nvec = max(0, s1 - s0) * vps;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.kv_stage + (((size_t)b * a.Kp1 + i) * nseg + s0) * (size_t)a.seg_bytes);
+      for (int v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * 4) {
+        uint4 r[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const long long v = v0 + (long long)u * blockDim.x;
-        if (v < nvec) r[u] = __ldcs(src + v);
-      }
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * blockDim.x;
+          if (v < nvec) r[u] = __ldcs(src + v);
+        }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const long long v = v0 + (long long)u * blockDim.x;
-        if (v < nvec) {
-          const int seg = s0 + (int)(v / vps), e = (int)(v - (long long)(seg - s0) * vps);
-          uint4* dst = reinterpret_cast<uint4*>(
-              a.kv_pool + (((size_t)blk * nseg + seg) * a.block_size + slot) * (size_t)a.seg_bytes);
-          __stcs(dst + e, r[u]);
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * blockDim.x;
+          if (v < nvec) {
+            const int seg = s0 + v / vps, e = v - (seg - s0) * vps;
+            uint4* dst = reinterpret_cast<uint4*>(
+                a.kv_pool + (((size_t)blk * nseg + seg) * a.block_size + slot) * (size_t)a.seg_bytes);
+            __stcs(dst + e, r[u]);
+          }
         }
       }
     }
-  }
-  if (a.hid_stage && part == 0) {
-    const int vps = a.hid_bytes / 16;
-    const uint4* src = reinterpret_cast<const uint4*>(a.hid_stage + ((size_t)b * a.Kp1 + i) * a.hid_bytes);
-    uint4* dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(a.hid_off[b] + i) * a.hid_bytes);
-    for (int v = threadIdx.x; v < vps; v += blockDim.x) __stcs(dst + v, __ldcs(src + v));
+    if (a.hid_stage && part == 0) {
+      const int hv = a.hid_bytes / 16;
+      const uint4* src =
+          reinterpret_cast<const uint4*>(a.hid_stage + ((size_t)b * a.Kp1 + i) * a.hid_bytes);
+      uint4* dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(a.hid_off[b] + i) * a.hid_bytes);
+      for (int v = threadIdx.x; v < hv; v += blockDim.x) __stcs(dst + v, __ldcs(src + v));
+    }
   }
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
-  commit_plan_kernel<<<1, kPlanThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  const size_t smem = (size_t)a.B * sizeof(int);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(commit_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return cudaGetLastError();
+  cudaError_t e = launch_pdl(commit_plan_kernel, dim3(1), dim3(kPlanThreads), smem, st, a);
   if (e != cudaSuccess) return e;
   if (a.B > 0 && a.Kp1 > 0 && (a.kv_stage || a.hid_stage)) {
-    commit_copy_kernel<<<dim3(a.B * a.Kp1, kCopyParts), kCopyThreads, 0, st>>>(a);
-    e = cudaGetLastError();
+    const int items = a.B * a.Kp1 * kCopyParts;
+    e = launch_pdl(commit_copy_kernel, dim3(min(items, 148 * 4)), dim3(kCopyThreads), 0, st, a);
   }
   return e;
 }

@@ -22,13 +22,16 @@ constexpr double kLn2 = 0.6931471805599453094172321214581766;
 // Row-statistics tiles: kTileBytes of one row, staged by one bulk copy into a
 // per-warp ring of kRsStages buffers; one CTA of kRsWarps warps per SM.
 #ifndef SPEC_RS_TILE
-#define SPEC_RS_TILE 8192
+#define SPEC_RS_TILE 4096
 #endif
 #ifndef SPEC_RS_WARPS
-#define SPEC_RS_WARPS 8
+#define SPEC_RS_WARPS 24
 #endif
 #ifndef SPEC_RS_STAGES
-#define SPEC_RS_STAGES 3
+#define SPEC_RS_STAGES 2
+#endif
+#ifndef SPEC_RS_PACKED
+#define SPEC_RS_PACKED 1  // packed FP32x2 FMAs in the exponent sums
 #endif
 constexpr int kTileBytes = SPEC_RS_TILE;
 constexpr int kRsWarps = SPEC_RS_WARPS;
@@ -49,6 +52,17 @@ struct Partial {
   float m;
   int idx;
   double s;
+};
+
+// Final statistics of one row, written by the warp that completes the row's
+// last tile: shift M = fl(m * c_hi) and L = log2 sum 2^(l*c - M) (so the
+// row's log2-partition is M + L), raw max m, first argmax (greedy rows), ok.
+struct RowFinal {
+  double M, L;
+  float m;
+  int amax;
+  int ok;
+  int pad;
 };
 
 template <typename T> struct Elem;
@@ -186,6 +200,37 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// ----------------------------------------------------------------------------
+// Programmatic dependent launch: every kernel of the library is launched with
+// programmatic stream serialization, waits for its stream predecessors before
+// touching memory (griddepcontrol.wait returns once they have completed and
+// their writes are visible) and lets its successor start launching early.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename Kern, typename... Args>
+static cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
+}
 
 // ----------------------------------------------------------------------------
 // Warp reductions

@@ -11,11 +11,14 @@
 // "Dynamische Verifizierungsrichtlinie" (N_i tentatively accepted tokens
 // before the final-layer check).
 //
-// Launch: grid (nsplit, B), 256 threads. Every CTA of a sequence repeats the
-// cheap combine + accept step; the residual row pair is split over the
-// nsplit CTAs, each writing tile sums of the weights; the last CTA to arrive
-// (atomic counter, no waiting) prefixes the tile sums, finds the tile holding
-// u' * Z, rescans that one tile and writes the outputs.
+// Two launches per check. (1) finish: one CTA per sequence combines the tile
+// partials of its rows (a warp per row), runs the accept test on all
+// positions (a lane per position, ballot for the first rejection) and, for
+// greedy sequences, writes the outputs. (2) draw: grid (nsplit, B); the
+// residual row pair of each sampled sequence is split over nsplit CTAs, each
+// writing tile sums of the weights; the last CTA to arrive (atomic counter,
+// no waiting) prefixes the tile sums, finds the tile holding u' * Z, rescans
+// that one tile and writes the outputs.
 #include <climits>
 
 #include "common.cuh"
@@ -29,48 +32,10 @@ constexpr int kUnroll = 4;  // residual tiles in flight per warp
 
 int decide_split(int B, int V) {
   const int nrt = residual_tiles(V);
-  int s = (4 * 148 + B - 1) / B;  // about four CTAs per SM over the whole grid
+  int s = (3 * 148) / (B > 0 ? B : 1);  // one wave of about three CTAs per SM
   if (s > kMaxSplit) s = kMaxSplit;
   if (s > nrt) s = nrt;
   return s < 1 ? 1 : s;
-}
-
-// Statistics of one row: raw max m, the exact shift M = fl(m * c_hi) and
-// L = log2 sum_v 2^(l_v*c - M), so log2 p(v) = l_v*c - (M + L); first argmax.
-struct RowStat {
-  double m, M, L;
-  int amax;
-  bool ok;
-};
-
-// Warp-cooperative combine of a row's tile partials.
-__device__ RowStat combine_row(const Partial* p, int ntiles, bool greedy, const Scale& sc,
-                               int lane) {
-  float mv = -INFINITY;
-  int mi = INT_MAX;
-  for (int t = lane; t < ntiles; t += 32) {
-    const Partial q = p[t];
-    if (q.m > mv || (q.m == mv && q.idx < mi)) { mv = q.m; mi = q.idx; }
-  }
-  warp_argmax(mv, mi);
-  RowStat r;
-  r.m = mv;
-  r.amax = mi;
-  r.M = 0.0;
-  r.L = 0.0;
-  r.ok = (mv > -INFINITY && mv < INFINITY);
-  if (r.ok && !greedy) {
-    r.M = (double)__fmul_rn(mv, sc.hi);
-    double s = 0.0;
-    for (int t = lane; t < ntiles; t += 32) {
-      const Partial q = p[t];
-      if (q.s != 0.0) s += q.s * exp2((double)__fmul_rn(q.m, sc.hi) - r.M);
-    }
-    s = warp_sum_d(s);
-    r.ok = (s > 0.0 && s < INFINITY);
-    r.L = log2(s);
-  }
-  return r;
 }
 
 // ---------------------------------------------------------------------------
@@ -303,32 +268,40 @@ __device__ bool draw_token(const DecideCommon& c, int b, int sp, const T* prow, 
 }
 
 // ---------------------------------------------------------------------------
-// Shared per-sequence state
+// Per-sequence state of the finish kernels
 // ---------------------------------------------------------------------------
+constexpr int kFinThreads = 512;
+constexpr int kFinWarps = kFinThreads / 32;
+constexpr long long kNaNBits = 0x7ff8000000000000ll;
+__device__ __forceinline__ double dnan() { return __longlong_as_double(kNaNBits); }
+
 struct SeqShared {
-  double m[kMaxRows], M[kMaxRows], L[kMaxRows];
+  double M[kMaxRows], L[kMaxRows];
+  float m[kMaxRows];
   int amax[kMaxRows];
   int ok[kMaxRows];
-  int a, bad, last, tok;
-  double Z;
+  int a, bad;
 };
 
-// Combine all rows of a sequence into shared memory (warp per row).
-__device__ void combine_rows(SeqShared& sh, const Partial* part, int row0, int nrows_seq,
-                             int ntiles, const bool* want, bool greedy, const Scale& sc) {
+// Combine the tile partials of the rows of one sequence (a warp per row) into
+// shared memory and into the RowFinal array (read later by the draw kernel).
+template <typename Want>
+__device__ void finish_rows(SeqShared& sh, const Partial* part, int ntiles, int row0, int nrows,
+                            Want want, bool greedy, float chi, RowFinal* fin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < nrows_seq; r += kWarps) {
-    if (!want[r]) {
-      if (lane == 0) { sh.ok[r] = 1; sh.m[r] = 0; sh.M[r] = 0; sh.L[r] = 0; sh.amax[r] = -1; }
+  for (int r = warp; r < nrows; r += kFinWarps) {
+    if (!want(r)) {
+      if (lane == 0) { sh.ok[r] = 1; sh.m[r] = 0.f; sh.M[r] = 0; sh.L[r] = 0; sh.amax[r] = -1; }
       continue;
     }
-    const RowStat s = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, sc, lane);
+    const RowFinal f = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, chi, lane);
     if (lane == 0) {
-      sh.m[r] = s.m;
-      sh.M[r] = s.M;
-      sh.L[r] = s.L;
-      sh.amax[r] = s.amax;
-      sh.ok[r] = s.ok;
+      fin[row0 + r] = f;
+      sh.m[r] = f.m;
+      sh.M[r] = f.M;
+      sh.L[r] = f.L;
+      sh.amax[r] = f.amax;
+      sh.ok[r] = f.ok;
     }
   }
 }
@@ -339,14 +312,14 @@ __device__ __forceinline__ const T* row_ptr(const unsigned char* base, long long
   return reinterpret_cast<const T*>(base + row * ld_bytes);
 }
 
-// One speculative check on n positions. Target row j: tp(j) with log2
-// partition sh.M + sh.L at index tr0 + j; draft law of position j: row dp(j)
-// with log2 partition dlt(j). Returns a via sh.a (warp 0); sh.bad is set if a
-// draft id is out of range.
+// One speculative check on n positions (warp 0). Target row j: tp(j) with log2
+// partition sh.M + sh.L at index j; draft law of position j: row dp(j) with
+// log2 partition dlt(j). Sets sh.a (first rejection, n if none) and sh.bad (a
+// draft id outside [0, V)). Writes p_j(x_j), q_j(x_j) to diag_p / diag_q.
 template <typename T, typename TP, typename DP, typename DS>
 __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const DecideCommon& c,
                             int b, bool greedy, double cd, const int32_t* drafts, TP tp, DP dp,
-                            DS dstat, int tr0, double* diag_p, double* diag_q) {
+                            DS dlt, double* diag_p, double* diag_q) {
   const int lane = threadIdx.x & 31;
   int a = n, bad = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
@@ -357,10 +330,10 @@ __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const Dec
       if (x < 0 || x >= c.V) {
         badj = true;
       } else if (greedy) {
-        acc = (x == sh.amax[tr0 + j]);
+        acc = (x == sh.amax[j]);
       } else {
-        const double lp = (double)load_elem(tp(j) + x) * cd - (sh.M[tr0 + j] + sh.L[tr0 + j]);
-        const double lq = (double)load_elem(dp(j) + x) * cd - dstat(j);
+        const double lp = (double)load_elem(tp(j) + x) * cd - (sh.M[j] + sh.L[j]);
+        const double lq = (double)load_elem(dp(j) + x) * cd - dlt(j);
         const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(pos0 + j),
                                       (uint32_t)stage).x;
         acc = (double)u < exp2(lp - lq);
@@ -374,198 +347,207 @@ __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const Dec
   if (lane == 0) { sh.a = a; sh.bad = bad; }
 }
 
+__device__ __forceinline__ bool rows_ok(const SeqShared& sh, int nrows) {
+  int bad = 0;
+  for (int r = 0; r < nrows; ++r) bad |= !sh.ok[r];
+  return !bad;
+}
+
 // ---------------------------------------------------------------------------
 // Chain verification
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(kDecideThreads)
-    chain_decide_kernel(ChainDecideArgs A) {
-  extern __shared__ double dyn_pre[];
+__global__ void __launch_bounds__(kFinThreads) chain_finish_kernel(ChainDecideArgs A) {
+  grid_dependency_wait();
   __shared__ SeqShared sh;
-  __shared__ bool want[kMaxRows];
   const DecideCommon& c = A.c;
-  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, V = c.V;
-  const int nrt = residual_tiles(V);
+  const int b = blockIdx.x, K = c.K, per = 2 * K + 1;
   const float Tb = c.temperature[b];
-  const bool tvalid = temp_valid(Tb);
-  const bool greedy = (Tb == 0.0f);
-  if (sp > 0 && (greedy || !tvalid)) return;
-  const Scale sc = tvalid && !greedy ? make_scale(Tb) : Scale{0.f, 0.f, 0.0};
-  const double cd = sc.d;
-  const int per = 2 * K + 1;
-  for (int r = threadIdx.x; r < per; r += blockDim.x) want[r] = (r <= K) || !greedy;
-  __syncthreads();
+  const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
   double* diag = c.diag ? c.diag + (size_t)b * (4 * K + 2) : nullptr;
-
   auto fail = [&]() {
-    if (threadIdx.x == 0) set_status(c.status, SPEC_EDEVICE);
+    if (threadIdx.x == 0) {
+      set_status(c.status, SPEC_EDEVICE);
+      A.accept_len[b] = -1;
+      c.dec[b] = SeqDecision{-1, 2};
+    }
     for (int j = threadIdx.x; j <= K; j += blockDim.x) A.out_tok[(size_t)b * (K + 1) + j] = -1;
-    if (threadIdx.x == 0) A.accept_len[b] = -1;
     if (diag)
-      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = __longlong_as_double(0x7ff8000000000000ll);
+      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
   };
-  if (!tvalid) { if (sp == 0) fail(); return; }
-
-  combine_rows(sh, c.part, b * per, per, c.ntiles, want, greedy, sc);
+  if (!tvalid) { fail(); grid_dependents_launch(); return; }
+  const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
+              sc.hi, c.fin);
   __syncthreads();
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
-  const unsigned char* tgt = A.tgt;
-  const unsigned char* drf = A.drf;
-  auto tp = [&](int j) { return row_ptr<T>(tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
-  auto dp = [&](int j) { return row_ptr<T>(drf, A.ld_drf, (long long)b * K + j); };
-  auto ds = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
-  if (threadIdx.x < 32) {
-    const bool dg = diag && sp == 0 && !greedy;
-    accept_scan<T>(sh, K, 0, 1, c, b, greedy, cd, drafts, tp, dp, ds, 0,
-                   dg ? diag + 2 * K + 1 : nullptr, dg ? diag + 3 * K + 1 : nullptr);
-  }
+  auto tp = [&](int j) { return row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
+  auto dp = [&](int j) { return row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + j); };
+  auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
+  if (threadIdx.x < 32)
+    accept_scan<T>(sh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
+                   diag && !greedy ? diag + 2 * K + 1 : nullptr,
+                   diag && !greedy ? diag + 3 * K + 1 : nullptr);
   __syncthreads();
-  int rowbad = 0;
-  for (int r = 0; r < per; ++r) rowbad |= (want[r] && !sh.ok[r]);
-  if (sh.bad || rowbad) { if (sp == 0) fail(); return; }
+  if (sh.bad || !rows_ok(sh, per)) { fail(); grid_dependents_launch(); return; }
   const int a = sh.a;
-
-  int tok;
-  double Z = __longlong_as_double(0x7ff8000000000000ll);
   if (greedy) {
-    tok = sh.amax[a];
+    for (int j = threadIdx.x; j <= K; j += blockDim.x)
+      A.out_tok[(size_t)b * (K + 1) + j] = j < a ? drafts[j] : (j == a ? sh.amax[a] : -1);
+    if (threadIdx.x == 0) { A.accept_len[b] = a; c.dec[b] = SeqDecision{a, 1}; }
+    if (diag)
+      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
   } else {
-    const T* prow = tp(a);
-    const T* qrow = a < K ? dp(a) : nullptr;
-    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sc);
-    const ProbCoef kq = make_coef(a < K ? ds(a) : 0.0, sc);
-    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 1u).y;
-    if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
+    if (threadIdx.x == 0) c.dec[b] = SeqDecision{a, 0};
+    if (diag)
+      for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
   }
-  // Emit.
+  grid_dependents_launch();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecideThreads) chain_draw_kernel(ChainDecideArgs A) {
+  grid_dependency_wait();
+  extern __shared__ double dyn_pre[];
+  const DecideCommon& c = A.c;
+  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, per = 2 * K + 1;
+  const SeqDecision d = c.dec[b];
+  if (d.state != 0) return;
+  const int a = d.a;
+  const Scale sc = make_scale(c.temperature[b]);
+  const RowFinal fp = c.fin[b * per + a];
+  const T* prow = row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + a);
+  const T* qrow = a < K ? row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + a) : nullptr;
+  double lq = 0.0;
+  if (a < K) {
+    const RowFinal fq = c.fin[b * per + K + 1 + a];
+    lq = fq.M + fq.L;
+  }
+  const ProbCoef kp = make_coef(fp.M + fp.L, sc), kq = make_coef(lq, sc);
+  const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 1u).y;
+  int tok;
+  double Z;
+  if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
+  const int32_t* drafts = c.draft_tok + (size_t)b * K;
   for (int j = threadIdx.x; j <= K; j += blockDim.x)
     A.out_tok[(size_t)b * (K + 1) + j] = j < a ? drafts[j] : (j == a ? tok : -1);
-  if (threadIdx.x == 0) A.accept_len[b] = a;
-  if (diag) {
-    for (int j = threadIdx.x; j < per; j += blockDim.x)
-      diag[j] = greedy ? __longlong_as_double(0x7ff8000000000000ll)
-                       : (sh.M[j] + sh.L[j]) * kLn2;
-    if (greedy)
-      for (int j = threadIdx.x; j < 2 * K; j += blockDim.x)
-        diag[per + j] = __longlong_as_double(0x7ff8000000000000ll);
-    if (threadIdx.x == 0) diag[4 * K + 1] = Z;
+  if (threadIdx.x == 0) {
+    A.accept_len[b] = a;
+    if (c.diag) c.diag[(size_t)b * (4 * K + 2) + 4 * K + 1] = Z;
   }
 }
-
-cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st) {
-  const int nrt = residual_tiles(a.c.V);
-  const size_t smem = 2 * (size_t)nrt * sizeof(double);
-  dim3 grid(a.c.nsplit, a.c.B);
-  if (a.c.dtype == SPEC_BF16) {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(chain_decide_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return cudaGetLastError();
-    chain_decide_kernel<__nv_bfloat16><<<grid, kDecideThreads, smem, st>>>(a);
-  } else {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(chain_decide_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return cudaGetLastError();
-    chain_decide_kernel<float><<<grid, kDecideThreads, smem, st>>>(a);
-  }
-  return cudaGetLastError();
-}
-
 
 // ---------------------------------------------------------------------------
 // Two-stage verification
 // ---------------------------------------------------------------------------
-constexpr long long kNaNBits = 0x7ff8000000000000ll;
-
 // Stage one: drafts (slots w..w+K-1) against L_i (slots w..w+K), draft law
-// L_d. The a1 accepted drafts and the drawn token join the window together
-// with the L_i statistics of their slots.
+// L_d; the a1 accepted drafts and the drawn token join the window with the
+// L_i statistics of their slots.
+__device__ __forceinline__ void window_append(const HierDecideArgs& A, int b, int w, int a,
+                                              const int32_t* drafts, int tok, const RowFinal* rf,
+                                              bool greedy, double cd) {
+  const int WC = A.Ni + A.c.K;
+  for (int j = threadIdx.x; j <= a; j += blockDim.x) {
+    const size_t slot = (size_t)b * WC + w + j;
+    A.win_tok[slot] = j < a ? drafts[j] : tok;
+    if (greedy) {
+      A.win_stat[2 * slot] = dnan();
+      A.win_stat[2 * slot + 1] = dnan();
+    } else {
+      const RowFinal f = rf[j];
+      A.win_stat[2 * slot] = f.m;
+      A.win_stat[2 * slot + 1] = (f.M + f.L - (double)f.m * cd) * kLn2;
+    }
+  }
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kDecideThreads)
-    hier1_decide_kernel(HierDecideArgs A) {
-  extern __shared__ double dyn_pre[];
+__global__ void __launch_bounds__(kFinThreads) hier1_finish_kernel(HierDecideArgs A) {
+  grid_dependency_wait();
   __shared__ SeqShared sh;
-  __shared__ bool want[kMaxRows];
   const DecideCommon& c = A.c;
-  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni;
-  const int WC = Ni + K;  // window capacity
-  const float Tb = c.temperature[b];
-  const bool tvalid = temp_valid(Tb);
-  const bool greedy = (Tb == 0.0f);
-  if (sp > 0 && (greedy || !tvalid)) return;
-  const int w = A.win_len[b];
-  const bool wvalid = (w >= 0 && w < Ni);
-  if (sp > 0 && !wvalid) return;
-  const Scale sc = tvalid && !greedy ? make_scale(Tb) : Scale{0.f, 0.f, 0.0};
-  const double cd = sc.d;
-  const int per = 2 * K + 1;
+  const int b = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni, WC = Ni + K, per = 2 * K + 1;
   const int D = 4 * K + 3 * S + 1;
   double* diag = c.diag ? c.diag + (size_t)b * D : nullptr;
-
   // Stage-two outputs default to "did not run"; stage two overwrites them.
-  if (sp == 0) {
-    for (int j = threadIdx.x; j < WC + 1; j += blockDim.x) A.commit_tok[(size_t)b * (WC + 1) + j] = -1;
-    if (threadIdx.x == 0) { A.commit_n[b] = 0; A.acc2[b] = -1; }
-    if (diag)
-      for (int j = threadIdx.x; j < D; j += blockDim.x) diag[j] = __longlong_as_double(kNaNBits);
-  }
-  if (!tvalid || !wvalid) {
-    if (sp == 0 && threadIdx.x == 0) { set_status(c.status, SPEC_EDEVICE); A.acc1[b] = -1; }
-    return;
-  }
-  for (int r = threadIdx.x; r < per; r += blockDim.x) want[r] = (r <= K) || !greedy;
-  __syncthreads();
-
-  combine_rows(sh, c.part, b * per, per, c.ntiles, want, greedy, sc);
+  for (int j = threadIdx.x; j < WC + 1; j += blockDim.x) A.commit_tok[(size_t)b * (WC + 1) + j] = -1;
+  if (threadIdx.x == 0) { A.commit_n[b] = 0; A.acc2[b] = -1; }
+  if (diag)
+    for (int j = threadIdx.x; j < D; j += blockDim.x) diag[j] = dnan();
+  const float Tb = c.temperature[b];
+  const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
+  const int w = A.win_len[b];
+  auto fail = [&]() {
+    if (threadIdx.x == 0) {
+      set_status(c.status, SPEC_EDEVICE);
+      A.acc1[b] = -1;
+      c.dec[b] = SeqDecision{-1, 2};
+    }
+  };
+  if (!tvalid || w < 0 || w >= Ni) { fail(); grid_dependents_launch(); return; }
+  const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
+              sc.hi, c.fin);
   __syncthreads();
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   const long long row0 = (long long)b * S + w;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, row0 + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_d, A.ld, row0 + j); };
-  auto ds = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
-  if (threadIdx.x < 32) {
-    const bool dg = diag && sp == 0 && !greedy;
-    accept_scan<T>(sh, K, w, 1, c, b, greedy, cd, drafts, tp, dp, ds, 0,
-                   dg ? diag + 2 * K + 1 : nullptr, dg ? diag + 3 * K + 1 : nullptr);
-  }
+  auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
+  if (threadIdx.x < 32)
+    accept_scan<T>(sh, K, w, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
+                   diag && !greedy ? diag + 2 * K + 1 : nullptr,
+                   diag && !greedy ? diag + 3 * K + 1 : nullptr);
   __syncthreads();
-  int rowbad = 0;
-  for (int r = 0; r < per; ++r) rowbad |= (want[r] && !sh.ok[r]);
-  if (sh.bad || rowbad) {
-    if (sp == 0 && threadIdx.x == 0) { set_status(c.status, SPEC_EDEVICE); A.acc1[b] = -1; }
-    return;
-  }
+  if (sh.bad || !rows_ok(sh, per)) { fail(); grid_dependents_launch(); return; }
   const int a = sh.a;
-  int tok;
-  double Z = __longlong_as_double(kNaNBits);
   if (greedy) {
-    tok = sh.amax[a];
+    window_append(A, b, w, a, drafts, sh.amax[a], nullptr, true, 0.0);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      A.win_len[b] = w + a + 1;
+      A.acc1[b] = a;
+      c.dec[b] = SeqDecision{a, 1};
+    }
   } else {
-    const T* prow = tp(a);
-    const T* qrow = a < K ? dp(a) : nullptr;
-    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sc);
-    const ProbCoef kq = make_coef(a < K ? ds(a) : 0.0, sc);
-    const float u =
-        spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(w + a), 1u).y;
-    if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
+    if (threadIdx.x == 0) c.dec[b] = SeqDecision{a, 0};
+    if (diag)
+      for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
   }
-  // Append a + 1 tokens and their L_i statistics to the window.
-  for (int j = threadIdx.x; j <= a; j += blockDim.x) {
-    const size_t slot = (size_t)b * WC + w + j;
-    A.win_tok[slot] = j < a ? drafts[j] : tok;
-    A.win_stat[2 * slot] = greedy ? __longlong_as_double(kNaNBits) : sh.m[j];
-    A.win_stat[2 * slot + 1] =
-        greedy ? __longlong_as_double(kNaNBits) : (sh.M[j] + sh.L[j] - sh.m[j] * cd) * kLn2;
+  grid_dependents_launch();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecideThreads) hier1_draw_kernel(HierDecideArgs A) {
+  grid_dependency_wait();
+  extern __shared__ double dyn_pre[];
+  const DecideCommon& c = A.c;
+  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, S = A.S, per = 2 * K + 1;
+  const SeqDecision d = c.dec[b];
+  if (d.state != 0) return;
+  const int a = d.a;
+  const int w = A.win_len[b];
+  const Scale sc = make_scale(c.temperature[b]);
+  const long long row0 = (long long)b * S + w;
+  const RowFinal fp = c.fin[b * per + a];
+  const T* prow = row_ptr<T>(A.lg_i, A.ld, row0 + a);
+  const T* qrow = a < K ? row_ptr<T>(A.lg_d, A.ld, row0 + a) : nullptr;
+  double lq = 0.0;
+  if (a < K) {
+    const RowFinal fq = c.fin[b * per + K + 1 + a];
+    lq = fq.M + fq.L;
   }
+  const ProbCoef kp = make_coef(fp.M + fp.L, sc), kq = make_coef(lq, sc);
+  const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(w + a), 1u).y;
+  int tok;
+  double Z;
+  if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
+  window_append(A, b, w, a, c.draft_tok + (size_t)b * K, tok, c.fin + (size_t)b * per, false, sc.d);
   __syncthreads();
   if (threadIdx.x == 0) {
     A.win_len[b] = w + a + 1;
     A.acc1[b] = a;
-  }
-  if (diag && !greedy) {
-    for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
-    if (threadIdx.x == 0) diag[4 * K + 1] = Z;
+    if (c.diag) c.diag[(size_t)b * (4 * K + 3 * S + 1) + 4 * K + 1] = Z;
   }
 }
 
@@ -573,59 +555,82 @@ __global__ void __launch_bounds__(kDecideThreads)
 // tokens (slots 0..W-1) against L_f (slots 0..W), draft law L_i from the
 // buffered statistics; commits a2 + 1 tokens and empties the window.
 template <typename T>
-__global__ void __launch_bounds__(kDecideThreads)
-    hier2_decide_kernel(HierDecideArgs A) {
-  extern __shared__ double dyn_pre[];
+__global__ void __launch_bounds__(kFinThreads) hier2_finish_kernel(HierDecideArgs A) {
+  grid_dependency_wait();
   __shared__ SeqShared sh;
-  __shared__ bool want[kMaxRows];
   const DecideCommon& c = A.c;
-  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni;
-  const int WC = Ni + K;
-  if (A.acc1[b] < 0) return;
+  const int b = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni, WC = Ni + K;
   const int W = A.win_len[b];
-  if (!(W >= Ni && W < S)) return;
-  const float Tb = c.temperature[b];
-  const bool greedy = (Tb == 0.0f);  // temperature validated by stage one
-  if (sp > 0 && greedy) return;
-  const Scale sc = !greedy ? make_scale(Tb) : Scale{0.f, 0.f, 0.0};
-  const double cd = sc.d;
-  const int D = 4 * K + 3 * S + 1;
-  double* diag = c.diag ? c.diag + (size_t)b * D + (4 * K + 2) : nullptr;
-  for (int r = threadIdx.x; r < S; r += blockDim.x) want[r] = (r <= W);
-  __syncthreads();
-
-  combine_rows(sh, c.part, b * S, W + 1, c.ntiles, want, greedy, sc);
+  if (A.acc1[b] < 0 || !(W >= Ni && W < S)) {
+    if (threadIdx.x == 0) c.dec[b] = SeqDecision{-1, 1};  // no second stage
+    grid_dependents_launch();
+    return;
+  }
+  const float Tb = c.temperature[b];  // validated by stage one
+  const bool greedy = (Tb == 0.0f);
+  const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+  double* diag = c.diag ? c.diag + (size_t)b * (4 * K + 3 * S + 1) + (4 * K + 2) : nullptr;
+  finish_rows(sh, c.part, c.ntiles, b * S, W + 1, [&](int) { return true; }, greedy, sc.hi, c.fin);
   __syncthreads();
   const int32_t* wtok = A.win_tok + (size_t)b * WC;
   const double* wst = A.win_stat + (size_t)b * WC * 2;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_f, A.ld, (long long)b * S + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, (long long)b * S + j); };
-  auto ds = [&](int j) { return wst[2 * j] * cd + wst[2 * j + 1] * kLog2e; };
-  if (threadIdx.x < 32) {
-    const bool dg = diag && sp == 0 && !greedy;
-    accept_scan<T>(sh, W, 0, 2, c, b, greedy, cd, wtok, tp, dp, ds, 0,
-                   dg ? diag + S : nullptr, dg ? diag + 2 * S - 1 : nullptr);
-  }
+  auto dl = [&](int j) { return wst[2 * j] * sc.d + wst[2 * j + 1] * kLog2e; };
+  if (threadIdx.x < 32)
+    accept_scan<T>(sh, W, 0, 2, c, b, greedy, sc.d, wtok, tp, dp, dl,
+                   diag && !greedy ? diag + S : nullptr, diag && !greedy ? diag + 2 * S - 1 : nullptr);
   __syncthreads();
-  int rowbad = 0;
-  for (int r = 0; r <= W; ++r) rowbad |= !sh.ok[r];
-  if (sh.bad || rowbad) {
-    if (sp == 0 && threadIdx.x == 0) { set_status(c.status, SPEC_EDEVICE); A.acc2[b] = -1; }
+  if (sh.bad || !rows_ok(sh, W + 1)) {
+    if (threadIdx.x == 0) {
+      set_status(c.status, SPEC_EDEVICE);
+      A.acc2[b] = -1;
+      c.dec[b] = SeqDecision{-1, 2};
+    }
+    grid_dependents_launch();
     return;
   }
   const int a = sh.a;
-  int tok;
-  double Z = __longlong_as_double(kNaNBits);
   if (greedy) {
-    tok = sh.amax[a];
+    for (int j = threadIdx.x; j < WC + 1; j += blockDim.x)
+      A.commit_tok[(size_t)b * (WC + 1) + j] = j < a ? wtok[j] : (j == a ? sh.amax[a] : -1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      A.commit_n[b] = a + 1;
+      A.acc2[b] = a;
+      A.win_len[b] = 0;
+      c.dec[b] = SeqDecision{a, 1};
+    }
   } else {
-    const T* prow = tp(a);
-    const T* qrow = a < W ? dp(a) : nullptr;
-    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sc);
-    const ProbCoef kq = make_coef(a < W ? ds(a) : 0.0, sc);
-    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 2u).y;
-    if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
+    if (threadIdx.x == 0) c.dec[b] = SeqDecision{a, 0};
+    if (diag)
+      for (int j = threadIdx.x; j <= W; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
   }
+  grid_dependents_launch();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecideThreads) hier2_draw_kernel(HierDecideArgs A) {
+  grid_dependency_wait();
+  extern __shared__ double dyn_pre[];
+  const DecideCommon& c = A.c;
+  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni, WC = Ni + K;
+  const SeqDecision d = c.dec[b];
+  if (d.state != 0) return;
+  const int a = d.a;
+  const int W = A.win_len[b];
+  const Scale sc = make_scale(c.temperature[b]);
+  const RowFinal fp = c.fin[b * S + a];
+  const double* wst = A.win_stat + (size_t)b * WC * 2;
+  const T* prow = row_ptr<T>(A.lg_f, A.ld, (long long)b * S + a);
+  const T* qrow = a < W ? row_ptr<T>(A.lg_i, A.ld, (long long)b * S + a) : nullptr;
+  const double lq = a < W ? wst[2 * a] * sc.d + wst[2 * a + 1] * kLog2e : 0.0;
+  const ProbCoef kp = make_coef(fp.M + fp.L, sc), kq = make_coef(lq, sc);
+  const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 2u).y;
+  int tok;
+  double Z;
+  if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
+  const int32_t* wtok = A.win_tok + (size_t)b * WC;
   for (int j = threadIdx.x; j < WC + 1; j += blockDim.x)
     A.commit_tok[(size_t)b * (WC + 1) + j] = j < a ? wtok[j] : (j == a ? tok : -1);
   __syncthreads();
@@ -633,41 +638,43 @@ __global__ void __launch_bounds__(kDecideThreads)
     A.commit_n[b] = a + 1;
     A.acc2[b] = a;
     A.win_len[b] = 0;
-  }
-  if (diag && !greedy) {
-    for (int j = threadIdx.x; j <= W; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
-    if (threadIdx.x == 0) diag[3 * S - 2] = Z;
+    if (c.diag) c.diag[(size_t)b * (4 * K + 3 * S + 1) + (4 * K + 2) + 3 * S - 2] = Z;
   }
 }
 
-template <typename K1, typename K2>
-static cudaError_t launch_decide(K1 kb, K2 kf, int dtype, dim3 grid, size_t smem,
-                                 const HierDecideArgs& a, cudaStream_t st) {
-  if (dtype == SPEC_BF16) {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-      return cudaGetLastError();
-    kb<<<grid, kDecideThreads, smem, st>>>(a);
-  } else {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-      return cudaGetLastError();
-    kf<<<grid, kDecideThreads, smem, st>>>(a);
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st) {
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+template <typename Kern, typename Args>
+static cudaError_t launch_draw(Kern k, const Args& a, cudaStream_t st) {
   const size_t smem = 2 * (size_t)residual_tiles(a.c.V) * sizeof(double);
-  return launch_decide(hier1_decide_kernel<__nv_bfloat16>, hier1_decide_kernel<float>, a.c.dtype,
-                       dim3(a.c.nsplit, a.c.B), smem, a, st);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return cudaGetLastError();
+  return launch_pdl(k, dim3(a.c.nsplit, a.c.B), dim3(kDecideThreads), smem, st, a);
+}
+template <typename Fin, typename Draw, typename Args>
+static cudaError_t launch_pair(Fin f, Draw d, const Args& a, cudaStream_t st) {
+  cudaError_t e = launch_pdl(f, dim3(a.c.B), dim3(kFinThreads), 0, st, a);
+  if (e != cudaSuccess) return e;
+  return launch_draw(d, a, st);
+}
+
+cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st) {
+  return a.c.dtype == SPEC_BF16
+             ? launch_pair(chain_finish_kernel<__nv_bfloat16>, chain_draw_kernel<__nv_bfloat16>, a, st)
+             : launch_pair(chain_finish_kernel<float>, chain_draw_kernel<float>, a, st);
+}
+cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st) {
+  return a.c.dtype == SPEC_BF16
+             ? launch_pair(hier1_finish_kernel<__nv_bfloat16>, hier1_draw_kernel<__nv_bfloat16>, a, st)
+             : launch_pair(hier1_finish_kernel<float>, hier1_draw_kernel<float>, a, st);
 }
 cudaError_t launch_hier2_decide(const HierDecideArgs& a, cudaStream_t st) {
-  const size_t smem = 2 * (size_t)residual_tiles(a.c.V) * sizeof(double);
-  return launch_decide(hier2_decide_kernel<__nv_bfloat16>, hier2_decide_kernel<float>, a.c.dtype,
-                       dim3(a.c.nsplit, a.c.B), smem, a, st);
+  return a.c.dtype == SPEC_BF16
+             ? launch_pair(hier2_finish_kernel<__nv_bfloat16>, hier2_draw_kernel<__nv_bfloat16>, a, st)
+             : launch_pair(hier2_finish_kernel<float>, hier2_draw_kernel<float>, a, st);
 }
 
 }  // namespace specv

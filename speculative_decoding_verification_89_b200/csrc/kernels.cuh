@@ -74,21 +74,72 @@ struct Hier2Rows {
   }
 };
 
+// Workspace pieces of the row-statistics step.
+struct RsBuffers {
+  Partial* part;    // [rows, tiles]
+  int* seq_cnt;     // [nseq] decide arrival counters, cleared here
+  int nseq;
+};
+
+// Combine a row's tile partials (warp-cooperative; result valid in lane 0).
+__device__ __forceinline__ RowFinal combine_row(const Partial* p, int ntiles, bool greedy,
+                                                float chi, int lane) {
+  float mv = -INFINITY;
+  int mi = 0x7fffffff;
+  for (int t = lane; t < ntiles; t += 32) {
+    const float m = p[t].m;
+    const int i = p[t].idx;
+    if (m > mv || (m == mv && i < mi)) { mv = m; mi = i; }
+  }
+  warp_argmax(mv, mi);
+  RowFinal f;
+  f.m = mv;
+  f.amax = mi;
+  f.M = 0.0;
+  f.L = 0.0;
+  f.pad = 0;
+  bool ok = (mv > -INFINITY && mv < INFINITY);
+  if (ok && !greedy) {
+    f.M = (double)__fmul_rn(mv, chi);
+    double s = 0.0;
+    for (int t = lane; t < ntiles; t += 32) {
+      const double st = p[t].s;
+      if (st != 0.0) s += st * exp2((double)__fmul_rn(p[t].m, chi) - f.M);
+    }
+    s = warp_sum_d(s);
+    ok = (s > 0.0 && s < INFINITY);
+    f.L = log2(s);
+  }
+  f.ok = ok;
+  return f;
+}
+
+// Outcome of a sequence's accept test: a = first rejection; state 0 = the
+// draw is pending, 1 = outputs already written (greedy, or no second stage),
+// 2 = invalid input.
+struct SeqDecision {
+  int a;
+  int state;
+};
+
 template <typename Rows>
-cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, Partial* part,
-                             int* zero_words, int nzero, int32_t* status, cudaStream_t st);
+cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, const RsBuffers& b,
+                             int32_t* status, cudaStream_t st);
 
 // ----------------------------------------------------------------------------
 // Decide kernels (accept test, first rejection, residual / bonus draw)
 // ----------------------------------------------------------------------------
 struct DecideCommon {
-  int dtype, B, K, V, ntiles;      // ntiles: row-statistics tiles per row
+  int dtype, B, K, V;
   const int32_t* draft_tok;
   const float* temperature;
   uint64_t seed;
   const int32_t* seq_id;
   uint32_t round;
-  const Partial* part;
+  const Partial* part;             // [rows, ntiles] tile partials
+  int ntiles;
+  RowFinal* fin;                   // [rows] final row statistics
+  SeqDecision* dec;                // [B]
   double* rsum;                    // [B, nrt] residual tile sums
   int* counters;                   // [B] arrival counters (zeroed by row stats)
   int nsplit;                      // CTAs per sequence for the residual pass

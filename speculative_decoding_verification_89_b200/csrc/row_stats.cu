@@ -46,6 +46,29 @@ __device__ __forceinline__ float vec_elem(uint4 w, int e, float*) {
   return __uint_as_float(word);
 }
 
+// Largest element of a lane's register-resident vectors.
+template <int kVpl>
+__device__ __forceinline__ float regs_max(const uint4* x, __nv_bfloat16*) {
+  __nv_bfloat162 m2 = __float2bfloat162_rn(-INFINITY);
+#pragma unroll
+  for (int i = 0; i < kVpl; ++i) {
+    uint4 w = x[i];
+    const __nv_bfloat162 a = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.x),
+                                     *reinterpret_cast<__nv_bfloat162*>(&w.y));
+    const __nv_bfloat162 b = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.z),
+                                     *reinterpret_cast<__nv_bfloat162*>(&w.w));
+    m2 = __hmax2(m2, __hmax2(a, b));
+  }
+  return fmaxf(__low2float(m2), __high2float(m2));
+}
+template <int kVpl>
+__device__ __forceinline__ float regs_max(const uint4* x, float*) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kVpl; ++i) m = fmaxf(m, vec_max(x[i], (float*)nullptr));
+  return m;
+}
+
 // Sum over one 16-byte vector of 2^(x*c - M) with c = chi + clo and M an
 // exact fp32 shift: two packed FP32x2 FMAs per element pair form the
 // exponent (the product x*chi - M is rounded once, relative to the small
@@ -70,6 +93,31 @@ __device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, fl
       ex2x2(expo2(make_float2(__uint_as_float(w.z), __uint_as_float(w.w)), chi, clo, nM));
   return __fadd2_rn(e0, e1);
 }
+// Scalar forms (one FMA pair per element): the same arithmetic without
+// packing, for builds where pair formation costs more than it saves.
+__device__ __forceinline__ float vec_expsum_s(uint4 w, float chi, float clo, float nM,
+                                              __nv_bfloat16*) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  float e[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float lo = bf_lo(ws[q]), hi = bf_hi(ws[q]);
+    e[2 * q] = ex2(fmaf(lo, clo, fmaf(lo, chi, nM)));
+    e[2 * q + 1] = ex2(fmaf(hi, clo, fmaf(hi, chi, nM)));
+  }
+  return ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+}
+__device__ __forceinline__ float vec_expsum_s(uint4 w, float chi, float clo, float nM, float*) {
+  float e[4];
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float x = __uint_as_float(ws[q]);
+    e[q] = ex2(fmaf(x, clo, fmaf(x, chi, nM)));
+  }
+  return (e[0] + e[1]) + (e[2] + e[3]);
+}
+
 // Scalar form of one term (tail elements).
 __device__ __forceinline__ float term(float x, float chi, float clo, float nM) {
   return ex2(fmaf(x, clo, fmaf(x, chi, nM)));
@@ -111,6 +159,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   constexpr int kEpt = kTileBytes / (int)sizeof(T);     // elements per tile
   constexpr int kVpl = kTileBytes / 16 / 32;            // vectors per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dependency_wait();
 
   // Clear the decide kernels' arrival counters (stream-ordered before them).
   if (blockIdx.x == 0)
@@ -166,6 +215,20 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   bool timed_out = false;
   int s = 0;  // stage of the item being consumed
 
+  // Hand stage s back to the copy engine with the next item of this warp.
+  auto refill = [&](int st) {
+    __syncwarp();
+    if (prod.r < nrows) {
+      if (lane == 0) {
+        fence_proxy_async_smem();
+        issue(st, prod);
+      }
+      ++inflight;
+      advance(prod);
+      settle(prod);
+    }
+  };
+
   for (; cons.r < nrows; s = (s + 1 == kRsStages) ? 0 : s + 1) {
     const bool ok = mbar_wait_bounded(&bars[s], (phase >> s) & 1u, kWaitLimitNs);
     if (__any_sync(0xffffffffu, !ok)) {
@@ -185,63 +248,128 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       clo = sc.lo;
     }
     const int nel = min(kEpt, V - t * kEpt);
-    const int nvec = (int)(((uint32_t)nel * sizeof(T)) >> 4);
-    const int ntail = nel - nvec * kVec;
     const uint4* buf = reinterpret_cast<const uint4*>(wbuf + s * kTileBytes);
-    const T* gtail = reinterpret_cast<const T*>(ref.ptr) + (size_t)t * kEpt + nvec * kVec;
-
-    // Pass 1: largest value and the first vector holding it.
     float best = -INFINITY;
-    int bestv = -1;
-#pragma unroll
-    for (int i = 0; i < kVpl; ++i) {
-      const int v = lane + 32 * i;
-      if (v < nvec) {
-        const float vm = vec_max(buf[v], (T*)nullptr);
-        if (vm > best) { best = vm; bestv = v; }
-      }
-    }
     int bidx = 0x7fffffff;
-    if (bestv >= 0) {
-      const uint4 w = buf[bestv];
-#pragma unroll
-      for (int e = kVec - 1; e >= 0; --e)
-        if (vec_elem(w, e, (T*)nullptr) == best) bidx = bestv * kVec + e;
-    }
-    float tailx = -INFINITY;
-    if (lane < ntail) {
-      tailx = load_elem(gtail + lane);
-      if (tailx > best) { best = tailx; bidx = nvec * kVec + lane; }
-    }
-    warp_argmax(best, bidx);
-
     double ssum = 0.0;
-    if (!greedy && best > -INFINITY && best < INFINITY) {
-      // Pass 2: sum of 2^(l*c - M) with the exact fp32 shift M = fl(m*chi).
-      const float M = __fmul_rn(best, chi);
-      if (fabsf(M) < 67108864.0f) {  // 2^26: 2^(m*c - M) <= 2^2
-        const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
-        const float2 nM2 = make_float2(-M, -M);
-        float2 acc = make_float2(0.0f, 0.0f);
+
+    if (nel == kEpt) {
+      // Full tile: each lane's vectors go to registers once; the stage is
+      // refilled before the arithmetic starts.
+      uint4 x[kVpl];
+#pragma unroll
+      for (int i = 0; i < kVpl; ++i) x[i] = buf[lane + 32 * i];
+      refill(s);
+      if (greedy) {
+        int bestv = -1;
 #pragma unroll
         for (int i = 0; i < kVpl; ++i) {
-          const int v = lane + 32 * i;
-          if (v < nvec) acc = __fadd2_rn(acc, vec_expsum(buf[v], chi2, clo2, nM2, (T*)nullptr));
+          const float vm = vec_max(x[i], (T*)nullptr);
+          if (vm > best) { best = vm; bestv = i; }
         }
-        float a = acc.x + acc.y;
-        if (lane < ntail) a += term(tailx, chi, clo, -M);
-        ssum = warp_sum_d((double)a);
+        if (bestv >= 0) {
+          uint4 w = x[0];
+#pragma unroll
+          for (int i = 1; i < kVpl; ++i)
+            if (i == bestv) w = x[i];
+#pragma unroll
+          for (int e = kVec - 1; e >= 0; --e)
+            if (vec_elem(w, e, (T*)nullptr) == best) bidx = (lane + 32 * bestv) * kVec + e;
+        }
+        warp_argmax(best, bidx);
       } else {
-        const float rr = fmaf(best, chi, -M) + best * clo;
-        float a = 0.0f;
+        best = regs_max<kVpl>(x, (T*)nullptr);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (best > -INFINITY && best < INFINITY) {
+          const float M = __fmul_rn(best, chi);
+          float a;
+          if (fabsf(M) < 67108864.0f) {  // 2^26: 2^(m*c - M) <= 2^2
+#if SPEC_RS_PACKED
+            const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
+            const float2 nM2 = make_float2(-M, -M);
+            float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int i = 0; i < kVpl; ++i)
+              acc = __fadd2_rn(acc, vec_expsum(x[i], chi2, clo2, nM2, (T*)nullptr));
+            a = acc.x + acc.y;
+#else
+            float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kVpl; i += 2) {
+              acc0 += vec_expsum_s(x[i], chi, clo, -M, (T*)nullptr);
+              if (i + 1 < kVpl) acc1 += vec_expsum_s(x[i + 1], chi, clo, -M, (T*)nullptr);
+            }
+            a = acc0 + acc1;
+#endif
+          } else {
+            const float rr = fmaf(best, chi, -M) + best * clo;
+            a = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kVpl; ++i) a += vec_expsum_far<T>(x[i], best, chi, clo, rr);
+          }
+          ssum = warp_sum_d((double)a);
+        }
+      }
+    } else {
+      // Last, partial tile of a row: guarded loads and a scalar tail.
+      const int nvec = (int)(((uint32_t)nel * sizeof(T)) >> 4);
+      const int ntail = nel - nvec * kVec;
+      const T* gtail = reinterpret_cast<const T*>(ref.ptr) + (size_t)t * kEpt + nvec * kVec;
+      float tailx = -INFINITY;
+      if (lane < ntail) tailx = load_elem(gtail + lane);
+      if (greedy) {
+        int bestv = -1;
         for (int i = 0; i < kVpl; ++i) {
           const int v = lane + 32 * i;
-          if (v < nvec) a += vec_expsum_far<T>(buf[v], best, chi, clo, rr);
+          if (v < nvec) {
+            const float vm = vec_max(buf[v], (T*)nullptr);
+            if (vm > best) { best = vm; bestv = v; }
+          }
         }
-        if (lane < ntail) a += term_far(tailx, best, chi, clo, rr);
-        ssum = warp_sum_d((double)a);
+        if (bestv >= 0) {
+          const uint4 w = buf[bestv];
+#pragma unroll
+          for (int e = kVec - 1; e >= 0; --e)
+            if (vec_elem(w, e, (T*)nullptr) == best) bidx = bestv * kVec + e;
+        }
+        if (tailx > best) { best = tailx; bidx = nvec * kVec + lane; }
+        warp_argmax(best, bidx);
+      } else {
+        for (int i = 0; i < kVpl; ++i) {
+          const int v = lane + 32 * i;
+          if (v < nvec) best = fmaxf(best, vec_max(buf[v], (T*)nullptr));
+        }
+        best = fmaxf(best, tailx);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (best > -INFINITY && best < INFINITY) {
+          const float M = __fmul_rn(best, chi);
+          float a = 0.0f;
+          if (fabsf(M) < 67108864.0f) {
+            const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
+            const float2 nM2 = make_float2(-M, -M);
+            float2 acc = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < kVpl; ++i) {
+              const int v = lane + 32 * i;
+              if (v < nvec) acc = __fadd2_rn(acc, vec_expsum(buf[v], chi2, clo2, nM2, (T*)nullptr));
+            }
+            a = acc.x + acc.y;
+            if (lane < ntail) a += term(tailx, chi, clo, -M);
+          } else {
+            const float rr = fmaf(best, chi, -M) + best * clo;
+            for (int i = 0; i < kVpl; ++i) {
+              const int v = lane + 32 * i;
+              if (v < nvec) a += vec_expsum_far<T>(buf[v], best, chi, clo, rr);
+            }
+            if (lane < ntail) a += term_far(tailx, best, chi, clo, rr);
+          }
+          ssum = warp_sum_d((double)a);
+        }
       }
+      refill(s);
     }
+
     if (lane == 0) {
       Partial p;
       p.m = best;
@@ -250,17 +378,6 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       part[(size_t)r * ntiles + t] = p;
     }
 
-    // Every lane is done with stage s; refill it.
-    __syncwarp();
-    if (prod.r < nrows) {
-      if (lane == 0) {
-        fence_proxy_async_smem();
-        issue(s, prod);
-      }
-      ++inflight;
-      advance(prod);
-      settle(prod);
-    }
     advance(cons);
     settle(cons);
   }
@@ -274,6 +391,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       mbar_wait_bounded(&bars[q], (phase >> q) & 1u, kWaitLimitNs);
     }
   }
+  grid_dependents_launch();
 }
 
 // ----------------------------------------------------------------------------
@@ -310,23 +428,23 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
   const long long need = (items + kRsWarps - 1) / kRsWarps;
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
-  kern<<<(int)grid, kRsWarps * 32, kRsSmem, st>>>(rows, nrows, V, part, zero_words, nzero, status);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kRsWarps * 32), kRsSmem, st, rows, nrows, V,
+                    part, zero_words, nzero, status);
 }
 
 template <typename Rows>
-cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, Partial* part,
-                             int* zero_words, int nzero, int32_t* status, cudaStream_t st) {
+cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, const RsBuffers& b,
+                             int32_t* status, cudaStream_t st) {
   if (dtype == SPEC_BF16)
-    return launch_rs<__nv_bfloat16>(rows, nrows, V, part, zero_words, nzero, status, st);
-  return launch_rs<float>(rows, nrows, V, part, zero_words, nzero, status, st);
+    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, b.seq_cnt, b.nseq, status, st);
+  return launch_rs<float>(rows, nrows, V, b.part, b.seq_cnt, b.nseq, status, st);
 }
 
-template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int, Partial*, int*,
-                                                 int, int32_t*, cudaStream_t);
-template cudaError_t launch_row_stats<Hier1Rows>(int, const Hier1Rows&, int, int, Partial*, int*,
-                                                 int, int32_t*, cudaStream_t);
-template cudaError_t launch_row_stats<Hier2Rows>(int, const Hier2Rows&, int, int, Partial*, int*,
-                                                 int, int32_t*, cudaStream_t);
+template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int,
+                                                 const RsBuffers&, int32_t*, cudaStream_t);
+template cudaError_t launch_row_stats<Hier1Rows>(int, const Hier1Rows&, int, int,
+                                                 const RsBuffers&, int32_t*, cudaStream_t);
+template cudaError_t launch_row_stats<Hier2Rows>(int, const Hier2Rows&, int, int,
+                                                 const RsBuffers&, int32_t*, cudaStream_t);
 
 }  // namespace specv
