@@ -22,10 +22,10 @@ constexpr double kLn2 = 0.6931471805599453094172321214581766;
 // Row-statistics tiles: kTileBytes of one row, staged by one bulk copy into a
 // per-warp ring of kRsStages buffers; one CTA of kRsWarps warps per SM.
 #ifndef SPEC_RS_TILE
-#define SPEC_RS_TILE 4096
+#define SPEC_RS_TILE 6144
 #endif
 #ifndef SPEC_RS_WARPS
-#define SPEC_RS_WARPS 24
+#define SPEC_RS_WARPS 16
 #endif
 #ifndef SPEC_RS_STAGES
 #define SPEC_RS_STAGES 2
