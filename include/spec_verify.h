@@ -230,6 +230,31 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
                       const void* hid_stage, void* hid_out, int32_t* hid_off,
                       int hidden, int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Chain verification without a caller workspace. The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory where they verify (a fixed memory budget, an allocator owned
+ * by a host program, a loop that must not call an allocator). It does what
+ * spec_verify_chain does, with the same arguments minus the workspace, and
+ * takes its scratch from an array of SPEC_NOALLOC_SCRATCH_BYTES compiled into
+ * the library; every GPU that loads the library holds that array until the
+ * process exits. It calls no allocating routine.
+ *   - Sizes whose workspace (spec_workspace_bytes(B, K, V, dtype, 0)) would
+ *     exceed the array return SPEC_EWORKSPACE and launch nothing.
+ *   - The first call on a device looks the array's device address up with
+ *     that device current; make that first call outside any stream capture.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents; each call clears what must start at zero. Calls that overlap
+ *     on the GPU (several streams or threads) race on it and must not be made.
+ * ------------------------------------------------------------------------- */
+#define SPEC_NOALLOC_SCRATCH_BYTES (16u << 20)
+int spec_verify_chain_noalloc(const void* tgt, int64_t ld_tgt, const void* drf,
+                              int64_t ld_drf, int dtype, int B, int K, int V,
+                              const int32_t* draft_tok, const float* temperature,
+                              uint64_t seed, const int32_t* seq_id, uint32_t round,
+                              int32_t* accept_len, int32_t* out_tok, double* diag,
+                              int32_t* dev_status, void* stream);
+
 /* Diagnostic: text of the last CUDA error behind a SPEC_ECUDA return on the
  * calling thread ("no error" if none). Static storage. */
 const char* spec_last_cuda_error(void);

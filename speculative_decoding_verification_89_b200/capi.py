@@ -44,6 +44,8 @@ _SIGS = {
                                _i, _i, _i, _p, _p, _p, _i, _p, _p]),
     "spec_philox_uniforms": (_i, [_u64, _p, _i, _p, _p]),
     "spec_last_cuda_error": (ctypes.c_char_p, []),
+    "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
+                                       _u32, _p, _p, _p, _p, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -125,6 +127,21 @@ def spec_verify_chain(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accep
         _ptr(temperature), seed, _ptr(seq_id), rnd, _ptr(accept_len), _ptr(out_tok),
         _ptr(diag), _ptr(dev_status), _ptr(ws), ws.numel(), _stream(stream))
     _check("spec_verify_chain", rc)
+
+
+def spec_verify_chain_noalloc(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
+                              out_tok, dev_status, diag=None, stream=None):
+    """spec_verify_chain for callers that cannot allocate: no workspace
+    argument; the library's built-in scratch array is used instead (see
+    include/spec_verify.h for its size and sharing rules)."""
+    B, Kp1, V = tgt.shape
+    K = Kp1 - 1
+    rc = _lib.spec_verify_chain_noalloc(
+        _ptr(tgt), _rows(tgt, Kp1), _ptr(drf) if K > 0 else None,
+        _rows(drf, K) if K > 0 else 0, _dtype_code(tgt), B, K, V, _ptr(draft_tok),
+        _ptr(temperature), seed, _ptr(seq_id), rnd, _ptr(accept_len), _ptr(out_tok),
+        _ptr(diag), _ptr(dev_status), _stream(stream))
+    _check("spec_verify_chain_noalloc", rc)
 
 
 def spec_chain_row_stats(tgt, drf, temperature, dev_status, ws, stream=None):

@@ -114,6 +114,8 @@ DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_to
 
 }  // namespace
 
+size_t specv::workspace_counter_bytes(int B) { return align_up((size_t)std::max(B, 1) * sizeof(int)); }
+
 #pragma GCC visibility push(default)
 extern "C" {
 

@@ -205,4 +205,8 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
 
+// Bytes at the start of a workspace that hold the arrival counters (the part
+// that must be zero when a call starts).
+size_t workspace_counter_bytes(int B);
+
 }  // namespace specv
