@@ -79,7 +79,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 /* Limits checked on the host. */
 #define SPEC_MAX_K 256           /* drafts per sequence per call      */
 #define SPEC_MAX_V (1 << 22)     /* vocabulary size                   */
-#define SPEC_MAX_COMMIT_B 32768  /* sequences per paged commit        */
+#define SPEC_MAX_COMMIT_B 16384  /* sequences per paged commit        */
 
 /* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
  * chain call, Ni > 0 a two-stage call. Returns 0 for invalid sizes. */

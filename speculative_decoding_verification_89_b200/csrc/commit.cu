@@ -21,58 +21,85 @@ namespace specv {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kCopyThreads = 256;
-constexpr int kCopyParts = 4;  // CTAs per kept token
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Block-wide exclusive scan of one int per thread (kPlanThreads threads).
-__device__ int block_excl_scan(int v, int* total) {
-  __shared__ int warp_sums[kPlanThreads / 32];
+// Block-wide exclusive scan of three ints per thread (kPlanThreads threads);
+// totals returned in tot.
+__device__ int3 block_excl_scan3(int3 v, int3* tot) {
+  __shared__ int3 warp_sums[kPlanThreads / 32];
+  __shared__ int3 s_tot;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+  int3 incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+    const int yx = __shfl_up_sync(0xffffffffu, incl.x, o);
+    const int yy = __shfl_up_sync(0xffffffffu, incl.y, o);
+    const int yz = __shfl_up_sync(0xffffffffu, incl.z, o);
+    if (lane >= o) { incl.x += yx; incl.y += yy; incl.z += yz; }
   }
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_sums[lane];
-    int wi = w;
+    const int3 w = warp_sums[lane];
+    int3 wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += y;
+      const int yx = __shfl_up_sync(0xffffffffu, wi.x, o);
+      const int yy = __shfl_up_sync(0xffffffffu, wi.y, o);
+      const int yz = __shfl_up_sync(0xffffffffu, wi.z, o);
+      if (lane >= o) { wi.x += yx; wi.y += yy; wi.z += yz; }
     }
-    warp_sums[lane] = wi - w;  // exclusive
+    warp_sums[lane] = make_int3(wi.x - w.x, wi.y - w.y, wi.z - w.z);  // exclusive
+    if (lane == 31) s_tot = wi;
   }
   __syncthreads();
-  const int excl = warp_sums[warp] + incl - v;
-  // Total: last thread's inclusive value.
-  __shared__ int s_total;
-  if (threadIdx.x == blockDim.x - 1) s_total = excl + v;
-  __syncthreads();
-  *total = s_total;
-  __syncthreads();  // warp_sums / s_total reusable afterwards
-  return excl;
+  const int3 base = warp_sums[warp];
+  *tot = s_tot;
+  return make_int3(base.x + incl.x - v.x, base.y + incl.y - v.y, base.z + incl.z - v.z);
 }
 
+// One CTA. Per-sequence inputs are read once into shared memory; every check
+// is made before anything is written.
 __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a) {
   grid_dependency_wait();
-  extern __shared__ int s_nb[];  // [B] blocks covered before the commit
-  __shared__ int s_bad, s_code;
-  if (threadIdx.x == 0) { s_bad = 0; s_code = 0; }
-  __syncthreads();
-  if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;  // sticky error
+  extern __shared__ int s_seq[];  // [3][B]: blocks before, blocks after, kept
+  int* s_nbo = s_seq;
+  int* s_nbn = s_seq + a.B;
+  int* s_kept = s_seq + 2 * a.B;
+  __shared__ int s_bad, s_code, s_ft;
+  if (threadIdx.x == 0) { s_bad = 0; s_code = 0; s_ft = *a.free_top; }
+  if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;  // sticky error (uniform)
   const int bs = a.block_size;
-  for (int b = threadIdx.x; b < a.B; b += blockDim.x) s_nb[b] = ceil_div(max(a.seq_lens[b], 0), bs);
+  // Each thread owns a contiguous run of sequences (sequence order matters
+  // for the allocation order).
+  const int per = ceil_div(a.B, blockDim.x);
+  const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
+  int3 cnt = make_int3(0, 0, 0);  // frees, allocations, kept rows
+  int bad = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int old_len = a.seq_lens[b];
+    const int base = a.base_len ? a.base_len[b] : old_len;
+    const int kept = a.keep[b] + a.keep_add;
+    int nbo = ceil_div(max(old_len, 0), bs), nbn = nbo;
+    if (kept < 0 || kept > a.Kp1 || base < 0 || base > old_len || old_len < 0) {
+      bad = 1;
+    } else {
+      nbn = ceil_div(base + kept, bs);
+      if (nbo > a.max_blocks || nbn > a.max_blocks) bad = 1;
+    }
+    s_nbo[b] = min(nbo, a.max_blocks);
+    s_nbn[b] = nbn;
+    s_kept[b] = kept;
+    cnt.x += max(0, nbo - nbn);
+    cnt.y += max(0, nbn - nbo);
+    cnt.z += kept;
+  }
   __syncthreads();
   // Every covered table entry must be a valid block id: one coalesced pass
   // over the flattened [B, max_blocks] table, loads batched per thread.
-  int bad = 0;
   const int nent = a.B * a.max_blocks;  // < 2^31, checked on the host
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;
   for (int e0 = threadIdx.x; e0 < nent; e0 += kBatch * blockDim.x) {
     int v[kBatch];
 #pragma unroll
@@ -85,31 +112,14 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
       const int e = e0 + k * blockDim.x;
       if (e < nent) {
         const int b = e / a.max_blocks, i = e - b * a.max_blocks;
-        if (i < s_nb[b] && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
+        if (i < s_nbo[b] && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
       }
     }
   }
-  // Each thread owns a contiguous run of sequences.
-  const int per = ceil_div(a.B, blockDim.x);
-  const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
-  int nfree = 0, nalloc = 0, nkept = 0;
-  for (int b = b0; b < b1; ++b) {
-    const int old_len = a.seq_lens[b];
-    const int base = a.base_len ? a.base_len[b] : old_len;
-    const int kept = a.keep[b] + a.keep_add;
-    if (kept < 0 || kept > a.Kp1 || base < 0 || base > old_len || old_len < 0) { bad = 1; continue; }
-    const int nb_old = ceil_div(old_len, bs), nb_new = ceil_div(base + kept, bs);
-    if (nb_old > a.max_blocks || nb_new > a.max_blocks) { bad = 1; continue; }
-    nfree += max(0, nb_old - nb_new);
-    nalloc += max(0, nb_new - nb_old);
-    nkept += kept;
-  }
   if (bad) atomicOr(&s_bad, 1);
-  int F, A, KT;
-  const int fpre = block_excl_scan(nfree, &F);
-  const int apre = block_excl_scan(nalloc, &A);
-  const int kpre = block_excl_scan(nkept, &KT);
-  const int ft = *a.free_top;
+  int3 tot;
+  const int3 pre = block_excl_scan3(cnt, &tot);  // its barriers also publish s_bad
+  const int F = tot.x, A = tot.y, KT = tot.z, ft = s_ft;
   if (threadIdx.x == 0) {
     if (s_bad || ft < 0 || ft > a.num_blocks || ft + F > a.num_blocks) s_code = SPEC_EINVAL;
     else if (ft + F < A) s_code = SPEC_ENOBLOCKS;
@@ -117,12 +127,11 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
   __syncthreads();
   // Blocks handed out come from stack positions [ft + F - A, ft + F); the
   // ones below ft must be valid ids (the pushed ones were checked above).
-  if (s_code == 0) {
+  if (s_code == 0)
     for (int p = max(0, ft + F - A) + threadIdx.x; p < ft; p += blockDim.x) {
       const int x = a.free_stack[p];
       if (x < 0 || x >= a.num_blocks) atomicOr(&s_bad, 1);
     }
-  }
   __syncthreads();
   if (threadIdx.x == 0 && s_code == 0 && s_bad) s_code = SPEC_EINVAL;
   __syncthreads();
@@ -131,96 +140,91 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
     return;
   }
   // Frees: push table tails in sequence order.
-  int fpos = ft + fpre;
+  int fpos = ft + pre.x;
   for (int b = b0; b < b1; ++b) {
-    const int old_len = a.seq_lens[b];
-    const int base = a.base_len ? a.base_len[b] : old_len;
-    const int kept = a.keep[b] + a.keep_add;
-    const int nb_old = ceil_div(old_len, bs), nb_new = ceil_div(base + kept, bs);
     int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-    for (int i = nb_new; i < nb_old; ++i) {
+    for (int i = s_nbn[b]; i < s_nbo[b]; ++i) {
       a.free_stack[fpos++] = tab[i];
       tab[i] = -1;
     }
   }
   __syncthreads();
-  // Allocations: pop from the top in sequence order; then lengths, offsets.
+  // Allocations: pop from the top in sequence order; lengths and offsets.
   const int top = ft + F;
-  int k = apre, off = kpre;
+  int k = pre.y, off = pre.z;
   for (int b = b0; b < b1; ++b) {
-    const int old_len = a.seq_lens[b];
-    const int base = a.base_len ? a.base_len[b] : old_len;
-    const int kept = a.keep[b] + a.keep_add;
-    const int nb_old = ceil_div(old_len, bs), nb_new = ceil_div(base + kept, bs);
     int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-    for (int i = nb_old; i < nb_new; ++i) tab[i] = a.free_stack[top - 1 - (k++)];
+    for (int i = s_nbo[b]; i < s_nbn[b]; ++i) tab[i] = a.free_stack[top - 1 - (k++)];
     if (a.hid_off) a.hid_off[b] = off;
-    off += kept;
+    off += s_kept[b];
   }
-  __syncthreads();  // every read of seq_lens / base_len is done
+  // New lengths: base + kept (base read above for the checks; read again
+  // here because base_len may be the same array as seq_lens).
+  __syncthreads();
   for (int b = b0; b < b1; ++b) {
     const int base = a.base_len ? a.base_len[b] : a.seq_lens[b];
-    a.seq_lens[b] = base + a.keep[b] + a.keep_add;
+    a.seq_lens[b] = base + s_kept[b];
   }
   if (threadIdx.x == 0) {
     *a.free_top = top - A;
     if (a.hid_off) a.hid_off[a.B] = KT;
   }
+  grid_dependents_launch();
 }
 
-// Copy of kept token rows: a grid-stride loop over (token, part) items; the
-// staged K/V segments of a token are split into kCopyParts parts.
+// Copy of kept token rows: a grid-stride loop of warps over (token, segment)
+// items. A segment is one (layer, K|V) slice of a token's staged row
+// (kv_heads * head_dim * 2 bytes, contiguous in both stage and pool); the
+// hidden row is cut into pieces of the same size after the K/V segments.
 __global__ void __launch_bounds__(kCopyThreads) commit_copy_kernel(CommitArgs a) {
   grid_dependency_wait();
   if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;
-  const int nitems = a.B * a.Kp1 * kCopyParts;
-  const int nseg = a.layers * 2;
-  const int segs_per = (nseg + kCopyParts - 1) / kCopyParts;
-  const int vps = a.seg_bytes / 16;  // vectors per segment
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int tok = item / kCopyParts, part = item - tok * kCopyParts;
+  const int lane = threadIdx.x & 31;
+  const int nseg = a.kv_stage ? a.layers * 2 : 0;
+  const int piece = a.kv_stage ? a.seg_bytes : 2048;
+  const int nhid = a.hid_stage ? (a.hid_bytes + piece - 1) / piece : 0;
+  const int per_tok = nseg + nhid;
+  const long long nitems = (long long)a.B * a.Kp1 * per_tok;
+  const long long gw = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long item = gw; item < nitems; item += nw) {
+    const int tok = (int)(item / per_tok), sidx = (int)(item - (long long)tok * per_tok);
     const int b = tok / a.Kp1, i = tok - b * a.Kp1;
     const int kept = a.keep[b] + a.keep_add;
     if (i >= kept) continue;
-    const int pos = a.seq_lens[b] - kept + i;  // base_len + i
-    if (a.kv_stage) {
+    const uint4* src;
+    uint4* dst;
+    int nvec;
+    if (sidx < nseg) {
+      const int pos = a.seq_lens[b] - kept + i;  // base_len + i
       const int blk = a.tables[(size_t)b * a.max_blocks + pos / a.block_size];
       const int slot = pos % a.block_size;
-      const int s0 = part * segs_per, s1 = min(nseg, s0 + segs_per);
-      const int nvec = max(0, s1 - s0) * vps;
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.kv_stage + (((size_t)b * a.Kp1 + i) * nseg + s0) * (size_t)a.seg_bytes);
-      for (int v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * 4) {
-        uint4 r[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = v0 + u * blockDim.x;
-          if (v < nvec) r[u] = __ldcs(src + v);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = v0 + u * blockDim.x;
-          if (v < nvec) {
-            const int seg = s0 + v / vps, e = v - (seg - s0) * vps;
-            uint4* dst = reinterpret_cast<uint4*>(
-                a.kv_pool + (((size_t)blk * nseg + seg) * a.block_size + slot) * (size_t)a.seg_bytes);
-            __stcs(dst + e, r[u]);
-          }
-        }
-      }
+      src = reinterpret_cast<const uint4*>(a.kv_stage +
+                                           (((size_t)b * a.Kp1 + i) * nseg + sidx) * a.seg_bytes);
+      dst = reinterpret_cast<uint4*>(
+          a.kv_pool + (((size_t)blk * nseg + sidx) * a.block_size + slot) * (size_t)a.seg_bytes);
+      nvec = a.seg_bytes / 16;
+    } else {
+      const int h = sidx - nseg;
+      const int off = h * piece, len = min(piece, a.hid_bytes - off);
+      src = reinterpret_cast<const uint4*>(a.hid_stage + ((size_t)b * a.Kp1 + i) * a.hid_bytes + off);
+      dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(a.hid_off[b] + i) * a.hid_bytes + off);
+      nvec = len / 16;
     }
-    if (a.hid_stage && part == 0) {
-      const int hv = a.hid_bytes / 16;
-      const uint4* src =
-          reinterpret_cast<const uint4*>(a.hid_stage + ((size_t)b * a.Kp1 + i) * a.hid_bytes);
-      uint4* dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(a.hid_off[b] + i) * a.hid_bytes);
-      for (int v = threadIdx.x; v < hv; v += blockDim.x) __stcs(dst + v, __ldcs(src + v));
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) r[u] = __ldcs(src + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) __stcs(dst + v0 + 32 * u, r[u]);
     }
   }
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)a.B * sizeof(int);
+  const size_t smem = 3 * (size_t)a.B * sizeof(int);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(commit_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
@@ -228,8 +232,7 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
   cudaError_t e = launch_pdl(commit_plan_kernel, dim3(1), dim3(kPlanThreads), smem, st, a);
   if (e != cudaSuccess) return e;
   if (a.B > 0 && a.Kp1 > 0 && (a.kv_stage || a.hid_stage)) {
-    const int items = a.B * a.Kp1 * kCopyParts;
-    e = launch_pdl(commit_copy_kernel, dim3(min(items, 148 * 4)), dim3(kCopyThreads), 0, st, a);
+    e = launch_pdl(commit_copy_kernel, dim3(148 * 4), dim3(kCopyThreads), 0, st, a);
   }
   return e;
 }

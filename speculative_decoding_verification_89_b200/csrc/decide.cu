@@ -28,11 +28,11 @@ namespace specv {
 
 constexpr int kMaxRows = 2 * SPEC_MAX_K + 1;
 constexpr int kWarps = kDecideThreads / 32;
-constexpr int kUnroll = 4;  // residual tiles in flight per warp
+constexpr int kUnroll = 8;  // residual tiles in flight per warp
 
 int decide_split(int B, int V) {
   const int nrt = residual_tiles(V);
-  int s = (3 * 148) / (B > 0 ? B : 1);  // one wave of about three CTAs per SM
+  int s = (4 * 148) / (B > 0 ? B : 1);  // one wave of about four CTAs per SM
   if (s > kMaxSplit) s = kMaxSplit;
   if (s > nrt) s = nrt;
   return s < 1 ? 1 : s;
@@ -148,6 +148,7 @@ __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const Pr
       if (lane == 0 && tb + u < t1) out[tb + u] = v;
     }
   }
+  if (lane == 0) __threadfence();  // the writers publish their tile sums
 }
 
 // Last CTA: prefix the tile sums, locate u' * Z, rescan that tile.
@@ -246,7 +247,6 @@ __device__ bool draw_token(const DecideCommon& c, int b, int sp, const T* prow, 
   double* tsum = c.rsum + (size_t)b * nrt;
   residual_tile_sums<T>(prow, qrow, c.V, kp, kq, min(nrt, sp * chunk), min(nrt, (sp + 1) * chunk),
                         tsum);
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = (atomicAdd(&c.counters[b], 1) == c.nsplit - 1);
   __syncthreads();
@@ -257,7 +257,6 @@ __device__ bool draw_token(const DecideCommon& c, int b, int sp, const T* prow, 
     // Residual mass zero as computed (p == q): draw from p instead.
     __syncthreads();
     residual_tile_sums<T>(prow, nullptr, c.V, kp, kq, 0, nrt, tsum);
-    __threadfence();
     __syncthreads();
     tok = residual_pick<T>(prow, nullptr, c.V, kp, kq, tsum, nrt, u, sh_pre, Z_out);
   }
@@ -270,7 +269,7 @@ __device__ bool draw_token(const DecideCommon& c, int b, int sp, const T* prow, 
 // ---------------------------------------------------------------------------
 // Per-sequence state of the finish kernels
 // ---------------------------------------------------------------------------
-constexpr int kFinThreads = 512;
+constexpr int kFinThreads = 1024;
 constexpr int kFinWarps = kFinThreads / 32;
 constexpr long long kNaNBits = 0x7ff8000000000000ll;
 __device__ __forceinline__ double dnan() { return __longlong_as_double(kNaNBits); }
@@ -289,7 +288,8 @@ template <typename Want>
 __device__ void finish_rows(SeqShared& sh, const Partial* part, int ntiles, int row0, int nrows,
                             Want want, bool greedy, float chi, RowFinal* fin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < nrows; r += kFinWarps) {
+  if (warp == kFinWarps - 1) return;  // the accept warp
+  for (int r = warp; r < nrows; r += kFinWarps - 1) {
     if (!want(r)) {
       if (lane == 0) { sh.ok[r] = 1; sh.m[r] = 0.f; sh.M[r] = 0; sh.L[r] = 0; sh.amax[r] = -1; }
       continue;
@@ -312,28 +312,52 @@ __device__ __forceinline__ const T* row_ptr(const unsigned char* base, long long
   return reinterpret_cast<const T*>(base + row * ld_bytes);
 }
 
-// One speculative check on n positions (warp 0). Target row j: tp(j) with log2
-// partition sh.M + sh.L at index j; draft law of position j: row dp(j) with
-// log2 partition dlt(j). Sets sh.a (first rejection, n if none) and sh.bad (a
-// draft id outside [0, V)). Writes p_j(x_j), q_j(x_j) to diag_p / diag_q.
+// Logits of the drafted tokens for the first 32 positions, fetched by the
+// accept warp while the other warps combine the rows.
+struct AcceptPre {
+  int x;        // draft id of position lane (or -1 past n)
+  float lt, ld; // target / draft logit at x
+};
+template <typename T, typename TP, typename DP>
+__device__ __forceinline__ AcceptPre accept_prefetch(int n, int V, bool greedy,
+                                                     const int32_t* drafts, TP tp, DP dp) {
+  const int lane = threadIdx.x & 31;
+  AcceptPre a{-1, 0.f, 0.f};
+  if (lane < n) {
+    a.x = drafts[lane];
+    if (!greedy && a.x >= 0 && a.x < V) {
+      a.lt = load_elem(tp(lane) + a.x);
+      a.ld = load_elem(dp(lane) + a.x);
+    }
+  }
+  return a;
+}
+
+// One speculative check on n positions (one warp). Target row j: tp(j) with
+// log2 partition sh.M + sh.L at index j; draft law of position j: row dp(j)
+// with log2 partition dlt(j). Sets sh.a (first rejection, n if none) and
+// sh.bad (a draft id outside [0, V)). Writes p_j(x_j), q_j(x_j) to diag_p /
+// diag_q. Positions below 32 use the prefetched logits.
 template <typename T, typename TP, typename DP, typename DS>
 __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const DecideCommon& c,
                             int b, bool greedy, double cd, const int32_t* drafts, TP tp, DP dp,
-                            DS dlt, double* diag_p, double* diag_q) {
+                            DS dlt, double* diag_p, double* diag_q, const AcceptPre& pre) {
   const int lane = threadIdx.x & 31;
   int a = n, bad = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + lane;
     bool acc = true, badj = false;
     if (j < n) {
-      const int x = drafts[j];
+      const int x = j0 == 0 ? pre.x : drafts[j];
       if (x < 0 || x >= c.V) {
         badj = true;
       } else if (greedy) {
         acc = (x == sh.amax[j]);
       } else {
-        const double lp = (double)load_elem(tp(j) + x) * cd - (sh.M[j] + sh.L[j]);
-        const double lq = (double)load_elem(dp(j) + x) * cd - dlt(j);
+        const float lt = j0 == 0 ? pre.lt : load_elem(tp(j) + x);
+        const float ld = j0 == 0 ? pre.ld : load_elem(dp(j) + x);
+        const double lp = (double)lt * cd - (sh.M[j] + sh.L[j]);
+        const double lq = (double)ld * cd - dlt(j);
         const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(pos0 + j),
                                       (uint32_t)stage).x;
         acc = (double)u < exp2(lp - lq);
@@ -377,17 +401,20 @@ __global__ void __launch_bounds__(kFinThreads) chain_finish_kernel(ChainDecideAr
   };
   if (!tvalid) { fail(); grid_dependents_launch(); return; }
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
-  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
-              sc.hi, c.fin);
-  __syncthreads();
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   auto tp = [&](int j) { return row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + j); };
   auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
-  if (threadIdx.x < 32)
+  const bool accept_warp = (threadIdx.x >> 5) == kFinWarps - 1;
+  AcceptPre pre{-1, 0.f, 0.f};
+  if (accept_warp) pre = accept_prefetch<T>(K, c.V, greedy, drafts, tp, dp);
+  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
+              sc.hi, c.fin);
+  __syncthreads();
+  if (accept_warp)
     accept_scan<T>(sh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
                    diag && !greedy ? diag + 2 * K + 1 : nullptr,
-                   diag && !greedy ? diag + 3 * K + 1 : nullptr);
+                   diag && !greedy ? diag + 3 * K + 1 : nullptr, pre);
   __syncthreads();
   if (sh.bad || !rows_ok(sh, per)) { fail(); grid_dependents_launch(); return; }
   const int a = sh.a;
@@ -406,7 +433,7 @@ __global__ void __launch_bounds__(kFinThreads) chain_finish_kernel(ChainDecideAr
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDecideThreads) chain_draw_kernel(ChainDecideArgs A) {
+__global__ void __launch_bounds__(kDecideThreads, 4) chain_draw_kernel(ChainDecideArgs A) {
   grid_dependency_wait();
   extern __shared__ double dyn_pre[];
   const DecideCommon& c = A.c;
@@ -486,18 +513,21 @@ __global__ void __launch_bounds__(kFinThreads) hier1_finish_kernel(HierDecideArg
   };
   if (!tvalid || w < 0 || w >= Ni) { fail(); grid_dependents_launch(); return; }
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
-  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
-              sc.hi, c.fin);
-  __syncthreads();
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   const long long row0 = (long long)b * S + w;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, row0 + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_d, A.ld, row0 + j); };
   auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
-  if (threadIdx.x < 32)
+  const bool accept_warp = (threadIdx.x >> 5) == kFinWarps - 1;
+  AcceptPre pre{-1, 0.f, 0.f};
+  if (accept_warp) pre = accept_prefetch<T>(K, c.V, greedy, drafts, tp, dp);
+  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
+              sc.hi, c.fin);
+  __syncthreads();
+  if (accept_warp)
     accept_scan<T>(sh, K, w, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
                    diag && !greedy ? diag + 2 * K + 1 : nullptr,
-                   diag && !greedy ? diag + 3 * K + 1 : nullptr);
+                   diag && !greedy ? diag + 3 * K + 1 : nullptr, pre);
   __syncthreads();
   if (sh.bad || !rows_ok(sh, per)) { fail(); grid_dependents_launch(); return; }
   const int a = sh.a;
@@ -518,7 +548,7 @@ __global__ void __launch_bounds__(kFinThreads) hier1_finish_kernel(HierDecideArg
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDecideThreads) hier1_draw_kernel(HierDecideArgs A) {
+__global__ void __launch_bounds__(kDecideThreads, 4) hier1_draw_kernel(HierDecideArgs A) {
   grid_dependency_wait();
   extern __shared__ double dyn_pre[];
   const DecideCommon& c = A.c;
@@ -570,16 +600,20 @@ __global__ void __launch_bounds__(kFinThreads) hier2_finish_kernel(HierDecideArg
   const bool greedy = (Tb == 0.0f);
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
   double* diag = c.diag ? c.diag + (size_t)b * (4 * K + 3 * S + 1) + (4 * K + 2) : nullptr;
-  finish_rows(sh, c.part, c.ntiles, b * S, W + 1, [&](int) { return true; }, greedy, sc.hi, c.fin);
-  __syncthreads();
   const int32_t* wtok = A.win_tok + (size_t)b * WC;
   const double* wst = A.win_stat + (size_t)b * WC * 2;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_f, A.ld, (long long)b * S + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, (long long)b * S + j); };
   auto dl = [&](int j) { return wst[2 * j] * sc.d + wst[2 * j + 1] * kLog2e; };
-  if (threadIdx.x < 32)
+  const bool accept_warp = (threadIdx.x >> 5) == kFinWarps - 1;
+  AcceptPre pre{-1, 0.f, 0.f};
+  if (accept_warp) pre = accept_prefetch<T>(W, c.V, greedy, wtok, tp, dp);
+  finish_rows(sh, c.part, c.ntiles, b * S, W + 1, [&](int) { return true; }, greedy, sc.hi, c.fin);
+  __syncthreads();
+  if (accept_warp)
     accept_scan<T>(sh, W, 0, 2, c, b, greedy, sc.d, wtok, tp, dp, dl,
-                   diag && !greedy ? diag + S : nullptr, diag && !greedy ? diag + 2 * S - 1 : nullptr);
+                   diag && !greedy ? diag + S : nullptr, diag && !greedy ? diag + 2 * S - 1 : nullptr,
+                   pre);
   __syncthreads();
   if (sh.bad || !rows_ok(sh, W + 1)) {
     if (threadIdx.x == 0) {
@@ -610,7 +644,7 @@ __global__ void __launch_bounds__(kFinThreads) hier2_finish_kernel(HierDecideArg
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDecideThreads) hier2_draw_kernel(HierDecideArgs A) {
+__global__ void __launch_bounds__(kDecideThreads, 4) hier2_draw_kernel(HierDecideArgs A) {
   grid_dependency_wait();
   extern __shared__ double dyn_pre[];
   const DecideCommon& c = A.c;

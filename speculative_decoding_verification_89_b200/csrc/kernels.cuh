@@ -82,11 +82,33 @@ struct RsBuffers {
 };
 
 // Combine a row's tile partials (warp-cooperative; result valid in lane 0).
+// Up to 4*32 tiles are read once into registers; longer rows loop.
 __device__ __forceinline__ RowFinal combine_row(const Partial* p, int ntiles, bool greedy,
                                                 float chi, int lane) {
+  constexpr int kReg = 4;
+  float pm[kReg];
+  double ps[kReg];
+  int pi[kReg];
+#pragma unroll
+  for (int k = 0; k < kReg; ++k) {
+    const int t = lane + 32 * k;
+    if (t < ntiles) {
+      const Partial q = p[t];
+      pm[k] = q.m;
+      pi[k] = q.idx;
+      ps[k] = q.s;
+    } else {
+      pm[k] = -INFINITY;
+      pi[k] = 0x7fffffff;
+      ps[k] = 0.0;
+    }
+  }
   float mv = -INFINITY;
   int mi = 0x7fffffff;
-  for (int t = lane; t < ntiles; t += 32) {
+#pragma unroll
+  for (int k = 0; k < kReg; ++k)
+    if (pm[k] > mv || (pm[k] == mv && pi[k] < mi)) { mv = pm[k]; mi = pi[k]; }
+  for (int t = lane + 32 * kReg; t < ntiles; t += 32) {
     const float m = p[t].m;
     const int i = p[t].idx;
     if (m > mv || (m == mv && i < mi)) { mv = m; mi = i; }
@@ -102,7 +124,10 @@ __device__ __forceinline__ RowFinal combine_row(const Partial* p, int ntiles, bo
   if (ok && !greedy) {
     f.M = (double)__fmul_rn(mv, chi);
     double s = 0.0;
-    for (int t = lane; t < ntiles; t += 32) {
+#pragma unroll
+    for (int k = 0; k < kReg; ++k)
+      if (ps[k] != 0.0) s += ps[k] * exp2((double)__fmul_rn(pm[k], chi) - f.M);
+    for (int t = lane + 32 * kReg; t < ntiles; t += 32) {
       const double st = p[t].s;
       if (st != 0.0) s += st * exp2((double)__fmul_rn(p[t].m, chi) - f.M);
     }
