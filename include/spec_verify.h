@@ -78,7 +78,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 
 /* Limits checked on the host. */
 #define SPEC_MAX_K 256           /* drafts per sequence per call      */
-#define SPEC_MAX_V (1 << 22)     /* vocabulary size                   */
+#define SPEC_MAX_V (1 << 21)     /* vocabulary size                   */
 #define SPEC_MAX_COMMIT_B 16384  /* sequences per paged commit        */
 
 /* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
@@ -110,10 +110,7 @@ const char* spec_status_string(int status);
  *               Z of the final draw (sum max(0, p_a - q_a), or sum p_K for the
  *               bonus). NaN for greedy sequences.
  * ws, ws_bytes: workspace of at least spec_workspace_bytes(B, K, V, dtype, 0)
- *               bytes, 256-byte aligned, zero-filled before its first use (it
- *               holds self-resetting arrival counters that every completed
- *               call leaves at zero; zero it again after a device error or
- *               before using it for other sizes).
+ *               bytes, 256-byte aligned. No initial contents are needed.
  * Equivalent to spec_chain_row_stats followed by spec_chain_decide.
  * ------------------------------------------------------------------------- */
 int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf,
@@ -244,7 +241,7 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
  *   - The first call on a device looks the array's device address up with
  *     that device current; make that first call outside any stream capture.
  *   - All calls share the one array and it keeps the previous call's
- *     contents; each call clears what must start at zero. Calls that overlap
+ *     contents (no call reads what an earlier one left). Calls that overlap
  *     on the GPU (several streams or threads) race on it and must not be made.
  * ------------------------------------------------------------------------- */
 #define SPEC_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -21,12 +21,12 @@ int stat_tiles(int V, int dtype) {
 }
 
 struct Layout {
-  size_t part, fin, dec, rsum, counters, total;
+  size_t part, fin, total;
   long long rows;
 };
 
-// Workspace: tile partials for the largest row set, residual tile sums and
-// the per-sequence arrival counters, each 256-byte aligned.
+// Workspace: final row statistics and tile partials for the largest row set,
+// each region 256-byte aligned.
 bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   if (B < 0 || K < 0 || K > SPEC_MAX_K || V < 1 || V > SPEC_MAX_V) return false;
   if (dtype != SPEC_F32 && dtype != SPEC_BF16) return false;
@@ -34,14 +34,10 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   const long long per = Ni > 0 ? (long long)std::max(2 * K + 1, Ni + K + 1) : 2LL * K + 1;
   const long long rows = (long long)B * per;
   if (rows * stat_tiles(V, dtype) >= (1LL << 31)) return false;  // 32-bit item indices
-  // Counters first, so a workspace zeroed once keeps them zero across calls.
   L->rows = rows;
-  L->counters = 0;
-  L->dec = align_up((size_t)std::max(B, 1) * sizeof(int));
-  L->fin = L->dec + align_up((size_t)std::max(B, 1) * sizeof(SeqDecision));
-  L->part = L->fin + align_up((size_t)rows * sizeof(RowFinal));
-  L->rsum = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
-  L->total = L->rsum + align_up((size_t)B * residual_tiles(V) * sizeof(double));
+  L->fin = 0;
+  L->part = align_up((size_t)rows * sizeof(RowFinal));
+  L->total = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
   return true;
 }
 
@@ -78,11 +74,9 @@ ChainCheck check_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t
   return c;
 }
 
-RsBuffers rs_buffers(void* ws, const Layout& L, int B) {
+RsBuffers rs_buffers(void* ws, const Layout& L) {
   RsBuffers b;
   b.part = reinterpret_cast<Partial*>((char*)ws + L.part);
-  b.seq_cnt = reinterpret_cast<int*>((char*)ws + L.counters);
-  b.nseq = B;
   return b;
 }
 
@@ -103,18 +97,12 @@ DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_to
   c.part = reinterpret_cast<const Partial*>((char*)ws + L.part);
   c.ntiles = stat_tiles(V, dtype);
   c.fin = reinterpret_cast<RowFinal*>((char*)ws + L.fin);
-  c.dec = reinterpret_cast<SeqDecision*>((char*)ws + L.dec);
-  c.rsum = reinterpret_cast<double*>((char*)ws + L.rsum);
-  c.counters = reinterpret_cast<int*>((char*)ws + L.counters);
-  c.nsplit = decide_split(B, V);
   c.diag = diag;
   c.status = dev_status;
   return c;
 }
 
 }  // namespace
-
-size_t specv::workspace_counter_bytes(int B) { return align_up((size_t)std::max(B, 1) * sizeof(int)); }
 
 #pragma GCC visibility push(default)
 extern "C" {
@@ -152,7 +140,7 @@ int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64
   rows.ld_drf = ld_drf * es;
   rows.temperature = temperature;
   rows.K = K;
-  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, ck.L, B),
+  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, ck.L),
                                       dev_status, (cudaStream_t)stream));
 }
 
@@ -214,7 +202,7 @@ int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64
   const int es = elem_size(dtype);
   const int S = Ni + K + 1;
   cudaStream_t st = (cudaStream_t)stream;
-  const RsBuffers rsb = rs_buffers(ws, L, B);
+  const RsBuffers rsb = rs_buffers(ws, L);
 
   HierDecideArgs a;
   a.c = common_args(dtype, B, K, V, draft_tok, temperature, seed, seq_id, round, diag, dev_status,

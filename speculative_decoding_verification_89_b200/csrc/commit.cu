@@ -96,23 +96,21 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
     cnt.z += kept;
   }
   __syncthreads();
-  // Every covered table entry must be a valid block id: one coalesced pass
-  // over the flattened [B, max_blocks] table, loads batched per thread.
-  const int nent = a.B * a.max_blocks;  // < 2^31, checked on the host
-  constexpr int kBatch = 16;
-  for (int e0 = threadIdx.x; e0 < nent; e0 += kBatch * blockDim.x) {
-    int v[kBatch];
+  // Every covered table entry must be a valid block id: a warp per sequence,
+  // its lanes over the table entries, loads batched.
+  {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    constexpr int kBatch = 8;
+    for (int b = warp; b < a.B; b += nwarps) {
+      const int nb = s_nbo[b];
+      const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+      for (int i0 = lane; i0 < nb; i0 += 32 * kBatch) {
+        int v[kBatch];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int e = e0 + k * blockDim.x;
-      v[k] = e < nent ? a.tables[e] : 0;
-    }
+        for (int k = 0; k < kBatch; ++k) v[k] = (i0 + 32 * k < nb) ? tab[i0 + 32 * k] : 0;
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int e = e0 + k * blockDim.x;
-      if (e < nent) {
-        const int b = e / a.max_blocks, i = e - b * a.max_blocks;
-        if (i < s_nbo[b] && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
+        for (int k = 0; k < kBatch; ++k)
+          if (i0 + 32 * k < nb && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
       }
     }
   }
@@ -172,26 +170,49 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
   grid_dependents_launch();
 }
 
-// Copy of kept token rows: a grid-stride loop of warps over (token, segment)
-// items. A segment is one (layer, K|V) slice of a token's staged row
-// (kv_heads * head_dim * 2 bytes, contiguous in both stage and pool); the
-// hidden row is cut into pieces of the same size after the K/V segments.
+// Copy of kept token rows. Every CTA scans the kept counts (the planner has
+// checked them) so kept rows are numbered 0..KT-1; warps then stride over
+// (kept row, segment) items. A segment is one (layer, K|V) slice of a token's
+// staged row (kv_heads * head_dim * 2 bytes, contiguous in both stage and
+// pool); the hidden row is cut into pieces of the same size after them.
 __global__ void __launch_bounds__(kCopyThreads) commit_copy_kernel(CommitArgs a) {
   grid_dependency_wait();
-  if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;
-  const int lane = threadIdx.x & 31;
+  extern __shared__ int s_off[];  // [B + 1] exclusive scan of kept rows
+  if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;  // uniform
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    int carry = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < a.B ? a.keep[b] + a.keep_add : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b < a.B) s_off[b] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_off[a.B] = carry;
+  }
+  __syncthreads();
+  const int KT = s_off[a.B];
   const int nseg = a.kv_stage ? a.layers * 2 : 0;
   const int piece = a.kv_stage ? a.seg_bytes : 2048;
   const int nhid = a.hid_stage ? (a.hid_bytes + piece - 1) / piece : 0;
   const int per_tok = nseg + nhid;
-  const long long nitems = (long long)a.B * a.Kp1 * per_tok;
-  const long long gw = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long item = gw; item < nitems; item += nw) {
-    const int tok = (int)(item / per_tok), sidx = (int)(item - (long long)tok * per_tok);
-    const int b = tok / a.Kp1, i = tok - b * a.Kp1;
-    const int kept = a.keep[b] + a.keep_add;
-    if (i >= kept) continue;
+  const int nitems = KT * per_tok;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int item = blockIdx.x * (blockDim.x >> 5) + warp; item < nitems; item += nw) {
+    const int k = item / per_tok, sidx = item - k * per_tok;
+    int lo = 0, hi = a.B - 1;  // the sequence b with s_off[b] <= k < s_off[b + 1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= k) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo, i = k - s_off[b];
+    const int kept = s_off[b + 1] - s_off[b];
     const uint4* src;
     uint4* dst;
     int nvec;
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__(kCopyThreads) commit_copy_kernel(CommitArgs a)
       const int h = sidx - nseg;
       const int off = h * piece, len = min(piece, a.hid_bytes - off);
       src = reinterpret_cast<const uint4*>(a.hid_stage + ((size_t)b * a.Kp1 + i) * a.hid_bytes + off);
-      dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(a.hid_off[b] + i) * a.hid_bytes + off);
+      dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(s_off[b] + i) * a.hid_bytes + off);
       nvec = len / 16;
     }
     for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
@@ -232,7 +253,12 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
   cudaError_t e = launch_pdl(commit_plan_kernel, dim3(1), dim3(kPlanThreads), smem, st, a);
   if (e != cudaSuccess) return e;
   if (a.B > 0 && a.Kp1 > 0 && (a.kv_stage || a.hid_stage)) {
-    e = launch_pdl(commit_copy_kernel, dim3(148 * 4), dim3(kCopyThreads), 0, st, a);
+    const size_t csmem = ((size_t)a.B + 1) * sizeof(int);
+    if (csmem > 48 * 1024 &&
+        cudaFuncSetAttribute(commit_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)csmem) != cudaSuccess)
+      return cudaGetLastError();
+    e = launch_pdl(commit_copy_kernel, dim3(148 * 4), dim3(kCopyThreads), csmem, st, a);
   }
   return e;
 }

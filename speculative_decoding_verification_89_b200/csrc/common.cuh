@@ -42,8 +42,6 @@ static_assert(kTileBytes % 512 == 0, "a tile is a whole number of warp-wide 16-b
 
 // Residual tiles: 32 lanes x 8 elements.
 constexpr int kResTile = 256;
-constexpr int kDecideThreads = 256;
-constexpr int kMaxSplit = 32;    // CTAs sharing one residual row pair
 
 // Per (row, tile) statistics: the tile's largest raw logit m, its first index,
 // and s = sum over the tile of 2^(l*c - M), c = log2(e) / T, with the exact
@@ -227,6 +225,29 @@ static cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
+}
+
+// Same, for a grid of thread-block clusters of `cluster` CTAs along x.
+template <typename Kern, typename... Args>
+static cudaError_t launch_pdl_cluster(Kern kern, dim3 grid, dim3 block, size_t smem,
+                                      cudaStream_t st, unsigned cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) cudaGetLastError();
   return e;

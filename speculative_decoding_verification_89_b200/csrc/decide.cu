@@ -11,32 +11,31 @@
 // "Dynamische Verifizierungsrichtlinie" (N_i tentatively accepted tokens
 // before the final-layer check).
 //
-// Two launches per check. (1) finish: one CTA per sequence combines the tile
-// partials of its rows (a warp per row), runs the accept test on all
-// positions (a lane per position, ballot for the first rejection) and, for
-// greedy sequences, writes the outputs. (2) draw: grid (nsplit, B); the
-// residual row pair of each sampled sequence is split over nsplit CTAs, each
-// writing tile sums of the weights; the last CTA to arrive (atomic counter,
-// no waiting) prefixes the tile sums, finds the tile holding u' * Z, rescans
-// that one tile and writes the outputs.
+// One launch per check: a thread-block cluster of kCluster CTAs per sequence.
+// The CTAs combine the tile partials of the sequence's rows (a warp per row)
+// into the leader CTA's shared memory (distributed shared memory), meet at a
+// cluster barrier, each run the accept test on all positions (a lane per
+// position, ballot for the first rejection), split the residual row pair
+// between them and write their tile sums into the leader, meet again, and the
+// leader prefixes the tile sums, finds the tile holding u' * Z, rescans that
+// one tile and writes the outputs. No atomics, no spinning, no second launch.
 #include <climits>
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace specv {
 
-constexpr int kMaxRows = 2 * SPEC_MAX_K + 1;
-constexpr int kWarps = kDecideThreads / 32;
-constexpr int kUnroll = 8;  // residual tiles in flight per warp
+namespace cg = cooperative_groups;
 
-int decide_split(int B, int V) {
-  const int nrt = residual_tiles(V);
-  int s = (4 * 148) / (B > 0 ? B : 1);  // one wave of about four CTAs per SM
-  if (s > kMaxSplit) s = kMaxSplit;
-  if (s > nrt) s = nrt;
-  return s < 1 ? 1 : s;
-}
+constexpr int kMaxRows = 2 * SPEC_MAX_K + 1;
+constexpr int kCluster = 4;                  // CTAs per sequence
+constexpr int kDecThreads = 512;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kRowWarps = kDecWarps - 1;     // the last warp of a CTA serves the accept test
+constexpr int kUnroll = 4;                   // residual tiles in flight per warp
 
 // ---------------------------------------------------------------------------
 // Residual weights of 8 consecutive elements
@@ -124,12 +123,17 @@ __device__ __forceinline__ double lane_sum8(const float w[8]) {
   return (double)(c.x + c.y);
 }
 
-// Tile sums of the weights over residual tiles [t0, t1) (one CTA's share).
+
+// ---------------------------------------------------------------------------
+// Residual tile sums and the draw
+// ---------------------------------------------------------------------------
+// Tile sums of the weights over residual tiles [t0, t1), written to out
+// (the leader CTA's shared memory, possibly remote).
 template <typename T>
 __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const ProbCoef& kp,
                                    const ProbCoef& kq, int t0, int t1, double* out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int tb = t0 + warp * kUnroll; tb < t1; tb += kWarps * kUnroll) {
+  for (int tb = t0 + warp * kUnroll; tb < t1; tb += kDecWarps * kUnroll) {
     double s[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -148,29 +152,24 @@ __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const Pr
       if (lane == 0 && tb + u < t1) out[tb + u] = v;
     }
   }
-  if (lane == 0) __threadfence();  // the writers publish their tile sums
 }
 
-// Last CTA: prefix the tile sums, locate u' * Z, rescan that tile.
-// Returns, in every thread, the drawn token (-1 if the weights have no mass);
-// *Z_out gets Z.
+// Leader: given all tile sums in shared memory (tsum), prefix them in a fixed
+// order, locate u * Z, rescan that tile and return the drawn token in every
+// thread (-1 if the weights have no mass). *Z_out gets Z.
 template <typename T>
 __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef& kp,
-                             const ProbCoef& kq, const double* tsum_g, int nrt, float u,
-                             double* sh_pre, double* Z_out) {
+                             const ProbCoef& kq, const double* tsum, double* pre, int nrt,
+                             float u, double* Z_out) {
   __shared__ double s_Z;
   __shared__ int s_tile, s_tok;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double* sh_sum = sh_pre + nrt;  // second half of the dynamic buffer
-  for (int t = threadIdx.x; t < nrt; t += blockDim.x) sh_sum[t] = __ldcg(tsum_g + t);
-  __syncthreads();
-  // Exclusive prefix over tiles in a fixed order (warp 0: each lane owns a
-  // contiguous run of tiles).
   if (warp == 0) {
+    // Each lane owns a contiguous run of tiles; lane sums are scanned.
     const int per = (nrt + 31) / 32;
     const int a = min(nrt, lane * per), b = min(nrt, a + per);
     double run = 0.0;
-    for (int t = a; t < b; ++t) run += sh_sum[t];
+    for (int t = a; t < b; ++t) run += tsum[t];
     double incl = run;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -180,8 +179,8 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
     double c = __shfl_up_sync(0xffffffffu, incl, 1);
     if (lane == 0) c = 0.0;
     for (int t = a; t < b; ++t) {
-      sh_pre[t] = c;
-      c += sh_sum[t];
+      pre[t] = c;
+      c += tsum[t];
     }
     if (lane == 31) s_Z = incl;
     if (lane == 0) s_tile = -1;
@@ -193,7 +192,7 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
   const double target = (double)u * Z;
   // The last tile with mass whose prefix does not exceed the target.
   for (int t = threadIdx.x; t < nrt; t += blockDim.x)
-    if (sh_pre[t] <= target && sh_sum[t] > 0.0) atomicMax(&s_tile, t);
+    if (pre[t] <= target && tsum[t] > 0.0) atomicMax(&s_tile, t);
   __syncthreads();
   const int tile = s_tile < 0 ? 0 : s_tile;  // s_tile >= 0 whenever Z > 0
   if (warp == 0) {
@@ -208,7 +207,7 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
     }
     double excl = __shfl_up_sync(0xffffffffu, incl, 1);
     if (lane == 0) excl = 0.0;
-    const double start = sh_pre[tile] + excl;
+    const double start = pre[tile] + excl;
     int found = INT_MAX;
     if (start <= target) {
       double acc = start;
@@ -234,74 +233,60 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
   return s_tok;
 }
 
-// Residual / bonus draw of one sequence, split over the sequence's CTAs.
-// Every CTA writes the tile sums of its share; the last to arrive picks the
-// token. Returns false in the CTAs that are not last (they are done).
+// Leader, after the cluster's tile sums are in: the draw, with the fall-back
+// to p when the residual mass is zero as computed (p == q).
 template <typename T>
-__device__ bool draw_token(const DecideCommon& c, int b, int sp, const T* prow, const T* qrow,
-                           const ProbCoef& kp, const ProbCoef& kq, float u, double* sh_pre,
-                           int* tok_out, double* Z_out) {
-  __shared__ int s_last;
-  const int nrt = residual_tiles(c.V);
-  const int chunk = (nrt + c.nsplit - 1) / c.nsplit;
-  double* tsum = c.rsum + (size_t)b * nrt;
-  residual_tile_sums<T>(prow, qrow, c.V, kp, kq, min(nrt, sp * chunk), min(nrt, (sp + 1) * chunk),
-                        tsum);
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&c.counters[b], 1) == c.nsplit - 1);
-  __syncthreads();
-  if (!s_last) return false;
-  __threadfence();
-  int tok = residual_pick<T>(prow, qrow, c.V, kp, kq, tsum, nrt, u, sh_pre, Z_out);
+__device__ int leader_draw(const T* prow, const T* qrow, int V, const ProbCoef& kp,
+                           const ProbCoef& kq, double* tsum, double* pre, float u, double* Z) {
+  const int nrt = residual_tiles(V);
+  int tok = residual_pick<T>(prow, qrow, V, kp, kq, tsum, pre, nrt, u, Z);
   if (tok < 0 && qrow) {
-    // Residual mass zero as computed (p == q): draw from p instead.
     __syncthreads();
-    residual_tile_sums<T>(prow, nullptr, c.V, kp, kq, 0, nrt, tsum);
+    residual_tile_sums<T>(prow, nullptr, V, kp, kq, 0, nrt, tsum);
     __syncthreads();
-    tok = residual_pick<T>(prow, nullptr, c.V, kp, kq, tsum, nrt, u, sh_pre, Z_out);
+    tok = residual_pick<T>(prow, nullptr, V, kp, kq, tsum, pre, nrt, u, Z);
   }
-  __syncthreads();
-  if (threadIdx.x == 0) c.counters[b] = 0;
-  *tok_out = tok;
-  return true;
+  return tok;
 }
 
 // ---------------------------------------------------------------------------
-// Per-sequence state of the finish kernels
+// Row statistics and the accept test
 // ---------------------------------------------------------------------------
-constexpr int kFinThreads = 1024;
-constexpr int kFinWarps = kFinThreads / 32;
 constexpr long long kNaNBits = 0x7ff8000000000000ll;
 __device__ __forceinline__ double dnan() { return __longlong_as_double(kNaNBits); }
 
+// Statistics of a sequence's rows, gathered in the leader CTA.
 struct SeqShared {
   double M[kMaxRows], L[kMaxRows];
   float m[kMaxRows];
   int amax[kMaxRows];
   int ok[kMaxRows];
-  int a, bad;
 };
 
-// Combine the tile partials of the rows of one sequence (a warp per row) into
-// shared memory and into the RowFinal array (read later by the draw kernel).
+// Combine the tile partials of a sequence's rows (a warp per row, over the
+// row warps of all CTAs of the cluster) into the leader's SeqShared (lsh,
+// distributed shared memory) and the RowFinal array.
 template <typename Want>
-__device__ void finish_rows(SeqShared& sh, const Partial* part, int ntiles, int row0, int nrows,
-                            Want want, bool greedy, float chi, RowFinal* fin) {
+__device__ void cluster_rows(SeqShared* lsh, unsigned rank, const Partial* part, int ntiles,
+                             int row0, int nrows, Want want, bool greedy, float chi,
+                             RowFinal* fin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == kFinWarps - 1) return;  // the accept warp
-  for (int r = warp; r < nrows; r += kFinWarps - 1) {
+  if (warp >= kRowWarps) return;
+  for (int r = (int)rank * kRowWarps + warp; r < nrows; r += kCluster * kRowWarps) {
     if (!want(r)) {
-      if (lane == 0) { sh.ok[r] = 1; sh.m[r] = 0.f; sh.M[r] = 0; sh.L[r] = 0; sh.amax[r] = -1; }
+      if (lane == 0) {
+        lsh->ok[r] = 1; lsh->m[r] = 0.f; lsh->M[r] = 0; lsh->L[r] = 0; lsh->amax[r] = -1;
+      }
       continue;
     }
     const RowFinal f = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, chi, lane);
     if (lane == 0) {
       fin[row0 + r] = f;
-      sh.m[r] = f.m;
-      sh.M[r] = f.M;
-      sh.L[r] = f.L;
-      sh.amax[r] = f.amax;
-      sh.ok[r] = f.ok;
+      lsh->m[r] = f.m;
+      lsh->M[r] = f.M;
+      lsh->L[r] = f.L;
+      lsh->amax[r] = f.amax;
+      lsh->ok[r] = f.ok;
     }
   }
 }
@@ -315,8 +300,8 @@ __device__ __forceinline__ const T* row_ptr(const unsigned char* base, long long
 // Logits of the drafted tokens for the first 32 positions, fetched by the
 // accept warp while the other warps combine the rows.
 struct AcceptPre {
-  int x;        // draft id of position lane (or -1 past n)
-  float lt, ld; // target / draft logit at x
+  int x;         // draft id of position lane (or -1 past n)
+  float lt, ld;  // target / draft logit at x
 };
 template <typename T, typename TP, typename DP>
 __device__ __forceinline__ AcceptPre accept_prefetch(int n, int V, bool greedy,
@@ -335,13 +320,15 @@ __device__ __forceinline__ AcceptPre accept_prefetch(int n, int V, bool greedy,
 
 // One speculative check on n positions (one warp). Target row j: tp(j) with
 // log2 partition sh.M + sh.L at index j; draft law of position j: row dp(j)
-// with log2 partition dlt(j). Sets sh.a (first rejection, n if none) and
-// sh.bad (a draft id outside [0, V)). Writes p_j(x_j), q_j(x_j) to diag_p /
-// diag_q. Positions below 32 use the prefetched logits.
+// with log2 partition dlt(j). Returns a (first rejection, n if none) in every
+// lane; *bad is set if a draft id lies outside [0, V). Writes p_j(x_j) and
+// q_j(x_j) to diag_p / diag_q when given. Positions below 32 use the
+// prefetched logits.
 template <typename T, typename TP, typename DP, typename DS>
-__device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const DecideCommon& c,
-                            int b, bool greedy, double cd, const int32_t* drafts, TP tp, DP dp,
-                            DS dlt, double* diag_p, double* diag_q, const AcceptPre& pre) {
+__device__ int accept_scan(const SeqShared* sh, int n, int pos0, int stage,
+                           const DecideCommon& c, int b, bool greedy, double cd,
+                           const int32_t* drafts, TP tp, DP dp, DS dlt, double* diag_p,
+                           double* diag_q, const AcceptPre& pre, int* bad_out) {
   const int lane = threadIdx.x & 31;
   int a = n, bad = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
@@ -352,11 +339,11 @@ __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const Dec
       if (x < 0 || x >= c.V) {
         badj = true;
       } else if (greedy) {
-        acc = (x == sh.amax[j]);
+        acc = (x == sh->amax[j]);
       } else {
         const float lt = j0 == 0 ? pre.lt : load_elem(tp(j) + x);
         const float ld = j0 == 0 ? pre.ld : load_elem(dp(j) + x);
-        const double lp = (double)lt * cd - (sh.M[j] + sh.L[j]);
+        const double lp = (double)lt * cd - (sh->M[j] + sh->L[j]);
         const double lq = (double)ld * cd - dlt(j);
         const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(pos0 + j),
                                       (uint32_t)stage).x;
@@ -368,110 +355,123 @@ __device__ void accept_scan(SeqShared& sh, int n, int pos0, int stage, const Dec
     const unsigned rej = __ballot_sync(0xffffffffu, j < n && !acc);
     if (rej && a == n) a = j0 + __ffs(rej) - 1;
   }
-  if (lane == 0) { sh.a = a; sh.bad = bad; }
+  *bad_out = bad;
+  return a;
 }
 
-__device__ __forceinline__ bool rows_ok(const SeqShared& sh, int nrows) {
+__device__ __forceinline__ bool rows_ok(const SeqShared* sh, int nrows) {
   int bad = 0;
-  for (int r = 0; r < nrows; ++r) bad |= !sh.ok[r];
+  for (int r = 0; r < nrows; ++r) bad |= !sh->ok[r];
   return !bad;
 }
+
+// Per-CTA outcome of the accept test (every CTA of the cluster computes it).
+struct Outcome {
+  int a, bad;
+};
 
 // ---------------------------------------------------------------------------
 // Chain verification
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(kFinThreads) chain_finish_kernel(ChainDecideArgs A) {
+__global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecideArgs A) {
   grid_dependency_wait();
+  cg::cluster_group cl = cg::this_cluster();
+  const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
+  __shared__ Outcome s_out;
+  extern __shared__ double dyn[];  // leader: [nrt] tile sums, [nrt] prefixes
+  SeqShared* lsh = cl.map_shared_rank(&sh, 0);
+  double* ltsum = cl.map_shared_rank(dyn, 0);
   const DecideCommon& c = A.c;
-  const int b = blockIdx.x, K = c.K, per = 2 * K + 1;
+  const int b = blockIdx.y, K = c.K, V = c.V, per = 2 * K + 1;
   const float Tb = c.temperature[b];
   const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
-  double* diag = c.diag ? c.diag + (size_t)b * (4 * K + 2) : nullptr;
-  auto fail = [&]() {
+  double* diag = (rank == 0 && c.diag) ? c.diag + (size_t)b * (4 * K + 2) : nullptr;
+  auto fail = [&]() {  // leader only
     if (threadIdx.x == 0) {
       set_status(c.status, SPEC_EDEVICE);
       A.accept_len[b] = -1;
-      c.dec[b] = SeqDecision{-1, 2};
     }
     for (int j = threadIdx.x; j <= K; j += blockDim.x) A.out_tok[(size_t)b * (K + 1) + j] = -1;
     if (diag)
       for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
   };
-  if (!tvalid) { fail(); grid_dependents_launch(); return; }
+  if (!tvalid) {  // same verdict in every CTA of the cluster: all leave here
+    if (rank == 0) fail();
+    return;
+  }
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   auto tp = [&](int j) { return row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + j); };
-  auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
-  const bool accept_warp = (threadIdx.x >> 5) == kFinWarps - 1;
+  auto dl = [&](int j) { return lsh->M[K + 1 + j] + lsh->L[K + 1 + j]; };
+  const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
   AcceptPre pre{-1, 0.f, 0.f};
-  if (accept_warp) pre = accept_prefetch<T>(K, c.V, greedy, drafts, tp, dp);
-  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
-              sc.hi, c.fin);
-  __syncthreads();
-  if (accept_warp)
-    accept_scan<T>(sh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
-                   diag && !greedy ? diag + 2 * K + 1 : nullptr,
-                   diag && !greedy ? diag + 3 * K + 1 : nullptr, pre);
-  __syncthreads();
-  if (sh.bad || !rows_ok(sh, per)) { fail(); grid_dependents_launch(); return; }
-  const int a = sh.a;
-  if (greedy) {
-    for (int j = threadIdx.x; j <= K; j += blockDim.x)
-      A.out_tok[(size_t)b * (K + 1) + j] = j < a ? drafts[j] : (j == a ? sh.amax[a] : -1);
-    if (threadIdx.x == 0) { A.accept_len[b] = a; c.dec[b] = SeqDecision{a, 1}; }
-    if (diag)
-      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
-  } else {
-    if (threadIdx.x == 0) c.dec[b] = SeqDecision{a, 0};
-    if (diag)
-      for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+  cl.sync();  // every CTA of the cluster is running: its shared memory may be used
+  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp);
+  cluster_rows(lsh, rank, c.part, c.ntiles, b * per, per,
+               [&](int r) { return r <= K || !greedy; }, greedy, sc.hi, c.fin);
+  cl.sync();  // the leader holds every row's statistics
+  if (accept_warp) {
+    int bad;
+    const int a = accept_scan<T>(lsh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
+                                 diag && !greedy ? diag + 2 * K + 1 : nullptr,
+                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad);
+    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per)};
   }
-  grid_dependents_launch();
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kDecideThreads, 4) chain_draw_kernel(ChainDecideArgs A) {
-  grid_dependency_wait();
-  extern __shared__ double dyn_pre[];
-  const DecideCommon& c = A.c;
-  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, per = 2 * K + 1;
-  const SeqDecision d = c.dec[b];
-  if (d.state != 0) return;
-  const int a = d.a;
-  const Scale sc = make_scale(c.temperature[b]);
-  const RowFinal fp = c.fin[b * per + a];
-  const T* prow = row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + a);
-  const T* qrow = a < K ? row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + a) : nullptr;
-  double lq = 0.0;
-  if (a < K) {
-    const RowFinal fq = c.fin[b * per + K + 1 + a];
-    lq = fq.M + fq.L;
+  __syncthreads();
+  const Outcome o = s_out;
+  const int nrt = residual_tiles(V);
+  const T* prow = nullptr;
+  const T* qrow = nullptr;
+  ProbCoef kp{}, kq{};
+  if (!o.bad && !greedy) {
+    prow = tp(o.a);
+    qrow = o.a < K ? dp(o.a) : nullptr;
+    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], sc);
+    kq = make_coef(o.a < K ? dl(o.a) : 0.0, sc);
+    const int chunk = (nrt + kCluster - 1) / kCluster;
+    residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
+                          min(nrt, ((int)rank + 1) * chunk), ltsum);
   }
-  const ProbCoef kp = make_coef(fp.M + fp.L, sc), kq = make_coef(lq, sc);
-  const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 1u).y;
+  cl.sync();  // every tile sum is in the leader
+  if (rank != 0) return;
+  if (o.bad) {
+    fail();
+    grid_dependents_launch();
+    return;
+  }
+  const int a = o.a;
   int tok;
-  double Z;
-  if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
-  const int32_t* drafts = c.draft_tok + (size_t)b * K;
+  double Z = dnan();
+  if (greedy) {
+    tok = sh.amax[a];
+  } else {
+    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 1u).y;
+    tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
+  }
   for (int j = threadIdx.x; j <= K; j += blockDim.x)
     A.out_tok[(size_t)b * (K + 1) + j] = j < a ? drafts[j] : (j == a ? tok : -1);
-  if (threadIdx.x == 0) {
-    A.accept_len[b] = a;
-    if (c.diag) c.diag[(size_t)b * (4 * K + 2) + 4 * K + 1] = Z;
+  if (threadIdx.x == 0) A.accept_len[b] = a;
+  if (diag) {
+    if (greedy) {
+      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
+    } else {
+      for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+      if (threadIdx.x == 0) diag[4 * K + 1] = Z;
+    }
   }
+  grid_dependents_launch();
 }
 
 // ---------------------------------------------------------------------------
 // Two-stage verification
 // ---------------------------------------------------------------------------
-// Stage one: drafts (slots w..w+K-1) against L_i (slots w..w+K), draft law
-// L_d; the a1 accepted drafts and the drawn token join the window with the
-// L_i statistics of their slots.
+// Window append (leader): a + 1 tokens at slots w.. with the L_i statistics of
+// their slots (raw max m and ln sum exp((l - m)/T)).
 __device__ __forceinline__ void window_append(const HierDecideArgs& A, int b, int w, int a,
-                                              const int32_t* drafts, int tok, const RowFinal* rf,
+                                              const int32_t* drafts, int tok, const SeqShared& sh,
                                               bool greedy, double cd) {
   const int WC = A.Ni + A.c.K;
   for (int j = threadIdx.x; j <= a; j += blockDim.x) {
@@ -481,234 +481,226 @@ __device__ __forceinline__ void window_append(const HierDecideArgs& A, int b, in
       A.win_stat[2 * slot] = dnan();
       A.win_stat[2 * slot + 1] = dnan();
     } else {
-      const RowFinal f = rf[j];
-      A.win_stat[2 * slot] = f.m;
-      A.win_stat[2 * slot + 1] = (f.M + f.L - (double)f.m * cd) * kLn2;
+      A.win_stat[2 * slot] = sh.m[j];
+      A.win_stat[2 * slot + 1] = (sh.M[j] + sh.L[j] - (double)sh.m[j] * cd) * kLn2;
     }
   }
 }
 
+// Stage one: drafts (slots w..w+K-1) against L_i (slots w..w+K), draft law
+// L_d; the a1 accepted drafts and the drawn token join the window.
 template <typename T>
-__global__ void __launch_bounds__(kFinThreads) hier1_finish_kernel(HierDecideArgs A) {
+__global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecideArgs A) {
   grid_dependency_wait();
+  cg::cluster_group cl = cg::this_cluster();
+  const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
+  __shared__ Outcome s_out;
+  extern __shared__ double dyn[];
+  SeqShared* lsh = cl.map_shared_rank(&sh, 0);
+  double* ltsum = cl.map_shared_rank(dyn, 0);
   const DecideCommon& c = A.c;
-  const int b = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni, WC = Ni + K, per = 2 * K + 1;
+  const int b = blockIdx.y, K = c.K, V = c.V, S = A.S, Ni = A.Ni, WC = Ni + K, per = 2 * K + 1;
   const int D = 4 * K + 3 * S + 1;
-  double* diag = c.diag ? c.diag + (size_t)b * D : nullptr;
-  // Stage-two outputs default to "did not run"; stage two overwrites them.
-  for (int j = threadIdx.x; j < WC + 1; j += blockDim.x) A.commit_tok[(size_t)b * (WC + 1) + j] = -1;
-  if (threadIdx.x == 0) { A.commit_n[b] = 0; A.acc2[b] = -1; }
-  if (diag)
-    for (int j = threadIdx.x; j < D; j += blockDim.x) diag[j] = dnan();
+  double* diag = (rank == 0 && c.diag) ? c.diag + (size_t)b * D : nullptr;
+  if (rank == 0) {  // stage-two outputs default to "did not run"
+    for (int j = threadIdx.x; j < WC + 1; j += blockDim.x)
+      A.commit_tok[(size_t)b * (WC + 1) + j] = -1;
+    if (threadIdx.x == 0) { A.commit_n[b] = 0; A.acc2[b] = -1; }
+    if (diag)
+      for (int j = threadIdx.x; j < D; j += blockDim.x) diag[j] = dnan();
+  }
   const float Tb = c.temperature[b];
   const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
   const int w = A.win_len[b];
-  auto fail = [&]() {
+  auto fail = [&]() {  // leader only
     if (threadIdx.x == 0) {
       set_status(c.status, SPEC_EDEVICE);
       A.acc1[b] = -1;
-      c.dec[b] = SeqDecision{-1, 2};
     }
   };
-  if (!tvalid || w < 0 || w >= Ni) { fail(); grid_dependents_launch(); return; }
+  if (!tvalid || w < 0 || w >= Ni) {
+    if (rank == 0) fail();
+    return;
+  }
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
   const int32_t* drafts = c.draft_tok + (size_t)b * K;
   const long long row0 = (long long)b * S + w;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, row0 + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_d, A.ld, row0 + j); };
-  auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
-  const bool accept_warp = (threadIdx.x >> 5) == kFinWarps - 1;
+  auto dl = [&](int j) { return lsh->M[K + 1 + j] + lsh->L[K + 1 + j]; };
+  const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
   AcceptPre pre{-1, 0.f, 0.f};
-  if (accept_warp) pre = accept_prefetch<T>(K, c.V, greedy, drafts, tp, dp);
-  finish_rows(sh, c.part, c.ntiles, b * per, per, [&](int r) { return r <= K || !greedy; }, greedy,
-              sc.hi, c.fin);
-  __syncthreads();
-  if (accept_warp)
-    accept_scan<T>(sh, K, w, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
-                   diag && !greedy ? diag + 2 * K + 1 : nullptr,
-                   diag && !greedy ? diag + 3 * K + 1 : nullptr, pre);
-  __syncthreads();
-  if (sh.bad || !rows_ok(sh, per)) { fail(); grid_dependents_launch(); return; }
-  const int a = sh.a;
-  if (greedy) {
-    window_append(A, b, w, a, drafts, sh.amax[a], nullptr, true, 0.0);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      A.win_len[b] = w + a + 1;
-      A.acc1[b] = a;
-      c.dec[b] = SeqDecision{a, 1};
-    }
-  } else {
-    if (threadIdx.x == 0) c.dec[b] = SeqDecision{a, 0};
-    if (diag)
-      for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+  cl.sync();
+  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp);
+  cluster_rows(lsh, rank, c.part, c.ntiles, b * per, per,
+               [&](int r) { return r <= K || !greedy; }, greedy, sc.hi, c.fin);
+  cl.sync();
+  if (accept_warp) {
+    int bad;
+    const int a = accept_scan<T>(lsh, K, w, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
+                                 diag && !greedy ? diag + 2 * K + 1 : nullptr,
+                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad);
+    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per)};
   }
-  grid_dependents_launch();
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kDecideThreads, 4) hier1_draw_kernel(HierDecideArgs A) {
-  grid_dependency_wait();
-  extern __shared__ double dyn_pre[];
-  const DecideCommon& c = A.c;
-  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, S = A.S, per = 2 * K + 1;
-  const SeqDecision d = c.dec[b];
-  if (d.state != 0) return;
-  const int a = d.a;
-  const int w = A.win_len[b];
-  const Scale sc = make_scale(c.temperature[b]);
-  const long long row0 = (long long)b * S + w;
-  const RowFinal fp = c.fin[b * per + a];
-  const T* prow = row_ptr<T>(A.lg_i, A.ld, row0 + a);
-  const T* qrow = a < K ? row_ptr<T>(A.lg_d, A.ld, row0 + a) : nullptr;
-  double lq = 0.0;
-  if (a < K) {
-    const RowFinal fq = c.fin[b * per + K + 1 + a];
-    lq = fq.M + fq.L;
+  __syncthreads();
+  const Outcome o = s_out;
+  const int nrt = residual_tiles(V);
+  const T* prow = nullptr;
+  const T* qrow = nullptr;
+  ProbCoef kp{}, kq{};
+  if (!o.bad && !greedy) {
+    prow = tp(o.a);
+    qrow = o.a < K ? dp(o.a) : nullptr;
+    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], sc);
+    kq = make_coef(o.a < K ? dl(o.a) : 0.0, sc);
+    const int chunk = (nrt + kCluster - 1) / kCluster;
+    residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
+                          min(nrt, ((int)rank + 1) * chunk), ltsum);
   }
-  const ProbCoef kp = make_coef(fp.M + fp.L, sc), kq = make_coef(lq, sc);
-  const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(w + a), 1u).y;
+  cl.sync();
+  if (rank != 0) return;
+  if (o.bad) {
+    fail();
+    grid_dependents_launch();
+    return;
+  }
+  const int a = o.a;
   int tok;
-  double Z;
-  if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
-  window_append(A, b, w, a, c.draft_tok + (size_t)b * K, tok, c.fin + (size_t)b * per, false, sc.d);
+  double Z = dnan();
+  if (greedy) {
+    tok = sh.amax[a];
+  } else {
+    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(w + a), 1u).y;
+    tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
+  }
+  window_append(A, b, w, a, drafts, tok, sh, greedy, sc.d);
+  if (diag && !greedy) {
+    for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+    if (threadIdx.x == 0) diag[4 * K + 1] = Z;
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     A.win_len[b] = w + a + 1;
     A.acc1[b] = a;
-    if (c.diag) c.diag[(size_t)b * (4 * K + 3 * S + 1) + 4 * K + 1] = Z;
   }
+  grid_dependents_launch();
 }
 
 // Stage two: for sequences whose window holds W >= Ni tokens, the window
 // tokens (slots 0..W-1) against L_f (slots 0..W), draft law L_i from the
 // buffered statistics; commits a2 + 1 tokens and empties the window.
 template <typename T>
-__global__ void __launch_bounds__(kFinThreads) hier2_finish_kernel(HierDecideArgs A) {
+__global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecideArgs A) {
   grid_dependency_wait();
+  cg::cluster_group cl = cg::this_cluster();
+  const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
+  __shared__ Outcome s_out;
+  extern __shared__ double dyn[];
+  SeqShared* lsh = cl.map_shared_rank(&sh, 0);
+  double* ltsum = cl.map_shared_rank(dyn, 0);
   const DecideCommon& c = A.c;
-  const int b = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni, WC = Ni + K;
+  const int b = blockIdx.y, K = c.K, V = c.V, S = A.S, Ni = A.Ni, WC = Ni + K;
   const int W = A.win_len[b];
-  if (A.acc1[b] < 0 || !(W >= Ni && W < S)) {
-    if (threadIdx.x == 0) c.dec[b] = SeqDecision{-1, 1};  // no second stage
-    grid_dependents_launch();
-    return;
-  }
+  if (A.acc1[b] < 0 || !(W >= Ni && W < S)) return;  // no second stage (every CTA)
   const float Tb = c.temperature[b];  // validated by stage one
   const bool greedy = (Tb == 0.0f);
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
-  double* diag = c.diag ? c.diag + (size_t)b * (4 * K + 3 * S + 1) + (4 * K + 2) : nullptr;
+  double* diag =
+      (rank == 0 && c.diag) ? c.diag + (size_t)b * (4 * K + 3 * S + 1) + (4 * K + 2) : nullptr;
   const int32_t* wtok = A.win_tok + (size_t)b * WC;
   const double* wst = A.win_stat + (size_t)b * WC * 2;
   auto tp = [&](int j) { return row_ptr<T>(A.lg_f, A.ld, (long long)b * S + j); };
   auto dp = [&](int j) { return row_ptr<T>(A.lg_i, A.ld, (long long)b * S + j); };
   auto dl = [&](int j) { return wst[2 * j] * sc.d + wst[2 * j + 1] * kLog2e; };
-  const bool accept_warp = (threadIdx.x >> 5) == kFinWarps - 1;
+  const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
   AcceptPre pre{-1, 0.f, 0.f};
-  if (accept_warp) pre = accept_prefetch<T>(W, c.V, greedy, wtok, tp, dp);
-  finish_rows(sh, c.part, c.ntiles, b * S, W + 1, [&](int) { return true; }, greedy, sc.hi, c.fin);
+  cl.sync();
+  if (accept_warp) pre = accept_prefetch<T>(W, V, greedy, wtok, tp, dp);
+  cluster_rows(lsh, rank, c.part, c.ntiles, b * S, W + 1, [&](int) { return true; }, greedy,
+               sc.hi, c.fin);
+  cl.sync();
+  if (accept_warp) {
+    int bad;
+    const int a = accept_scan<T>(lsh, W, 0, 2, c, b, greedy, sc.d, wtok, tp, dp, dl,
+                                 diag && !greedy ? diag + S : nullptr,
+                                 diag && !greedy ? diag + 2 * S - 1 : nullptr, pre, &bad);
+    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, W + 1)};
+  }
   __syncthreads();
-  if (accept_warp)
-    accept_scan<T>(sh, W, 0, 2, c, b, greedy, sc.d, wtok, tp, dp, dl,
-                   diag && !greedy ? diag + S : nullptr, diag && !greedy ? diag + 2 * S - 1 : nullptr,
-                   pre);
-  __syncthreads();
-  if (sh.bad || !rows_ok(sh, W + 1)) {
+  const Outcome o = s_out;
+  const int nrt = residual_tiles(V);
+  const T* prow = nullptr;
+  const T* qrow = nullptr;
+  ProbCoef kp{}, kq{};
+  if (!o.bad && !greedy) {
+    prow = tp(o.a);
+    qrow = o.a < W ? dp(o.a) : nullptr;
+    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], sc);
+    kq = make_coef(o.a < W ? dl(o.a) : 0.0, sc);
+    const int chunk = (nrt + kCluster - 1) / kCluster;
+    residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
+                          min(nrt, ((int)rank + 1) * chunk), ltsum);
+  }
+  cl.sync();
+  if (rank != 0) return;
+  if (o.bad) {
     if (threadIdx.x == 0) {
       set_status(c.status, SPEC_EDEVICE);
       A.acc2[b] = -1;
-      c.dec[b] = SeqDecision{-1, 2};
     }
     grid_dependents_launch();
     return;
   }
-  const int a = sh.a;
-  if (greedy) {
-    for (int j = threadIdx.x; j < WC + 1; j += blockDim.x)
-      A.commit_tok[(size_t)b * (WC + 1) + j] = j < a ? wtok[j] : (j == a ? sh.amax[a] : -1);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      A.commit_n[b] = a + 1;
-      A.acc2[b] = a;
-      A.win_len[b] = 0;
-      c.dec[b] = SeqDecision{a, 1};
-    }
-  } else {
-    if (threadIdx.x == 0) c.dec[b] = SeqDecision{a, 0};
-    if (diag)
-      for (int j = threadIdx.x; j <= W; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
-  }
-  grid_dependents_launch();
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kDecideThreads, 4) hier2_draw_kernel(HierDecideArgs A) {
-  grid_dependency_wait();
-  extern __shared__ double dyn_pre[];
-  const DecideCommon& c = A.c;
-  const int b = blockIdx.y, sp = blockIdx.x, K = c.K, S = A.S, Ni = A.Ni, WC = Ni + K;
-  const SeqDecision d = c.dec[b];
-  if (d.state != 0) return;
-  const int a = d.a;
-  const int W = A.win_len[b];
-  const Scale sc = make_scale(c.temperature[b]);
-  const RowFinal fp = c.fin[b * S + a];
-  const double* wst = A.win_stat + (size_t)b * WC * 2;
-  const T* prow = row_ptr<T>(A.lg_f, A.ld, (long long)b * S + a);
-  const T* qrow = a < W ? row_ptr<T>(A.lg_i, A.ld, (long long)b * S + a) : nullptr;
-  const double lq = a < W ? wst[2 * a] * sc.d + wst[2 * a + 1] * kLog2e : 0.0;
-  const ProbCoef kp = make_coef(fp.M + fp.L, sc), kq = make_coef(lq, sc);
-  const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 2u).y;
+  const int a = o.a;
   int tok;
-  double Z;
-  if (!draw_token<T>(c, b, sp, prow, qrow, kp, kq, u, dyn_pre, &tok, &Z)) return;
-  const int32_t* wtok = A.win_tok + (size_t)b * WC;
+  double Z = dnan();
+  if (greedy) {
+    tok = sh.amax[a];
+  } else {
+    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 2u).y;
+    tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
+  }
   for (int j = threadIdx.x; j < WC + 1; j += blockDim.x)
     A.commit_tok[(size_t)b * (WC + 1) + j] = j < a ? wtok[j] : (j == a ? tok : -1);
+  if (diag && !greedy) {
+    for (int j = threadIdx.x; j <= W; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+    if (threadIdx.x == 0) diag[3 * S - 2] = Z;
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     A.commit_n[b] = a + 1;
     A.acc2[b] = a;
     A.win_len[b] = 0;
-    if (c.diag) c.diag[(size_t)b * (4 * K + 3 * S + 1) + (4 * K + 2) + 3 * S - 2] = Z;
   }
+  grid_dependents_launch();
 }
 
 // ---------------------------------------------------------------------------
-// Launchers
+// Launchers: grid (kCluster, B), clusters of kCluster CTAs along x.
 // ---------------------------------------------------------------------------
 template <typename Kern, typename Args>
-static cudaError_t launch_draw(Kern k, const Args& a, cudaStream_t st) {
+static cudaError_t launch_decide(Kern k, const Args& a, cudaStream_t st) {
   const size_t smem = 2 * (size_t)residual_tiles(a.c.V) * sizeof(double);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess)
     return cudaGetLastError();
-  return launch_pdl(k, dim3(a.c.nsplit, a.c.B), dim3(kDecideThreads), smem, st, a);
-}
-template <typename Fin, typename Draw, typename Args>
-static cudaError_t launch_pair(Fin f, Draw d, const Args& a, cudaStream_t st) {
-  cudaError_t e = launch_pdl(f, dim3(a.c.B), dim3(kFinThreads), 0, st, a);
-  if (e != cudaSuccess) return e;
-  return launch_draw(d, a, st);
+  return launch_pdl_cluster(k, dim3(kCluster, a.c.B), dim3(kDecThreads), smem, st, kCluster, a);
 }
 
 cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st) {
-  return a.c.dtype == SPEC_BF16
-             ? launch_pair(chain_finish_kernel<__nv_bfloat16>, chain_draw_kernel<__nv_bfloat16>, a, st)
-             : launch_pair(chain_finish_kernel<float>, chain_draw_kernel<float>, a, st);
+  return a.c.dtype == SPEC_BF16 ? launch_decide(chain_decide_kernel<__nv_bfloat16>, a, st)
+                                : launch_decide(chain_decide_kernel<float>, a, st);
 }
 cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st) {
-  return a.c.dtype == SPEC_BF16
-             ? launch_pair(hier1_finish_kernel<__nv_bfloat16>, hier1_draw_kernel<__nv_bfloat16>, a, st)
-             : launch_pair(hier1_finish_kernel<float>, hier1_draw_kernel<float>, a, st);
+  return a.c.dtype == SPEC_BF16 ? launch_decide(hier1_decide_kernel<__nv_bfloat16>, a, st)
+                                : launch_decide(hier1_decide_kernel<float>, a, st);
 }
 cudaError_t launch_hier2_decide(const HierDecideArgs& a, cudaStream_t st) {
-  return a.c.dtype == SPEC_BF16
-             ? launch_pair(hier2_finish_kernel<__nv_bfloat16>, hier2_draw_kernel<__nv_bfloat16>, a, st)
-             : launch_pair(hier2_finish_kernel<float>, hier2_draw_kernel<float>, a, st);
+  return a.c.dtype == SPEC_BF16 ? launch_decide(hier2_decide_kernel<__nv_bfloat16>, a, st)
+                                : launch_decide(hier2_decide_kernel<float>, a, st);
 }
 
 }  // namespace specv

@@ -77,8 +77,6 @@ struct Hier2Rows {
 // Workspace pieces of the row-statistics step.
 struct RsBuffers {
   Partial* part;    // [rows, tiles]
-  int* seq_cnt;     // [nseq] decide arrival counters, cleared here
-  int nseq;
 };
 
 // Combine a row's tile partials (warp-cooperative; result valid in lane 0).
@@ -139,13 +137,6 @@ __device__ __forceinline__ RowFinal combine_row(const Partial* p, int ntiles, bo
   return f;
 }
 
-// Outcome of a sequence's accept test: a = first rejection; state 0 = the
-// draw is pending, 1 = outputs already written (greedy, or no second stage),
-// 2 = invalid input.
-struct SeqDecision {
-  int a;
-  int state;
-};
 
 template <typename Rows>
 cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, const RsBuffers& b,
@@ -164,10 +155,6 @@ struct DecideCommon {
   const Partial* part;             // [rows, ntiles] tile partials
   int ntiles;
   RowFinal* fin;                   // [rows] final row statistics
-  SeqDecision* dec;                // [B]
-  double* rsum;                    // [B, nrt] residual tile sums
-  int* counters;                   // [B] arrival counters (zeroed by row stats)
-  int nsplit;                      // CTAs per sequence for the residual pass
   double* diag;
   int32_t* status;
 };
@@ -200,7 +187,6 @@ struct HierDecideArgs {
 cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st);
 cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st);
 cudaError_t launch_hier2_decide(const HierDecideArgs& a, cudaStream_t st);
-int decide_split(int B, int V);   // CTAs per sequence for the residual pass
 __host__ __device__ __forceinline__ int residual_tiles(int V) {  // kResTile tiles per row
   return (V + kResTile - 1) / kResTile;
 }
@@ -230,8 +216,6 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
 
-// Bytes at the start of a workspace that hold the arrival counters (the part
-// that must be zero when a call starts).
-size_t workspace_counter_bytes(int B);
+
 
 }  // namespace specv

@@ -15,7 +15,7 @@
 // the first call on each device, with that device current, asks the runtime
 // for the address (cudaGetSymbolAddress) and keeps it, so make that first call
 // outside any stream capture. The array is shared by every call and keeps the
-// previous call's contents; the call clears the part that must start at zero.
+// previous call's contents, none of which a later call reads before writing.
 // Calls that overlap on the GPU (other streams, other threads) race on it.
 #include <mutex>
 
@@ -63,12 +63,6 @@ int spec_verify_chain_noalloc(const void* tgt, int64_t ld_tgt, const void* drf, 
   if (need > kScratchBytes) return SPEC_EWORKSPACE;
   void* ws = nullptr;
   cudaError_t e = scratch_address(&ws);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return SPEC_ECUDA;
-  }
-  // The arrival counters at the start of the scratch must begin at zero.
-  e = cudaMemsetAsync(ws, 0, specv::workspace_counter_bytes(B), (cudaStream_t)stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return SPEC_ECUDA;

@@ -152,18 +152,13 @@ __device__ __forceinline__ float vec_expsum_far<float>(uint4 w, float m, float c
 
 template <typename T, typename Rows>
 __global__ void __launch_bounds__(kRsWarps * 32, 1)
-    row_stats_kernel(Rows rows, int nrows, int V, Partial* __restrict__ part,
-                     int* __restrict__ zero_words, int nzero, int32_t* status) {
+    row_stats_kernel(Rows rows, int nrows, int V, Partial* __restrict__ part, int32_t* status) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int kVec = VecOf<T>::n;
   constexpr int kEpt = kTileBytes / (int)sizeof(T);     // elements per tile
   constexpr int kVpl = kTileBytes / 16 / 32;            // vectors per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dependency_wait();
-
-  // Clear the decide kernels' arrival counters (stream-ordered before them).
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero_words[i] = 0;
 
   unsigned char* wbuf = smem + (size_t)warp * kRsStages * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kRsWarps * kRsStages * kTileBytes) +
@@ -409,8 +404,8 @@ static int rs_grid() {
 }
 
 template <typename T, typename Rows>
-static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, int* zero_words,
-                             int nzero, int32_t* status, cudaStream_t st) {
+static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, int32_t* status,
+                             cudaStream_t st) {
   auto kern = row_stats_kernel<T, Rows>;
   static bool smem_set = false;  // once per instantiation (same on every B200)
   if (!smem_set) {
@@ -429,15 +424,15 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
   return launch_pdl(kern, dim3((unsigned)grid), dim3(kRsWarps * 32), kRsSmem, st, rows, nrows, V,
-                    part, zero_words, nzero, status);
+                    part, status);
 }
 
 template <typename Rows>
 cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, const RsBuffers& b,
                              int32_t* status, cudaStream_t st) {
   if (dtype == SPEC_BF16)
-    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, b.seq_cnt, b.nseq, status, st);
-  return launch_rs<float>(rows, nrows, V, b.part, b.seq_cnt, b.nseq, status, st);
+    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, status, st);
+  return launch_rs<float>(rows, nrows, V, b.part, status, st);
 }
 
 template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int,
