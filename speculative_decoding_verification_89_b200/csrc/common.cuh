@@ -30,9 +30,6 @@ constexpr double kLn2 = 0.6931471805599453094172321214581766;
 #ifndef SPEC_RS_STAGES
 #define SPEC_RS_STAGES 2
 #endif
-#ifndef SPEC_RS_PACKED
-#define SPEC_RS_PACKED 1  // packed FP32x2 FMAs in the exponent sums
-#endif
 constexpr int kTileBytes = SPEC_RS_TILE;
 constexpr int kRsWarps = SPEC_RS_WARPS;
 constexpr int kRsStages = SPEC_RS_STAGES;
@@ -43,9 +40,11 @@ static_assert(kTileBytes % 512 == 0, "a tile is a whole number of warp-wide 16-b
 // Residual tiles: 32 lanes x 8 elements.
 constexpr int kResTile = 256;
 
-// Per (row, tile) statistics: the tile's largest raw logit m, its first index,
-// and s = sum over the tile of 2^(l*c - M), c = log2(e) / T, with the exact
-// fp32 shift M = fl(m * c_hi) (c_hi from make_scale; M is recomputed from m).
+// Statistics of a run of consecutive tiles of one row, stored at the run's
+// first tile (the run's other tiles hold empty partials: m = -inf, s = 0):
+// the run's largest raw logit m, its first index (greedy rows), and
+// s = sum over the run of 2^(l*c - M), c = log2(e) / T, with the exact fp32
+// shift M = fl(m * c_hi) (c_hi from make_scale; M is recomputed from m).
 struct Partial {
   float m;
   int idx;

@@ -1,20 +1,24 @@
-// Row statistics: for every logit row the verification needs, the running
-// maximum, its first index and the sum of exponentials at temperature T,
-// computed per 8 KiB vocabulary tile.
+// Row statistics: for every logit row the verification needs, the maximum,
+// its first index and the sum of exponentials at temperature T, as partial
+// statistics over runs of consecutive vocabulary tiles.
 //
 // Step "temperature softmax over V" behind every check of HiSpec
 // (gist.science summary of arXiv 2510.01336, section 2: the three exits L_d,
 // L_i, L_f each give a token distribution; "Verlustfreie Garantie" compares
 // them). p = softmax(l / T) needs max and sum over the whole vocabulary row.
 //
-// Design (B200): a persistent grid; each warp owns a ring of kRsStages tile
-// buffers in shared memory, filled by 1-D bulk copies (TMA engine, no tensor
-// map, no multicast) that complete on per-stage mbarriers. A warp walks the
-// (row, tile) items i = gw, gw + nw, ... so every SM streams; two passes over
-// the staged tile (max with first index, then the sum of 2^((l - m) c)) and
-// warp shuffles give one Partial per (row, tile). Rows that need no
-// statistics (draft rows of greedy sequences, slots outside a window) are
-// skipped without traffic.
+// Design (B200): a persistent grid, one CTA of kRsWarps warps per SM. The
+// rows that need statistics (not the draft rows of greedy sequences, not the
+// slots outside a window) are first listed in shared memory; their
+// (row, tile) items are then dealt out as one contiguous run per warp, so a
+// warp changes row at most a few times. Each warp owns a ring of kRsStages
+// tile buffers filled by 1-D bulk copies (TMA engine, no tensor map, no
+// multicast) that complete on per-stage mbarriers. Per lane, the largest
+// logit and the sum of 2^(l*c - M) are carried across the tiles of a row with
+// a shift M that moves only when the exponents would exceed 2^64, so a tile
+// costs no warp shuffle and no division; the lanes are combined once per row
+// run into one Partial at the run's first tile (its other tiles get empty
+// partials).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -93,31 +97,6 @@ __device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, fl
       ex2x2(expo2(make_float2(__uint_as_float(w.z), __uint_as_float(w.w)), chi, clo, nM));
   return __fadd2_rn(e0, e1);
 }
-// Scalar forms (one FMA pair per element): the same arithmetic without
-// packing, for builds where pair formation costs more than it saves.
-__device__ __forceinline__ float vec_expsum_s(uint4 w, float chi, float clo, float nM,
-                                              __nv_bfloat16*) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-  float e[8];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float lo = bf_lo(ws[q]), hi = bf_hi(ws[q]);
-    e[2 * q] = ex2(fmaf(lo, clo, fmaf(lo, chi, nM)));
-    e[2 * q + 1] = ex2(fmaf(hi, clo, fmaf(hi, chi, nM)));
-  }
-  return ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-}
-__device__ __forceinline__ float vec_expsum_s(uint4 w, float chi, float clo, float nM, float*) {
-  float e[4];
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float x = __uint_as_float(ws[q]);
-    e[q] = ex2(fmaf(x, clo, fmaf(x, chi, nM)));
-  }
-  return (e[0] + e[1]) + (e[2] + e[3]);
-}
-
 // Scalar form of one term (tail elements).
 __device__ __forceinline__ float term(float x, float chi, float clo, float nM) {
   return ex2(fmaf(x, clo, fmaf(x, chi, nM)));
@@ -150,81 +129,120 @@ __device__ __forceinline__ float vec_expsum_far<float>(uint4 w, float m, float c
           term_far(__uint_as_float(w.w), m, chi, clo, rr));
 }
 
+// A launch lists at most kMaxListRows rows (the host splits larger calls).
+constexpr int kMaxListRows = 8192;
+constexpr int kRsSmemTotal = kRsSmem + kMaxListRows * (int)sizeof(int);
+static_assert(kRsSmemTotal <= 227 * 1024, "row list and ring exceed shared memory");
+constexpr float kShiftSlack = 64.0f;  // exponents above the shift stay below 2^64
+constexpr float kFarShift = 67108864.0f;  // 2^26: beyond, 2^(m*c - M) itself may overflow
+
+template <typename T> __device__ __forceinline__ uint4 neg_inf_vec();
+template <> __device__ __forceinline__ uint4 neg_inf_vec<__nv_bfloat16>() {
+  return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+}
+template <> __device__ __forceinline__ uint4 neg_inf_vec<float>() {
+  return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);
+}
+
 template <typename T, typename Rows>
 __global__ void __launch_bounds__(kRsWarps * 32, 1)
-    row_stats_kernel(Rows rows, int nrows, int V, Partial* __restrict__ part, int32_t* status) {
+    row_stats_kernel(Rows rows, int row_base, int nrows, int V, Partial* __restrict__ part,
+                     int32_t* status) {
   extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_wsum[kRsWarps];
   constexpr int kVec = VecOf<T>::n;
   constexpr int kEpt = kTileBytes / (int)sizeof(T);     // elements per tile
   constexpr int kVpl = kTileBytes / 16 / 32;            // vectors per lane
+  constexpr int kThreads = kRsWarps * 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  grid_dependency_wait();
 
   unsigned char* wbuf = smem + (size_t)warp * kRsStages * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kRsWarps * kRsStages * kTileBytes) +
                    warp * kRsStages;
+  int* s_list = reinterpret_cast<int*>(smem + kRsSmem);
   if (lane == 0) {
     for (int s = 0; s < kRsStages; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
   }
-  __syncwarp();
+  grid_dependency_wait();
 
-  const int ntiles = (V + kEpt - 1) / kEpt;
-  const int gw = blockIdx.x * kRsWarps + warp;
-  const int nw = gridDim.x * kRsWarps;
-  const int dr = nw / ntiles, dt = nw - dr * ntiles;
-
-  // Item cursors (row, tile) advanced by nw items at a time, skipping rows
-  // that need no statistics.
-  struct Cursor {
-    int r, t;
-  };
-  auto advance = [&](Cursor& c) {
-    c.t += dt;
-    c.r += dr;
-    if (c.t >= ntiles) { c.t -= ntiles; ++c.r; }
-  };
-  auto settle = [&](Cursor& c) {
-    while (c.r < nrows && !rows.get(c.r).valid) advance(c);
-  };
-  auto issue = [&](int s, const Cursor& c) {
-    const RowRef ref = rows.get(c.r);
-    const int nel = min(kEpt, V - c.t * kEpt);
-    const uint32_t bytes = ((uint32_t)nel * sizeof(T)) & ~15u;
-    mbar_arrive_expect_tx(&bars[s], bytes);
-    if (bytes) bulk_g2s(wbuf + s * kTileBytes, ref.ptr + (size_t)c.t * kTileBytes, bytes, &bars[s]);
-  };
-
-  Cursor prod{gw / ntiles, gw % ntiles};
-  settle(prod);
-  int inflight = 0;
-  for (int s = 0; s < kRsStages && prod.r < nrows; ++s) {
-    if (lane == 0) issue(s, prod);
-    ++inflight;
-    advance(prod);
-    settle(prod);
+  // The rows that need statistics, in order: each thread tests a contiguous
+  // run of at most 32 rows, a block scan places them.
+  {
+    const int per = (nrows + kThreads - 1) / kThreads;
+    const int q0 = min(nrows, (int)threadIdx.x * per), q1 = min(nrows, q0 + per);
+    uint32_t vmask = 0;
+    int cnt = 0;
+    for (int q = q0; q < q1; ++q)
+      if (rows.get(row_base + q).valid) {
+        vmask |= 1u << (q - q0);
+        ++cnt;
+      }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    for (int w = 0; w < warp; ++w) pos += s_wsum[w];
+    for (int q = q0; q < q1; ++q)
+      if ((vmask >> (q - q0)) & 1u) s_list[pos++] = q;
   }
-  Cursor cons{gw / ntiles, gw % ntiles};
-  settle(cons);
+  int nlisted = 0;
+  for (int w = 0; w < kRsWarps; ++w) nlisted += s_wsum[w];
+  __syncthreads();
+
+  // This warp's run of items [i0, i1) over (listed row, tile).
+  const int ntiles = (V + kEpt - 1) / kEpt;
+  const long long nitems = (long long)nlisted * ntiles;
+  const int gw = blockIdx.x * kRsWarps + warp, nw = gridDim.x * kRsWarps;
+  const long long i0 = nitems * gw / nw, i1 = nitems * (gw + 1) / nw;
+  const int nmine = (int)(i1 - i0);
+  const int k0 = (int)(i0 / ntiles), t0 = (int)(i0 - (long long)k0 * ntiles);
+
+  // Producer: lane 0 issues the copies, every lane keeps the cursor.
+  int pk = k0, pt = t0, pleft = nmine, pk_row = -1;
+  const unsigned char* pptr = nullptr;
+  auto issue = [&](int st) {
+    if (pk != pk_row) {
+      pk_row = pk;
+      pptr = rows.get(row_base + s_list[pk]).ptr;
+    }
+    if (lane == 0) {
+      const int nel = min(kEpt, V - pt * kEpt);
+      const uint32_t bytes = ((uint32_t)nel * sizeof(T)) & ~15u;
+      fence_proxy_async_smem();  // the warp's reads of this stage come first
+      mbar_arrive_expect_tx(&bars[st], bytes);
+      if (bytes) bulk_g2s(wbuf + st * kTileBytes, pptr + (size_t)pt * kTileBytes, bytes, &bars[st]);
+    }
+    if (++pt == ntiles) { pt = 0; ++pk; }
+    --pleft;
+  };
+  int inflight = 0;
+  for (int st = 0; st < kRsStages && pleft > 0; ++st) {
+    issue(st);
+    ++inflight;
+  }
+
+  // Consumer state of the current row run (per lane).
+  int ck = k0, ct = t0;
   uint32_t phase = 0;
   bool timed_out = false;
   int s = 0;  // stage of the item being consumed
+  int row = 0, run_t0 = 0;
+  const T* rptr = nullptr;
+  bool greedy = false;
+  float chi = 0.0f, clo = 0.0f;
+  float mrun = -INFINITY;    // largest logit of the lane in the run
+  float anchor = -INFINITY;  // the logit that set the shift
+  float Msh = 0.0f;          // shift fl(anchor * chi)
+  double acc = 0.0;          // sum of 2^(l*c - Msh) over the lane's elements
+  int gidx = 0x7fffffff;     // greedy rows: first index of mrun
 
-  // Hand stage s back to the copy engine with the next item of this warp.
-  auto refill = [&](int st) {
-    __syncwarp();
-    if (prod.r < nrows) {
-      if (lane == 0) {
-        fence_proxy_async_smem();
-        issue(st, prod);
-      }
-      ++inflight;
-      advance(prod);
-      settle(prod);
-    }
-  };
-
-  for (; cons.r < nrows; s = (s + 1 == kRsStages) ? 0 : s + 1) {
+  for (int it = 0; it < nmine; ++it, s = (s + 1 == kRsStages) ? 0 : s + 1) {
     const bool ok = mbar_wait_bounded(&bars[s], (phase >> s) & 1u, kWaitLimitNs);
     if (__any_sync(0xffffffffu, !ok)) {
       timed_out = true;
@@ -233,148 +251,142 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     phase ^= 1u << s;
     --inflight;
 
-    const int r = cons.r, t = cons.t;
-    const RowRef ref = rows.get(r);
-    const bool greedy = (ref.T == 0.0f);
-    float chi = 0.0f, clo = 0.0f;
-    if (!greedy) {
-      const Scale sc = make_scale(ref.T);
-      chi = sc.hi;
-      clo = sc.lo;
+    if (it == 0 || ct == 0) {  // a row run starts
+      row = row_base + s_list[ck];
+      const RowRef ref = rows.get(row);
+      rptr = reinterpret_cast<const T*>(ref.ptr);
+      greedy = (ref.T == 0.0f);
+      if (!greedy) {
+        const Scale sc = make_scale(ref.T);
+        chi = sc.hi;
+        clo = sc.lo;
+      }
+      run_t0 = ct;
+      mrun = anchor = -INFINITY;
+      Msh = 0.0f;
+      acc = 0.0;
+      gidx = 0x7fffffff;
     }
-    const int nel = min(kEpt, V - t * kEpt);
-    const uint4* buf = reinterpret_cast<const uint4*>(wbuf + s * kTileBytes);
-    float best = -INFINITY;
-    int bidx = 0x7fffffff;
-    double ssum = 0.0;
 
+    // The lane's vectors of the staged tile go to registers; the stage is
+    // refilled before the arithmetic starts. Past the row's end the vectors
+    // read as -inf; a tail of fewer than 16 bytes comes from global memory.
+    const int nel = min(kEpt, V - ct * kEpt);
+    const uint4* buf = reinterpret_cast<const uint4*>(wbuf + s * kTileBytes);
+    uint4 x[kVpl];
+    int nvec = kEpt / kVec, ntail = 0;
+    float tailx = -INFINITY;
     if (nel == kEpt) {
-      // Full tile: each lane's vectors go to registers once; the stage is
-      // refilled before the arithmetic starts.
-      uint4 x[kVpl];
 #pragma unroll
       for (int i = 0; i < kVpl; ++i) x[i] = buf[lane + 32 * i];
-      refill(s);
-      if (greedy) {
-        int bestv = -1;
+    } else {
+      nvec = (int)(((uint32_t)nel * sizeof(T)) >> 4);
+      ntail = nel - nvec * kVec;
 #pragma unroll
-        for (int i = 0; i < kVpl; ++i) {
-          const float vm = vec_max(x[i], (T*)nullptr);
-          if (vm > best) { best = vm; bestv = i; }
-        }
-        if (bestv >= 0) {
-          uint4 w = x[0];
+      for (int i = 0; i < kVpl; ++i) {
+        const int v = lane + 32 * i;
+        x[i] = v < nvec ? buf[v] : neg_inf_vec<T>();
+      }
+      if (lane < ntail) tailx = load_elem(rptr + (size_t)ct * kEpt + nvec * kVec + lane);
+    }
+    __syncwarp();
+    if (pleft > 0) {
+      issue(s);
+      ++inflight;
+    }
+
+    if (greedy) {
+      // First index of the lane's largest element: vectors in index order,
+      // strict comparisons keep the earliest.
+      float tb = -INFINITY;
+      int bv = -1;
 #pragma unroll
-          for (int i = 1; i < kVpl; ++i)
-            if (i == bestv) w = x[i];
+      for (int i = 0; i < kVpl; ++i) {
+        const float vm = vec_max(x[i], (T*)nullptr);
+        if (vm > tb) { tb = vm; bv = i; }
+      }
+      if (tb > mrun) {
+        uint4 w = x[0];
 #pragma unroll
-          for (int e = kVec - 1; e >= 0; --e)
-            if (vec_elem(w, e, (T*)nullptr) == best) bidx = (lane + 32 * bestv) * kVec + e;
-        }
-        warp_argmax(best, bidx);
-      } else {
-        best = regs_max<kVpl>(x, (T*)nullptr);
+        for (int i = 1; i < kVpl; ++i)
+          if (i == bv) w = x[i];
+        int ef = 0;
 #pragma unroll
-        for (int o = 16; o; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-        if (best > -INFINITY && best < INFINITY) {
-          const float M = __fmul_rn(best, chi);
-          float a;
-          if (fabsf(M) < 67108864.0f) {  // 2^26: 2^(m*c - M) <= 2^2
-#if SPEC_RS_PACKED
-            const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
-            const float2 nM2 = make_float2(-M, -M);
-            float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int i = 0; i < kVpl; ++i)
-              acc = __fadd2_rn(acc, vec_expsum(x[i], chi2, clo2, nM2, (T*)nullptr));
-            a = acc.x + acc.y;
-#else
-            float acc0 = 0.0f, acc1 = 0.0f;
-#pragma unroll
-            for (int i = 0; i < kVpl; i += 2) {
-              acc0 += vec_expsum_s(x[i], chi, clo, -M, (T*)nullptr);
-              if (i + 1 < kVpl) acc1 += vec_expsum_s(x[i + 1], chi, clo, -M, (T*)nullptr);
-            }
-            a = acc0 + acc1;
-#endif
-          } else {
-            const float rr = fmaf(best, chi, -M) + best * clo;
-            a = 0.0f;
-#pragma unroll
-            for (int i = 0; i < kVpl; ++i) a += vec_expsum_far<T>(x[i], best, chi, clo, rr);
-          }
-          ssum = warp_sum_d((double)a);
-        }
+        for (int e = kVec - 1; e >= 0; --e)
+          if (vec_elem(w, e, (T*)nullptr) == tb) ef = e;
+        mrun = tb;
+        gidx = ct * kEpt + (lane + 32 * bv) * kVec + ef;
+      }
+      if (tailx > mrun) {
+        mrun = tailx;
+        gidx = ct * kEpt + nvec * kVec + lane;
       }
     } else {
-      // Last, partial tile of a row: guarded loads and a scalar tail.
-      const int nvec = (int)(((uint32_t)nel * sizeof(T)) >> 4);
-      const int ntail = nel - nvec * kVec;
-      const T* gtail = reinterpret_cast<const T*>(ref.ptr) + (size_t)t * kEpt + nvec * kVec;
-      float tailx = -INFINITY;
-      if (lane < ntail) tailx = load_elem(gtail + lane);
-      if (greedy) {
-        int bestv = -1;
-        for (int i = 0; i < kVpl; ++i) {
-          const int v = lane + 32 * i;
-          if (v < nvec) {
-            const float vm = vec_max(buf[v], (T*)nullptr);
-            if (vm > best) { best = vm; bestv = v; }
-          }
-        }
-        if (bestv >= 0) {
-          const uint4 w = buf[bestv];
-#pragma unroll
-          for (int e = kVec - 1; e >= 0; --e)
-            if (vec_elem(w, e, (T*)nullptr) == best) bidx = bestv * kVec + e;
-        }
-        if (tailx > best) { best = tailx; bidx = nvec * kVec + lane; }
-        warp_argmax(best, bidx);
-      } else {
-        for (int i = 0; i < kVpl; ++i) {
-          const int v = lane + 32 * i;
-          if (v < nvec) best = fmaxf(best, vec_max(buf[v], (T*)nullptr));
-        }
-        best = fmaxf(best, tailx);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-        if (best > -INFINITY && best < INFINITY) {
-          const float M = __fmul_rn(best, chi);
-          float a = 0.0f;
-          if (fabsf(M) < 67108864.0f) {
-            const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
-            const float2 nM2 = make_float2(-M, -M);
-            float2 acc = make_float2(0.0f, 0.0f);
-            for (int i = 0; i < kVpl; ++i) {
-              const int v = lane + 32 * i;
-              if (v < nvec) acc = __fadd2_rn(acc, vec_expsum(buf[v], chi2, clo2, nM2, (T*)nullptr));
-            }
-            a = acc.x + acc.y;
-            if (lane < ntail) a += term(tailx, chi, clo, -M);
-          } else {
-            const float rr = fmaf(best, chi, -M) + best * clo;
-            for (int i = 0; i < kVpl; ++i) {
-              const int v = lane + 32 * i;
-              if (v < nvec) a += vec_expsum_far<T>(buf[v], best, chi, clo, rr);
-            }
-            if (lane < ntail) a += term_far(tailx, best, chi, clo, rr);
-          }
-          ssum = warp_sum_d((double)a);
+      const float tm = fmaxf(regs_max<kVpl>(x, (T*)nullptr), tailx);
+      if (tm > mrun) {
+        mrun = tm;
+        // Move the shift on the lane's first finite maximum, or when the
+        // exponents could exceed 2^kShiftSlack.
+        if (!(anchor > -INFINITY) || fmaf(tm, chi, -Msh) > kShiftSlack) {
+          const float Mn = __fmul_rn(tm, chi);
+          if (acc != 0.0) acc *= exp2((double)Msh - (double)Mn);
+          anchor = tm;
+          Msh = Mn;
         }
       }
-      refill(s);
+      const bool has = anchor > -INFINITY;
+      float a = 0.0f;
+      if (__all_sync(0xffffffffu, !has || fabsf(Msh) < kFarShift)) {
+        if (has) {
+          const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
+          const float2 nM2 = make_float2(-Msh, -Msh);
+          float2 a0 = make_float2(0.0f, 0.0f), a1 = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int i = 0; i < kVpl; i += 2) {
+            a0 = __fadd2_rn(a0, vec_expsum(x[i], chi2, clo2, nM2, (T*)nullptr));
+            if (i + 1 < kVpl) a1 = __fadd2_rn(a1, vec_expsum(x[i + 1], chi2, clo2, nM2, (T*)nullptr));
+          }
+          const float2 a2 = __fadd2_rn(a0, a1);
+          a = a2.x + a2.y;
+          if (lane < ntail) a += term(tailx, chi, clo, -Msh);
+        }
+      } else if (has) {
+        const float rr = fmaf(anchor, chi, -Msh) + anchor * clo;
+#pragma unroll
+        for (int i = 0; i < kVpl; ++i) a += vec_expsum_far<T>(x[i], anchor, chi, clo, rr);
+        if (lane < ntail) a += term_far(tailx, anchor, chi, clo, rr);
+      }
+      acc += (double)a;
     }
 
-    if (lane == 0) {
+    // End of the row or of this warp's items: one Partial for the run.
+    const int t_last = ct;
+    if (++ct == ntiles) { ct = 0; ++ck; }
+    if (ct == 0 || it + 1 == nmine) {
       Partial p;
-      p.m = best;
-      p.idx = bidx == 0x7fffffff ? bidx : t * kEpt + bidx;
-      p.s = ssum;
-      part[(size_t)r * ntiles + t] = p;
+      if (greedy) {
+        float v = mrun;
+        int i = gidx;
+        warp_argmax(v, i);
+        p.m = v;
+        p.idx = i;
+        p.s = 0.0;
+      } else {
+        float m = mrun;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        double sl = 0.0;
+        if (m > -INFINITY && m < INFINITY && acc != 0.0)
+          sl = acc * exp2((double)Msh - (double)__fmul_rn(m, chi));
+        p.m = m;
+        p.idx = 0x7fffffff;
+        p.s = warp_sum_d(sl);
+      }
+      Partial* prow = part + (size_t)row * ntiles;
+      if (lane == 0) prow[run_t0] = p;
+      for (int t = run_t0 + 1 + lane; t <= t_last; t += 32)
+        prow[t] = Partial{-INFINITY, 0x7fffffff, 0.0};
     }
-
-    advance(cons);
-    settle(cons);
   }
 
   if (timed_out) {
@@ -409,7 +421,8 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
   auto kern = row_stats_kernel<T, Rows>;
   static bool smem_set = false;  // once per instantiation (same on every B200)
   if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmem);
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmemTotal);
     if (e != cudaSuccess) {
       cudaGetLastError();  // do not leave the error pending for later calls
       return e;
@@ -417,14 +430,19 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
     smem_set = true;
   }
   constexpr int kEpt = kTileBytes / (int)sizeof(T);
-  const long long items = (long long)nrows * ((V + kEpt - 1) / kEpt);
-  if (items >= (1LL << 31)) return cudaErrorInvalidValue;
-  long long grid = rs_grid();
-  const long long need = (items + kRsWarps - 1) / kRsWarps;
-  if (grid > need) grid = need;
-  if (grid < 1) grid = 1;
-  return launch_pdl(kern, dim3((unsigned)grid), dim3(kRsWarps * 32), kRsSmem, st, rows, nrows, V,
-                    part, status);
+  const long long ntiles = (V + kEpt - 1) / kEpt;
+  for (int r0 = 0; r0 < nrows; r0 += kMaxListRows) {
+    const int n = nrows - r0 < kMaxListRows ? nrows - r0 : kMaxListRows;
+    const long long items = (long long)n * ntiles;
+    long long grid = rs_grid();
+    const long long need = (items + kRsWarps - 1) / kRsWarps;
+    if (grid > need) grid = need;
+    if (grid < 1) grid = 1;
+    const cudaError_t e = launch_pdl(kern, dim3((unsigned)grid), dim3(kRsWarps * 32),
+                                     (size_t)kRsSmemTotal, st, rows, r0, n, V, part, status);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <typename Rows>
