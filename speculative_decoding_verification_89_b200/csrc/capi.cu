@@ -126,6 +126,25 @@ const char* spec_status_string(int status) {
   }
 }
 
+// Leading positions whose rows the row-statistics kernel streams last, so
+// the draw that follows finds them in L2: as many (at most 2) as fit in 60%
+// of the L2 with rows_per_pos rows per position and sequence.
+static int late_positions(int B, int V, int dtype, int rows_per_pos) {
+  static int l2 = -1;  // bytes; the same on every device of a B200 node
+  if (l2 < 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
+      cudaGetLastError();
+      v = 0;
+    }
+    l2 = v;
+  }
+  const double per_pos = (double)B * rows_per_pos * V * elem_size(dtype);
+  const int n = per_pos > 0.0 ? (int)(0.6 * l2 / per_pos) : 0;
+  return n > 2 ? 2 : n;
+}
+
 int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
                          int dtype, int B, int K, int V, const float* temperature,
                          int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
@@ -140,6 +159,7 @@ int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64
   rows.ld_drf = ld_drf * es;
   rows.temperature = temperature;
   rows.K = K;
+  rows.late_pos = late_positions(B, V, dtype, 2);
   return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, ck.L),
                                       dev_status, (cudaStream_t)stream));
 }
@@ -230,6 +250,7 @@ int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64
   r1.K = K;
   r1.S = S;
   r1.Ni = Ni;
+  r1.late_pos = late_positions(B, V, dtype, 2);
   cudaError_t e = launch_row_stats(dtype, r1, B * (2 * K + 1), V, rsb, dev_status, st);
   if (e == cudaSuccess) e = launch_hier1_decide(a, st);
   Hier2Rows r2;
@@ -240,6 +261,7 @@ int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64
   r2.acc1 = acc1;
   r2.S = S;
   r2.Ni = Ni;
+  r2.late_pos = late_positions(B, V, dtype, 1);
   if (e == cudaSuccess) e = launch_row_stats(dtype, r2, B * S, V, rsb, dev_status, st);
   if (e == cudaSuccess) e = launch_hier2_decide(a, st);
   return cuda_status(e);

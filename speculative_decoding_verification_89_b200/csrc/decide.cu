@@ -35,32 +35,45 @@ constexpr int kCluster = 4;                  // CTAs per sequence
 constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kRowWarps = kDecWarps - 1;     // the last warp of a CTA serves the accept test
-constexpr int kUnroll = 4;                   // residual tiles in flight per warp
+// Residual tiles whose loads a warp keeps in flight together (64 bytes per
+// lane and row).
+template <typename T>
+constexpr int kResGroup = sizeof(T) == 2 ? 4 : 2;
 
 // ---------------------------------------------------------------------------
 // Residual weights of 8 consecutive elements
 // ---------------------------------------------------------------------------
+// 8 consecutive logits as raw 16-byte vectors (one for bf16, two for fp32);
+// zeros when `on` is false (nothing is read then).
 template <typename T>
-__device__ __forceinline__ void load8(const T* row, int e0, int V, float x[8]);
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* row, int e0, int V,
-                                                     float x[8]) {
-  if (e0 + 8 <= V) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + e0));
-    x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
-    x[4] = bf_lo(w.z); x[5] = bf_hi(w.z); x[6] = bf_lo(w.w); x[7] = bf_hi(w.w);
-  } else {
+struct Raw8 {
+  uint4 v[sizeof(T) / 2];
+};
+template <typename T>
+__device__ __forceinline__ Raw8<T> raw8(const T* row, int e0, bool on) {
+  Raw8<T> r;
+  const uint4* p = reinterpret_cast<const uint4*>(row + e0);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = (e0 + e < V) ? load_elem(row + e0 + e) : -INFINITY;
-  }
+  for (int i = 0; i < (int)(sizeof(T) / 2); ++i)
+    r.v[i] = on ? __ldg(p + i) : make_uint4(0u, 0u, 0u, 0u);
+  return r;
 }
-template <>
-__device__ __forceinline__ void load8<float>(const float* row, int e0, int V, float x[8]) {
+__device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16>& r, float x[8]) {
+  const uint4 w = r.v[0];
+  x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
+  x[4] = bf_lo(w.z); x[5] = bf_hi(w.z); x[6] = bf_lo(w.w); x[7] = bf_hi(w.w);
+}
+__device__ __forceinline__ void unpack8(const Raw8<float>& r, float x[8]) {
+  x[0] = __uint_as_float(r.v[0].x); x[1] = __uint_as_float(r.v[0].y);
+  x[2] = __uint_as_float(r.v[0].z); x[3] = __uint_as_float(r.v[0].w);
+  x[4] = __uint_as_float(r.v[1].x); x[5] = __uint_as_float(r.v[1].y);
+  x[6] = __uint_as_float(r.v[1].z); x[7] = __uint_as_float(r.v[1].w);
+}
+// Elements e0 .. e0+7 of a row of V elements; -inf past the end.
+template <typename T>
+__device__ __forceinline__ void load8(const T* row, int e0, int V, float x[8]) {
   if (e0 + 8 <= V) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(row + e0));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(row + e0 + 4));
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    unpack8(raw8(row, e0, true), x);
   } else {
 #pragma unroll
     for (int e = 0; e < 8; ++e) x[e] = (e0 + e < V) ? load_elem(row + e0 + e) : -INFINITY;
@@ -89,30 +102,38 @@ __device__ __forceinline__ float2 prob2(float2 x, const ProbCoef& k) {
   return make_float2(ex2(t.x), ex2(t.y));
 }
 
-// Weights w = max(0, p - q) (or p when there is no draft row) of 8 elements.
-template <typename T>
-__device__ __forceinline__ void weights8(const T* prow, const T* qrow, int e0, int V,
-                                         const ProbCoef& kp, const ProbCoef& kq, float w[8]) {
-  float xp[8];
-  load8<T>(prow, e0, V, xp);
-  if (qrow) {
-    float xq[8];
-    load8<T>(qrow, e0, V, xq);
+// Weights w = max(0, p - q) (or p when there is no draft row) of 8 elements
+// given their logits.
+__device__ __forceinline__ void weights_of(const float xp[8], const float xq[8], bool has_q,
+                                           const ProbCoef& kp, const ProbCoef& kq, float w[8]) {
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float2 p = prob2(make_float2(xp[e], xp[e + 1]), kp);
+  for (int e = 0; e < 8; e += 2) {
+    const float2 p = prob2(make_float2(xp[e], xp[e + 1]), kp);
+    if (has_q) {
       const float2 q = prob2(make_float2(xq[e], xq[e + 1]), kq);
       w[e] = fmaxf(p.x - q.x, 0.0f);
       w[e + 1] = fmaxf(p.y - q.y, 0.0f);
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float2 p = prob2(make_float2(xp[e], xp[e + 1]), kp);
+    } else {
       w[e] = p.x;
       w[e + 1] = p.y;
     }
   }
+}
+// Same, reading the 8 elements at e0 (any e0 < V).
+template <typename T>
+__device__ __forceinline__ void weights8(const T* prow, const T* qrow, int e0, int V,
+                                         const ProbCoef& kp, const ProbCoef& kq, float w[8]) {
+  float xp[8], xq[8];
+  if (e0 + 8 <= V) {  // both loads in flight together
+    const Raw8<T> rp = raw8(prow, e0, true);
+    const Raw8<T> rq = raw8(qrow ? qrow : prow, e0, qrow != nullptr);
+    unpack8(rp, xp);
+    unpack8(rq, xq);
+  } else {
+    load8<T>(prow, e0, V, xp);
+    if (qrow) load8<T>(qrow, e0, V, xq);
+  }
+  weights_of(xp, xq, qrow != nullptr, kp, kq, w);
 }
 // A lane's 8 weights summed pairwise in fp32 (error ~ 3 ulp of the small
 // sum), then widened; tiles and lanes combine in fp64.
@@ -128,26 +149,44 @@ __device__ __forceinline__ double lane_sum8(const float w[8]) {
 // Residual tile sums and the draw
 // ---------------------------------------------------------------------------
 // Tile sums of the weights over residual tiles [t0, t1), written to out
-// (the leader CTA's shared memory, possibly remote).
+// (the leader CTA's shared memory, possibly remote). A warp takes groups of
+// kResGroup tiles and issues all their loads before using any.
 template <typename T>
 __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const ProbCoef& kp,
                                    const ProbCoef& kq, int t0, int t1, double* out) {
+  constexpr int G = kResGroup<T>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int tb = t0 + warp * kUnroll; tb < t1; tb += kDecWarps * kUnroll) {
-    double s[kUnroll];
+  const bool hq = qrow != nullptr;
+  for (int tb = t0 + warp * G; tb < t1; tb += kDecWarps * G) {
+    Raw8<T> rp[G], rq[G];
+    bool full[G];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int t = tb + u;
+    for (int u = 0; u < G; ++u) {
+      const int e0 = (tb + u) * kResTile + lane * 8;
+      full[u] = tb + u < t1 && e0 + 8 <= V;
+      rp[u] = raw8(prow, e0, full[u]);
+      rq[u] = raw8(hq ? qrow : prow, e0, full[u] && hq);
+    }
+    double s[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      const int t = tb + u, e0 = t * kResTile + lane * 8;
       float w[8];
-      if (t < t1) {
-        weights8<T>(prow, qrow, t * kResTile + lane * 8, V, kp, kq, w);
-        s[u] = lane_sum8(w);
+      if (full[u]) {
+        float xp[8], xq[8];
+        unpack8(rp[u], xp);
+        unpack8(rq[u], xq);
+        weights_of(xp, xq, hq, kp, kq, w);
+      } else if (t < t1 && e0 < V) {
+        weights8<T>(prow, qrow, e0, V, kp, kq, w);  // the row's ragged end
       } else {
-        s[u] = 0.0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = 0.0f;
       }
+      s[u] = lane_sum8(w);
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < G; ++u) {
       const double v = warp_sum_d(s[u]);
       if (lane == 0 && tb + u < t1) out[tb + u] = v;
     }
@@ -161,38 +200,44 @@ template <typename T>
 __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef& kp,
                              const ProbCoef& kq, const double* tsum, double* pre, int nrt,
                              float u, double* Z_out) {
-  __shared__ double s_Z;
+  __shared__ double s_wtot[kDecWarps];
   __shared__ int s_tile, s_tok;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp == 0) {
-    // Each lane owns a contiguous run of tiles; lane sums are scanned.
-    const int per = (nrt + 31) / 32;
-    const int a = min(nrt, lane * per), b = min(nrt, a + per);
-    double run = 0.0;
-    for (int t = a; t < b; ++t) run += tsum[t];
-    double incl = run;
+  // Each thread owns a contiguous run of tiles; the run sums are scanned over
+  // the block (warp shuffles, then the warp totals in order).
+  const int per = (nrt + kDecThreads - 1) / kDecThreads;
+  const int a = min(nrt, (int)threadIdx.x * per), b = min(nrt, a + per);
+  double run = 0.0;
+  for (int t = a; t < b; ++t) run += tsum[t];
+  double incl = run;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    double c = __shfl_up_sync(0xffffffffu, incl, 1);
-    if (lane == 0) c = 0.0;
-    for (int t = a; t < b; ++t) {
-      pre[t] = c;
-      c += tsum[t];
-    }
-    if (lane == 31) s_Z = incl;
-    if (lane == 0) s_tile = -1;
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  if (lane == 31) s_wtot[warp] = incl;
+  if (threadIdx.x == 0) s_tile = -1;
   __syncthreads();
-  const double Z = s_Z;
+  double Z = 0.0, c = 0.0;
+#pragma unroll
+  for (int w = 0; w < kDecWarps; ++w) {
+    if (w == warp) c = Z;
+    Z += s_wtot[w];
+  }
   *Z_out = Z;
   if (!(Z > 0.0)) return -1;
   const double target = (double)u * Z;
   // The last tile with mass whose prefix does not exceed the target.
-  for (int t = threadIdx.x; t < nrt; t += blockDim.x)
-    if (pre[t] <= target && tsum[t] > 0.0) atomicMax(&s_tile, t);
+  c += excl;
+  int cand = -1;
+  for (int t = a; t < b; ++t) {
+    pre[t] = c;
+    if (c <= target && tsum[t] > 0.0) cand = t;
+    c += tsum[t];
+  }
+  if (cand >= 0) atomicMax(&s_tile, cand);
   __syncthreads();
   const int tile = s_tile < 0 ? 0 : s_tile;  // s_tile >= 0 whenever Z > 0
   if (warp == 0) {
@@ -263,32 +308,45 @@ struct SeqShared {
   int ok[kMaxRows];
 };
 
+// Split cluster barrier: every CTA arrives once it runs; a thread waits (once)
+// before its first access to another CTA's shared memory.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait;" ::: "memory");
+}
+
 // Combine the tile partials of a sequence's rows (a warp per row, over the
 // row warps of all CTAs of the cluster) into the leader's SeqShared (lsh,
-// distributed shared memory) and the RowFinal array.
+// distributed shared memory) and the RowFinal array. Completes the start
+// barrier of the cluster in every thread: the first row's partials are read
+// before the wait.
 template <typename Want>
 __device__ void cluster_rows(SeqShared* lsh, unsigned rank, const Partial* part, int ntiles,
                              int row0, int nrows, Want want, bool greedy, float chi,
                              RowFinal* fin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp >= kRowWarps) return;
-  for (int r = (int)rank * kRowWarps + warp; r < nrows; r += kCluster * kRowWarps) {
-    if (!want(r)) {
-      if (lane == 0) {
-        lsh->ok[r] = 1; lsh->m[r] = 0.f; lsh->M[r] = 0; lsh->L[r] = 0; lsh->amax[r] = -1;
+  bool waited = false;
+  if (warp < kRowWarps) {
+    for (int r = (int)rank * kRowWarps + warp; r < nrows; r += kCluster * kRowWarps) {
+      RowFinal f{0.0, 0.0, 0.f, -1, 1, 0};
+      if (want(r)) f = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, chi, lane);
+      if (!waited) {
+        cluster_wait();
+        waited = true;
       }
-      continue;
-    }
-    const RowFinal f = combine_row(part + (size_t)(row0 + r) * ntiles, ntiles, greedy, chi, lane);
-    if (lane == 0) {
-      fin[row0 + r] = f;
-      lsh->m[r] = f.m;
-      lsh->M[r] = f.M;
-      lsh->L[r] = f.L;
-      lsh->amax[r] = f.amax;
-      lsh->ok[r] = f.ok;
+      if (lane == 0) {
+        if (want(r)) fin[row0 + r] = f;
+        lsh->m[r] = f.m;
+        lsh->M[r] = f.M;
+        lsh->L[r] = f.L;
+        lsh->amax[r] = f.amax;
+        lsh->ok[r] = f.ok;
+      }
     }
   }
+  if (!waited) cluster_wait();
 }
 
 template <typename T>
@@ -297,17 +355,21 @@ __device__ __forceinline__ const T* row_ptr(const unsigned char* base, long long
   return reinterpret_cast<const T*>(base + row * ld_bytes);
 }
 
-// Logits of the drafted tokens for the first 32 positions, fetched by the
-// accept warp while the other warps combine the rows.
+// Logits of the drafted tokens and the Philox uniforms of the first 32
+// positions, fetched by the accept warp while the other warps combine the
+// rows.
 struct AcceptPre {
   int x;         // draft id of position lane (or -1 past n)
   float lt, ld;  // target / draft logit at x
+  float ua, ud;  // accept and draw uniforms of position pos0 + lane
 };
 template <typename T, typename TP, typename DP>
 __device__ __forceinline__ AcceptPre accept_prefetch(int n, int V, bool greedy,
-                                                     const int32_t* drafts, TP tp, DP dp) {
+                                                     const int32_t* drafts, TP tp, DP dp,
+                                                     const DecideCommon& c, int b, int pos0,
+                                                     int stage) {
   const int lane = threadIdx.x & 31;
-  AcceptPre a{-1, 0.f, 0.f};
+  AcceptPre a{-1, 0.f, 0.f, 0.f, 0.f};
   if (lane < n) {
     a.x = drafts[lane];
     if (!greedy && a.x >= 0 && a.x < V) {
@@ -315,20 +377,28 @@ __device__ __forceinline__ AcceptPre accept_prefetch(int n, int V, bool greedy,
       a.ld = load_elem(dp(lane) + a.x);
     }
   }
+  if (lane <= n && !greedy) {
+    const float2 u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round,
+                                   (uint32_t)(pos0 + lane), (uint32_t)stage);
+    a.ua = u.x;
+    a.ud = u.y;
+  }
   return a;
 }
 
 // One speculative check on n positions (one warp). Target row j: tp(j) with
 // log2 partition sh.M + sh.L at index j; draft law of position j: row dp(j)
 // with log2 partition dlt(j). Returns a (first rejection, n if none) in every
-// lane; *bad is set if a draft id lies outside [0, V). Writes p_j(x_j) and
-// q_j(x_j) to diag_p / diag_q when given. Positions below 32 use the
-// prefetched logits.
+// lane; *bad is set if a draft id lies outside [0, V); *u_draw gets the draw
+// uniform of position a (sampled rows only). Writes p_j(x_j) and q_j(x_j) to
+// diag_p / diag_q when given. Positions below 32 use the prefetched logits
+// and uniforms.
 template <typename T, typename TP, typename DP, typename DS>
 __device__ int accept_scan(const SeqShared* sh, int n, int pos0, int stage,
                            const DecideCommon& c, int b, bool greedy, double cd,
                            const int32_t* drafts, TP tp, DP dp, DS dlt, double* diag_p,
-                           double* diag_q, const AcceptPre& pre, int* bad_out) {
+                           double* diag_q, const AcceptPre& pre, int* bad_out,
+                           float* u_draw) {
   const int lane = threadIdx.x & 31;
   int a = n, bad = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
@@ -345,8 +415,9 @@ __device__ int accept_scan(const SeqShared* sh, int n, int pos0, int stage,
         const float ld = j0 == 0 ? pre.ld : load_elem(dp(j) + x);
         const double lp = (double)lt * cd - (sh->M[j] + sh->L[j]);
         const double lq = (double)ld * cd - dlt(j);
-        const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(pos0 + j),
-                                      (uint32_t)stage).x;
+        const float u = j0 == 0 ? pre.ua
+                                : spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round,
+                                                (uint32_t)(pos0 + j), (uint32_t)stage).x;
         acc = (double)u < exp2(lp - lq);
         if (diag_p) { diag_p[j] = exp2(lp); diag_q[j] = exp2(lq); }
       }
@@ -356,6 +427,10 @@ __device__ int accept_scan(const SeqShared* sh, int n, int pos0, int stage,
     if (rej && a == n) a = j0 + __ffs(rej) - 1;
   }
   *bad_out = bad;
+  const float ud = __shfl_sync(0xffffffffu, pre.ud, a & 31);
+  *u_draw = (a < 32 || greedy) ? ud
+                               : spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round,
+                                               (uint32_t)(pos0 + a), (uint32_t)stage).y;
   return a;
 }
 
@@ -368,6 +443,7 @@ __device__ __forceinline__ bool rows_ok(const SeqShared* sh, int nrows) {
 // Per-CTA outcome of the accept test (every CTA of the cluster computes it).
 struct Outcome {
   int a, bad;
+  float u_draw;
 };
 
 // ---------------------------------------------------------------------------
@@ -376,6 +452,7 @@ struct Outcome {
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecideArgs A) {
   grid_dependency_wait();
+  cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
@@ -408,17 +485,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
   auto dl = [&](int j) { return lsh->M[K + 1 + j] + lsh->L[K + 1 + j]; };
   const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
   AcceptPre pre{-1, 0.f, 0.f};
-  cl.sync();  // every CTA of the cluster is running: its shared memory may be used
-  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp);
+  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp, c, b, 0, 1);
   cluster_rows(lsh, rank, c.part, c.ntiles, b * per, per,
                [&](int r) { return r <= K || !greedy; }, greedy, sc.hi, c.fin);
   cl.sync();  // the leader holds every row's statistics
   if (accept_warp) {
     int bad;
+    float ud;
     const int a = accept_scan<T>(lsh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
                                  diag && !greedy ? diag + 2 * K + 1 : nullptr,
-                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad);
-    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per)};
+                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad, &ud);
+    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per), ud};
   }
   __syncthreads();
   const Outcome o = s_out;
@@ -448,7 +525,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
   if (greedy) {
     tok = sh.amax[a];
   } else {
-    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 1u).y;
+    const float u = o.u_draw;
     tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
   }
   for (int j = threadIdx.x; j <= K; j += blockDim.x)
@@ -492,6 +569,7 @@ __device__ __forceinline__ void window_append(const HierDecideArgs& A, int b, in
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecideArgs A) {
   grid_dependency_wait();
+  cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
@@ -531,17 +609,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
   auto dl = [&](int j) { return lsh->M[K + 1 + j] + lsh->L[K + 1 + j]; };
   const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
   AcceptPre pre{-1, 0.f, 0.f};
-  cl.sync();
-  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp);
+  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp, c, b, w, 1);
   cluster_rows(lsh, rank, c.part, c.ntiles, b * per, per,
                [&](int r) { return r <= K || !greedy; }, greedy, sc.hi, c.fin);
   cl.sync();
   if (accept_warp) {
     int bad;
+    float ud;
     const int a = accept_scan<T>(lsh, K, w, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
                                  diag && !greedy ? diag + 2 * K + 1 : nullptr,
-                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad);
-    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per)};
+                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad, &ud);
+    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per), ud};
   }
   __syncthreads();
   const Outcome o = s_out;
@@ -571,7 +649,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
   if (greedy) {
     tok = sh.amax[a];
   } else {
-    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)(w + a), 1u).y;
+    const float u = o.u_draw;
     tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
   }
   window_append(A, b, w, a, drafts, tok, sh, greedy, sc.d);
@@ -593,6 +671,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecideArgs A) {
   grid_dependency_wait();
+  cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
@@ -616,17 +695,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
   auto dl = [&](int j) { return wst[2 * j] * sc.d + wst[2 * j + 1] * kLog2e; };
   const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
   AcceptPre pre{-1, 0.f, 0.f};
-  cl.sync();
-  if (accept_warp) pre = accept_prefetch<T>(W, V, greedy, wtok, tp, dp);
+  if (accept_warp) pre = accept_prefetch<T>(W, V, greedy, wtok, tp, dp, c, b, 0, 2);
   cluster_rows(lsh, rank, c.part, c.ntiles, b * S, W + 1, [&](int) { return true; }, greedy,
                sc.hi, c.fin);
   cl.sync();
   if (accept_warp) {
     int bad;
+    float ud;
     const int a = accept_scan<T>(lsh, W, 0, 2, c, b, greedy, sc.d, wtok, tp, dp, dl,
                                  diag && !greedy ? diag + S : nullptr,
-                                 diag && !greedy ? diag + 2 * S - 1 : nullptr, pre, &bad);
-    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, W + 1)};
+                                 diag && !greedy ? diag + 2 * S - 1 : nullptr, pre, &bad, &ud);
+    if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, W + 1), ud};
   }
   __syncthreads();
   const Outcome o = s_out;
@@ -659,7 +738,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
   if (greedy) {
     tok = sh.amax[a];
   } else {
-    const float u = spec_uniforms(c.seed, (uint32_t)c.seq_id[b], c.round, (uint32_t)a, 2u).y;
+    const float u = o.u_draw;
     tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
   }
   for (int j = threadIdx.x; j < WC + 1; j += blockDim.x)

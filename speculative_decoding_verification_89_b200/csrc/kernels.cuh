@@ -20,6 +20,11 @@ __device__ __forceinline__ RowRef make_row(const unsigned char* ptr, float T, bo
   return r;
 }
 
+// Each Rows type also names its "late" rows: those of positions below
+// late_pos, which the draw after the check is most likely to read again (the
+// first rejection falls at position j with probability decreasing in j). The
+// row-statistics kernel streams them last so they are still in L2.
+
 // Chain verification rows, grouped by sequence: for sequence b, rows
 // b*(2K+1) + j are target row j (j <= K) and then draft row j - K - 1.
 struct ChainRows {
@@ -28,6 +33,11 @@ struct ChainRows {
   long long ld_tgt, ld_drf;  // row strides in bytes
   const float* temperature;
   int K;
+  int late_pos;
+  __device__ __forceinline__ bool late(int r) const {
+    const int per = 2 * K + 1, j = r % per;
+    return (j <= K ? j : j - K - 1) < late_pos;
+  }
   __device__ __forceinline__ RowRef get(int r) const {
     const int per = 2 * K + 1, b = r / per, j = r - b * per;
     const float T = __ldg(temperature + b);
@@ -45,6 +55,11 @@ struct Hier1Rows {
   const float* temperature;
   const int32_t* win_len;
   int K, S, Ni;
+  int late_pos;
+  __device__ __forceinline__ bool late(int r) const {
+    const int per = 2 * K + 1, j = r % per;
+    return (j <= K ? j : j - K - 1) < late_pos;
+  }
   __device__ __forceinline__ RowRef get(int r) const {
     const int per = 2 * K + 1, b = r / per, j = r - b * per;
     const float T = __ldg(temperature + b);
@@ -66,6 +81,8 @@ struct Hier2Rows {
   const int32_t* win_len;
   const int32_t* acc1;
   int S, Ni;
+  int late_pos;
+  __device__ __forceinline__ bool late(int r) const { return r % S < late_pos; }
   __device__ __forceinline__ RowRef get(int r) const {
     const int b = r / S, s = r - b * S;
     const int W = win_len[b];

@@ -166,17 +166,24 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   }
   grid_dependency_wait();
 
-  // The rows that need statistics, in order: each thread tests a contiguous
-  // run of at most 32 rows, a block scan places them.
+  // The rows that need statistics: the early ones in order, then the late
+  // ones in order. Each thread tests a contiguous run of at most 32 rows; a
+  // block scan of the packed counts (early | late << 16) places them.
+  int n_early = 0, n_late = 0;
   {
     const int per = (nrows + kThreads - 1) / kThreads;
     const int q0 = min(nrows, (int)threadIdx.x * per), q1 = min(nrows, q0 + per);
-    uint32_t vmask = 0;
+    uint32_t vmask = 0, lmask = 0;
     int cnt = 0;
     for (int q = q0; q < q1; ++q)
       if (rows.get(row_base + q).valid) {
         vmask |= 1u << (q - q0);
-        ++cnt;
+        if (rows.late(row_base + q)) {
+          lmask |= 1u << (q - q0);
+          cnt += 1 << 16;
+        } else {
+          cnt += 1;
+        }
       }
     int incl = cnt;
 #pragma unroll
@@ -186,49 +193,82 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     }
     if (lane == 31) s_wsum[warp] = incl;
     __syncthreads();
-    int pos = incl - cnt;
-    for (int w = 0; w < warp; ++w) pos += s_wsum[w];
+    int pos = incl - cnt, tot = 0;
+    for (int w = 0; w < kRsWarps; ++w) {
+      if (w < warp) pos += s_wsum[w];
+      tot += s_wsum[w];
+    }
+    n_early = tot & 0xffff;
+    n_late = tot >> 16;
+    int pe = pos & 0xffff, pl = n_early + (pos >> 16);
     for (int q = q0; q < q1; ++q)
-      if ((vmask >> (q - q0)) & 1u) s_list[pos++] = q;
+      if ((vmask >> (q - q0)) & 1u) s_list[((lmask >> (q - q0)) & 1u) ? pl++ : pe++] = q;
   }
-  int nlisted = 0;
-  for (int w = 0; w < kRsWarps; ++w) nlisted += s_wsum[w];
   __syncthreads();
 
-  // This warp's run of items [i0, i1) over (listed row, tile).
+  // This warp's items: a contiguous share of the early rows' (listed row,
+  // tile) items, then a contiguous share of the late rows' items.
   const int ntiles = (V + kEpt - 1) / kEpt;
-  const long long nitems = (long long)nlisted * ntiles;
   const int gw = blockIdx.x * kRsWarps + warp, nw = gridDim.x * kRsWarps;
-  const long long i0 = nitems * gw / nw, i1 = nitems * (gw + 1) / nw;
-  const int nmine = (int)(i1 - i0);
-  const int k0 = (int)(i0 / ntiles), t0 = (int)(i0 - (long long)k0 * ntiles);
+  const long long ne = (long long)n_early * ntiles, nl = (long long)n_late * ntiles;
+  const long long e0 = ne * gw / nw, e1 = ne * (gw + 1) / nw;
+  const long long l0 = ne + nl * gw / nw, l1 = ne + nl * (gw + 1) / nw;
+  struct Cursor {
+    int k, t, left, seg;  // listed row, tile, items left in segment, segment
+  };
+  auto start = [&](Cursor& c, long long i, long long n, int seg) {
+    c.k = (int)(i / ntiles);
+    c.t = (int)(i - (long long)c.k * ntiles);
+    c.left = (int)n;
+    c.seg = seg;
+  };
+  auto begin = [&](Cursor& c) {
+    start(c, e0, e1 - e0, 0);
+    if (c.left == 0) start(c, l0, l1 - l0, 1);
+  };
+  auto advance = [&](Cursor& c) {
+    if (++c.t == ntiles) { c.t = 0; ++c.k; }
+    if (--c.left == 0 && c.seg == 0) start(c, l0, l1 - l0, 1);
+  };
+  // Streamed-once lines make room first when late rows are to stay in L2.
+  const bool hint = n_late > 0;
+  const uint64_t pol = l2_evict_first();
 
   // Producer: lane 0 issues the copies, every lane keeps the cursor.
-  int pk = k0, pt = t0, pleft = nmine, pk_row = -1;
+  Cursor pc;
+  begin(pc);
+  int pk_row = -1;
   const unsigned char* pptr = nullptr;
   auto issue = [&](int st) {
-    if (pk != pk_row) {
-      pk_row = pk;
-      pptr = rows.get(row_base + s_list[pk]).ptr;
+    if (pc.k != pk_row) {
+      pk_row = pc.k;
+      pptr = rows.get(row_base + s_list[pc.k]).ptr;
     }
     if (lane == 0) {
-      const int nel = min(kEpt, V - pt * kEpt);
+      const int nel = min(kEpt, V - pc.t * kEpt);
       const uint32_t bytes = ((uint32_t)nel * sizeof(T)) & ~15u;
       fence_proxy_async_smem();  // the warp's reads of this stage come first
       mbar_arrive_expect_tx(&bars[st], bytes);
-      if (bytes) bulk_g2s(wbuf + st * kTileBytes, pptr + (size_t)pt * kTileBytes, bytes, &bars[st]);
+      const unsigned char* src = pptr + (size_t)pc.t * kTileBytes;
+      if (bytes) {
+        if (hint && pc.seg == 0)
+          bulk_g2s_hint(wbuf + st * kTileBytes, src, bytes, &bars[st], pol);
+        else
+          bulk_g2s(wbuf + st * kTileBytes, src, bytes, &bars[st]);
+      }
     }
-    if (++pt == ntiles) { pt = 0; ++pk; }
-    --pleft;
+    advance(pc);
   };
   int inflight = 0;
-  for (int st = 0; st < kRsStages && pleft > 0; ++st) {
+  for (int st = 0; st < kRsStages && pc.left > 0; ++st) {
     issue(st);
     ++inflight;
   }
 
   // Consumer state of the current row run (per lane).
-  int ck = k0, ct = t0;
+  Cursor cc;
+  begin(cc);
+  bool fresh = true;  // the next item starts a row run
   uint32_t phase = 0;
   bool timed_out = false;
   int s = 0;  // stage of the item being consumed
@@ -242,7 +282,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   double acc = 0.0;          // sum of 2^(l*c - Msh) over the lane's elements
   int gidx = 0x7fffffff;     // greedy rows: first index of mrun
 
-  for (int it = 0; it < nmine; ++it, s = (s + 1 == kRsStages) ? 0 : s + 1) {
+  for (; cc.left > 0; s = (s + 1 == kRsStages) ? 0 : s + 1) {
     const bool ok = mbar_wait_bounded(&bars[s], (phase >> s) & 1u, kWaitLimitNs);
     if (__any_sync(0xffffffffu, !ok)) {
       timed_out = true;
@@ -251,8 +291,10 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     phase ^= 1u << s;
     --inflight;
 
-    if (it == 0 || ct == 0) {  // a row run starts
-      row = row_base + s_list[ck];
+    const int ct = cc.t;
+    if (fresh) {  // a row run starts
+      fresh = false;
+      row = row_base + s_list[cc.k];
       const RowRef ref = rows.get(row);
       rptr = reinterpret_cast<const T*>(ref.ptr);
       greedy = (ref.T == 0.0f);
@@ -290,7 +332,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       if (lane < ntail) tailx = load_elem(rptr + (size_t)ct * kEpt + nvec * kVec + lane);
     }
     __syncwarp();
-    if (pleft > 0) {
+    if (pc.left > 0) {
       issue(s);
       ++inflight;
     }
@@ -359,10 +401,12 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       acc += (double)a;
     }
 
-    // End of the row or of this warp's items: one Partial for the run.
-    const int t_last = ct;
-    if (++ct == ntiles) { ct = 0; ++ck; }
-    if (ct == 0 || it + 1 == nmine) {
+    // End of the row, of a segment or of this warp's items: one Partial for
+    // the run.
+    const int t_last = ct, k_was = cc.k;
+    advance(cc);
+    if (cc.k != k_was || cc.left == 0) {
+      fresh = true;
       Partial p;
       if (greedy) {
         float v = mrun;
