@@ -21,6 +21,7 @@ namespace specv {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kCopyThreads = 256;
+constexpr int kCopyCtasPerSm = 8;  // 64 warps per SM: one round of items for most calls
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -59,16 +60,24 @@ __device__ int3 block_excl_scan3(int3 v, int3* tot) {
   return make_int3(base.x + incl.x - v.x, base.y + incl.y - v.y, base.z + incl.z - v.z);
 }
 
-// One CTA. Per-sequence inputs are read once into shared memory; every check
-// is made before anything is written.
+// One CTA. Two rounds of global reads: (1) the per-sequence lengths and
+// counts, (2) after a block scan, every covered table entry (validation), the
+// tails to be freed and the stack entries to be popped below the old top,
+// the last two cached in shared memory. Every check is made before anything
+// is written; the writes then need no further reads while the caches hold.
+constexpr int kPushCache = 2048;   // freed entries cached in push order
+constexpr int kStackCache = 2048;  // stack entries popped from below the old top
+
 __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a) {
   grid_dependency_wait();
-  extern __shared__ int s_seq[];  // [3][B]: blocks before, blocks after, kept
+  extern __shared__ int s_seq[];  // [3][B]: blocks before, new length, kept
   int* s_nbo = s_seq;
-  int* s_nbn = s_seq + a.B;
+  int* s_len = s_seq + a.B;
   int* s_kept = s_seq + 2 * a.B;
-  __shared__ int s_bad, s_code, s_ft;
-  if (threadIdx.x == 0) { s_bad = 0; s_code = 0; s_ft = *a.free_top; }
+  __shared__ int s_push[kPushCache];
+  __shared__ int s_stack[kStackCache];
+  __shared__ int s_bad, s_sbad, s_code, s_ft;
+  if (threadIdx.x == 0) { s_bad = 0; s_sbad = 0; s_code = 0; s_ft = *a.free_top; }
   if (a.status && *(volatile int32_t*)a.status != SPEC_OK) return;  // sticky error (uniform)
   const int bs = a.block_size;
   // Each thread owns a contiguous run of sequences (sequence order matters
@@ -82,86 +91,102 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
     const int base = a.base_len ? a.base_len[b] : old_len;
     const int kept = a.keep[b] + a.keep_add;
     int nbo = ceil_div(max(old_len, 0), bs), nbn = nbo;
+    bool ok = true;
     if (kept < 0 || kept > a.Kp1 || base < 0 || base > old_len || old_len < 0) {
-      bad = 1;
+      ok = false;
     } else {
       nbn = ceil_div(base + kept, bs);
-      if (nbo > a.max_blocks || nbn > a.max_blocks) bad = 1;
+      if (nbo > a.max_blocks || nbn > a.max_blocks) ok = false;
     }
+    if (!ok) bad = 1;
     s_nbo[b] = min(nbo, a.max_blocks);
-    s_nbn[b] = nbn;
+    s_len[b] = ok ? base + kept : 0;
     s_kept[b] = kept;
     cnt.x += max(0, nbo - nbn);
     cnt.y += max(0, nbn - nbo);
     cnt.z += kept;
   }
-  __syncthreads();
-  // Every covered table entry must be a valid block id: a warp per sequence,
-  // its lanes over the table entries, loads batched.
-  {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    constexpr int kBatch = 8;
-    for (int b = warp; b < a.B; b += nwarps) {
-      const int nb = s_nbo[b];
-      const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-      for (int i0 = lane; i0 < nb; i0 += 32 * kBatch) {
-        int v[kBatch];
-#pragma unroll
-        for (int k = 0; k < kBatch; ++k) v[k] = (i0 + 32 * k < nb) ? tab[i0 + 32 * k] : 0;
-#pragma unroll
-        for (int k = 0; k < kBatch; ++k)
-          if (i0 + 32 * k < nb && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
-      }
-    }
-  }
   if (bad) atomicOr(&s_bad, 1);
   int3 tot;
-  const int3 pre = block_excl_scan3(cnt, &tot);  // its barriers also publish s_bad
+  const int3 pre = block_excl_scan3(cnt, &tot);  // its barriers also publish s_ft, s_bad
   const int F = tot.x, A = tot.y, KT = tot.z, ft = s_ft;
-  if (threadIdx.x == 0) {
-    if (s_bad || ft < 0 || ft > a.num_blocks || ft + F > a.num_blocks) s_code = SPEC_EINVAL;
-    else if (ft + F < A) s_code = SPEC_ENOBLOCKS;
+  const bool sizes_ok = !s_bad && ft >= 0 && ft <= a.num_blocks && ft + F <= a.num_blocks;
+  // Pops come from stack positions [lo, ft + F): those at or above ft are the
+  // entries pushed by this call, those below ft are read here.
+  const int lo = max(0, ft + F - A);
+  const bool cached = F <= kPushCache && ft - lo <= kStackCache;
+  if (sizes_ok) {
+    // Every covered table entry must be a valid block id: a warp per
+    // sequence, its lanes over the entries, loads batched.
+    {
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+      constexpr int kBatch = 8;
+      for (int b = warp; b < a.B; b += nwarps) {
+        const int nb = s_nbo[b];
+        const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+        for (int i0 = lane; i0 < nb; i0 += 32 * kBatch) {
+          int v[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) v[k] = (i0 + 32 * k < nb) ? tab[i0 + 32 * k] : 0;
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k)
+            if (i0 + 32 * k < nb && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
+        }
+      }
+    }
+    // Tails to be freed, cached in push order (same round of reads).
+    if (cached) {
+      int fpos = pre.x;
+      for (int b = b0; b < b1; ++b) {
+        const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+        for (int i = ceil_div(s_len[b], bs); i < s_nbo[b]; ++i) s_push[fpos++] = tab[i];
+      }
+    }
+    if (bad) atomicOr(&s_bad, 1);
+    // Stack entries popped from below the old top must be valid ids.
+    int sbad = 0;
+    for (int p = lo + threadIdx.x; p < ft; p += blockDim.x) {
+      const int x = a.free_stack[p];
+      if (x < 0 || x >= a.num_blocks) sbad = 1;
+      if (cached) s_stack[p - lo] = x;
+    }
+    if (sbad) atomicOr(&s_sbad, 1);
   }
   __syncthreads();
-  // Blocks handed out come from stack positions [ft + F - A, ft + F); the
-  // ones below ft must be valid ids (the pushed ones were checked above).
-  if (s_code == 0)
-    for (int p = max(0, ft + F - A) + threadIdx.x; p < ft; p += blockDim.x) {
-      const int x = a.free_stack[p];
-      if (x < 0 || x >= a.num_blocks) atomicOr(&s_bad, 1);
-    }
-  __syncthreads();
-  if (threadIdx.x == 0 && s_code == 0 && s_bad) s_code = SPEC_EINVAL;
+  if (threadIdx.x == 0) {  // the order of the checks fixes which status wins
+    if (!sizes_ok || s_bad) s_code = SPEC_EINVAL;
+    else if (ft + F < A) s_code = SPEC_ENOBLOCKS;
+    else if (s_sbad) s_code = SPEC_EINVAL;
+  }
   __syncthreads();
   if (s_code != 0) {
     if (threadIdx.x == 0) set_status(a.status, s_code);
     return;
   }
   // Frees: push table tails in sequence order.
-  int fpos = ft + pre.x;
+  int fpos = pre.x;
   for (int b = b0; b < b1; ++b) {
     int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-    for (int i = s_nbn[b]; i < s_nbo[b]; ++i) {
-      a.free_stack[fpos++] = tab[i];
+    for (int i = ceil_div(s_len[b], bs); i < s_nbo[b]; ++i) {
+      a.free_stack[ft + fpos] = cached ? s_push[fpos] : tab[i];
+      ++fpos;
       tab[i] = -1;
     }
   }
-  __syncthreads();
+  if (!cached) __syncthreads();  // pops below read the pushed entries back
   // Allocations: pop from the top in sequence order; lengths and offsets.
   const int top = ft + F;
   int k = pre.y, off = pre.z;
   for (int b = b0; b < b1; ++b) {
     int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-    for (int i = s_nbo[b]; i < s_nbn[b]; ++i) tab[i] = a.free_stack[top - 1 - (k++)];
+    const int nbn = ceil_div(s_len[b], bs);
+    for (int i = s_nbo[b]; i < nbn; ++i) {
+      const int p = top - 1 - (k++);
+      tab[i] = !cached ? a.free_stack[p] : (p >= ft ? s_push[p - ft] : s_stack[p - lo]);
+    }
     if (a.hid_off) a.hid_off[b] = off;
     off += s_kept[b];
-  }
-  // New lengths: base + kept (base read above for the checks; read again
-  // here because base_len may be the same array as seq_lens).
-  __syncthreads();
-  for (int b = b0; b < b1; ++b) {
-    const int base = a.base_len ? a.base_len[b] : a.seq_lens[b];
-    a.seq_lens[b] = base + s_kept[b];
+    a.seq_lens[b] = s_len[b];
   }
   if (threadIdx.x == 0) {
     *a.free_top = top - A;
@@ -258,7 +283,8 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
         cudaFuncSetAttribute(commit_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)csmem) != cudaSuccess)
       return cudaGetLastError();
-    e = launch_pdl(commit_copy_kernel, dim3(148 * 4), dim3(kCopyThreads), csmem, st, a);
+    e = launch_pdl(commit_copy_kernel, dim3(sm_count() * kCopyCtasPerSm), dim3(kCopyThreads), csmem,
+                   st, a);
   }
   return e;
 }

@@ -226,6 +226,22 @@ __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Streaming multiprocessors of the current device (148 on a B200), looked up
+// once per process.
+static inline int sm_count() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      v = 0;
+    }
+    sms = v > 0 ? v : 148;
+  }
+  return sms;
+}
+
 template <typename Kern, typename... Args>
 static cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                              Args... args) {

@@ -448,17 +448,6 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
 // ----------------------------------------------------------------------------
 // Launchers
 // ----------------------------------------------------------------------------
-static int rs_grid() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
-}
-
 template <typename T, typename Rows>
 static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, int32_t* status,
                              cudaStream_t st) {
@@ -478,7 +467,7 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
   for (int r0 = 0; r0 < nrows; r0 += kMaxListRows) {
     const int n = nrows - r0 < kMaxListRows ? nrows - r0 : kMaxListRows;
     const long long items = (long long)n * ntiles;
-    long long grid = rs_grid();
+    long long grid = sm_count();
     const long long need = (items + kRsWarps - 1) / kRsWarps;
     if (grid > need) grid = need;
     if (grid < 1) grid = 1;
