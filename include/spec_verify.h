@@ -16,6 +16,9 @@
  *         2603.03251, Technische Zusammenfassung section 2 item 1 (an outcome
  *         is the accepted count plus a bonus token) and section 3.B (residual
  *         distribution proportional to the target-minus-draft difference).
+ *   [SV]  "Optimierung der Inferenzgeschwindigkeit von Sprachmodellen durch
+ *         spekulative Dekodierung" (mind-verse.de), SVIP paragraphs: the
+ *         entropy of the draft-token distribution as the draft-length signal.
  * The pages print no formulas. The rules implemented are the standard
  * speculative-sampling rules they appeal to: with p = softmax(l_target / T)
  * and q = softmax(l_draft / T), draft x_j is accepted iff u_j * q_j(x_j) <
@@ -29,7 +32,8 @@
  * Randomness: Philox4x32-10 (Salmon et al., SC'11), key = (seed & 0xffffffff,
  * seed >> 32), counter = (seq_id[b], round, position, stage); lane 0 is the
  * accept uniform, lane 1 the draw uniform; u = (2*(x >> 9) + 1) * 2^-24.
- * Stage 1 = chain verification and the first stage; stage 2 = second stage.
+ * Stage 0 = draft step; stage 1 = chain verification and the first stage;
+ * stage 2 = second stage.
  *
  * Conventions for every call
  *   - Pointers are DEVICE memory owned by the caller unless a comment says
@@ -226,6 +230,39 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
                       void* kv_pool, int layers, int kv_heads, int head_dim,
                       const void* hid_stage, void* hid_out, int32_t* hid_off,
                       int hidden, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Draft step ([HS] Kernmechanismus: the shallow exit L_d drafts the tokens the
+ * deeper exits check; [SV] the entropy of the drafting distribution). The
+ * pages print no interface; this is the step that produces the draft_tok of
+ * the verification calls, one slot per sequence.
+ *
+ * logits : drafting-exit rows [B, V]; row b starts at element b * ld.
+ * dtype  : SPEC_F32 or SPEC_BF16.
+ * temperature : float [B]: 0 (greedy: argmax, smallest id on ties) or within
+ *               [1e-6, 1e6]; anything else marks the row invalid.
+ * seed, seq_id (int32 [B]), round, pos (int32 [B]) : Philox counter
+ *               (seq_id[b], round, pos[b], 0); its lane 1 drives the draw,
+ *               pos[b] being the slot the drafted token will occupy.
+ * out_tok     : out int32 [B]: the smallest v with sum_{t<=v} q_t > u * sum_t
+ *               q_t, q = softmax(l / T) (the argmax for T == 0); -1 for an
+ *               invalid row.
+ * out_logq    : optional out double [B] (NULL to skip): ln q(out_tok); 0 for
+ *               greedy rows, NaN for invalid ones.
+ * out_entropy : optional out double [B] (NULL to skip): -sum_v q_v ln q_v in
+ *               nats; 0 for greedy rows, NaN for invalid ones.
+ * dev_status  : SPEC_EDEVICE for an invalid temperature or a row without a
+ *               finite maximum.
+ * ws, ws_bytes: spec_draft_workspace_bytes(B, V, dtype) bytes, 256-byte
+ *               aligned. No initial contents are needed.
+ * ------------------------------------------------------------------------- */
+size_t spec_draft_workspace_bytes(int B, int V, int dtype);
+int spec_draft_sample(const void* logits, int64_t ld, int dtype, int B, int V,
+                      const float* temperature, uint64_t seed,
+                      const int32_t* seq_id, uint32_t round, const int32_t* pos,
+                      int32_t* out_tok, double* out_logq, double* out_entropy,
+                      int32_t* dev_status, void* ws, size_t ws_bytes,
+                      void* stream);
 
 /* ---------------------------------------------------------------------------
  * Chain verification without a caller workspace. The paper has no

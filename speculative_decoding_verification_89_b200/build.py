@@ -13,8 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libspecverify.so")
-SOURCES = ["row_stats.cu", "decide.cu", "commit.cu", "capi.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "kernels.cuh"]
+SOURCES = ["row_stats.cu", "decide.cu", "draft.cu", "commit.cu", "capi.cu", "noalloc.cu"]
+HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh"]
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",

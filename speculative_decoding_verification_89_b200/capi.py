@@ -46,6 +46,9 @@ _SIGS = {
     "spec_last_cuda_error": (ctypes.c_char_p, []),
     "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
                                        _u32, _p, _p, _p, _p, _p]),
+    "spec_draft_workspace_bytes": (_sz, [_i, _i, _i]),
+    "spec_draft_sample": (_i, [_p, _i64, _i, _i, _i, _p, _u64, _p, _u32, _p, _p, _p, _p, _p,
+                               _p, _sz, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -211,3 +214,30 @@ def spec_philox_uniforms(seed, ctr, out, stream=None):
     """ctr: uint32-valued int32 tensor [n, 4] on the device; out: float [n, 2]."""
     rc = _lib.spec_philox_uniforms(seed, _ptr(ctr), ctr.shape[0], _ptr(out), _stream(stream))
     _check("spec_philox_uniforms", rc)
+
+
+def spec_draft_workspace_bytes(B, V, dtype):
+    code = dtype if isinstance(dtype, int) else (SPEC_BF16 if dtype == torch.bfloat16 else SPEC_F32)
+    return int(_lib.spec_draft_workspace_bytes(B, V, code))
+
+
+def draft_workspace(B, V, dtype, device="cuda"):
+    """A workspace tensor of the size a draft step needs."""
+    n = spec_draft_workspace_bytes(B, V, dtype)
+    if n == 0:
+        raise ValueError("invalid sizes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def spec_draft_sample(logits, temperature, seed, seq_id, rnd, pos, out_tok, dev_status, ws,
+                      logq=None, entropy=None, stream=None):
+    """logits [B, V] (contiguous rows, evenly spaced); out_tok int32 [B];
+    optional logq / entropy float64 [B]."""
+    if logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits must be [B, V] with contiguous rows")
+    B, V = logits.shape
+    rc = _lib.spec_draft_sample(_ptr(logits), logits.stride(0), _dtype_code(logits), B, V,
+                                _ptr(temperature), seed, _ptr(seq_id), rnd, _ptr(pos),
+                                _ptr(out_tok), _ptr(logq), _ptr(entropy), _ptr(dev_status),
+                                _ptr(ws), ws.numel(), _stream(stream))
+    _check("spec_draft_sample", rc)

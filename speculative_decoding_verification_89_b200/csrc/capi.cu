@@ -41,6 +41,21 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   return true;
 }
 
+// Draft-step workspace: run partials and first moments of the B rows.
+struct DraftLayout {
+  size_t part, mom, total;
+};
+bool draft_layout(int B, int V, int dtype, DraftLayout* L) {
+  if (B < 0 || V < 1 || V > SPEC_MAX_V) return false;
+  if (dtype != SPEC_F32 && dtype != SPEC_BF16) return false;
+  const long long n = (long long)B * stat_tiles(V, dtype);
+  if (n >= (1LL << 31)) return false;
+  L->part = 0;
+  L->mom = align_up((size_t)n * sizeof(Partial));
+  L->total = L->mom + align_up((size_t)n * sizeof(double));
+  return true;
+}
+
 bool rows_ok(const void* p, int64_t ld, int V, int dtype) {
   if (!p || !aligned(p, 16)) return false;
   if (ld < V) return false;
@@ -77,6 +92,7 @@ ChainCheck check_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t
 RsBuffers rs_buffers(void* ws, const Layout& L) {
   RsBuffers b;
   b.part = reinterpret_cast<Partial*>((char*)ws + L.part);
+  b.mom = nullptr;
   return b;
 }
 
@@ -316,6 +332,30 @@ int spec_commit_paged(int B, int block_size, int max_blocks, int32_t* block_tabl
   a.hid_off = hid_off;
   a.status = dev_status;
   return cuda_status(launch_commit(a, (cudaStream_t)stream));
+}
+
+size_t spec_draft_workspace_bytes(int B, int V, int dtype) {
+  DraftLayout L;
+  if (!draft_layout(B, V, dtype, &L)) return 0;
+  return L.total;
+}
+
+int spec_draft_sample(const void* logits, int64_t ld, int dtype, int B, int V,
+                      const float* temperature, uint64_t seed, const int32_t* seq_id,
+                      uint32_t round, const int32_t* pos, int32_t* out_tok, double* out_logq,
+                      double* out_entropy, int32_t* dev_status, void* ws, size_t ws_bytes,
+                      void* stream) {
+  DraftLayout L;
+  if (!draft_layout(B, V, dtype, &L)) return SPEC_EINVAL;
+  if (B == 0) return SPEC_OK;
+  if (!rows_ok(logits, ld, V, dtype) || !temperature || !seq_id || !pos || !out_tok)
+    return SPEC_EINVAL;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < L.total) return SPEC_EWORKSPACE;
+  return cuda_status(launch_draft_step(
+      dtype, (const unsigned char*)logits, ld * elem_size(dtype), B, V, temperature, seed, seq_id,
+      round, pos, reinterpret_cast<Partial*>((char*)ws + L.part),
+      reinterpret_cast<double*>((char*)ws + L.mom), out_tok, out_logq, out_entropy, dev_status,
+      (cudaStream_t)stream));
 }
 
 const char* spec_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }

@@ -28,6 +28,7 @@ __device__ __forceinline__ RowRef make_row(const unsigned char* ptr, float T, bo
 // Chain verification rows, grouped by sequence: for sequence b, rows
 // b*(2K+1) + j are target row j (j <= K) and then draft row j - K - 1.
 struct ChainRows {
+  static constexpr bool kEntropy = false;
   const unsigned char* tgt;
   const unsigned char* drf;
   long long ld_tgt, ld_drf;  // row strides in bytes
@@ -49,6 +50,7 @@ struct ChainRows {
 // Stage one of the two-stage check: per sequence, L_i rows at slots
 // w .. w+K, then L_d rows at slots w .. w+K-1 (w = window length).
 struct Hier1Rows {
+  static constexpr bool kEntropy = false;
   const unsigned char* lg_i;
   const unsigned char* lg_d;
   long long ld;  // bytes
@@ -75,6 +77,7 @@ struct Hier1Rows {
 // Stage two: L_f rows at slots 0 .. W of sequences whose window holds
 // W >= Ni tokens after stage one (rows b*S + s).
 struct Hier2Rows {
+  static constexpr bool kEntropy = false;
   const unsigned char* lg_f;
   long long ld;
   const float* temperature;
@@ -91,9 +94,23 @@ struct Hier2Rows {
   }
 };
 
+// Draft step: row b of the drafting exit's logits, one row per sequence; the
+// row statistics also gather the first moment the entropy needs.
+struct DraftRows {
+  static constexpr bool kEntropy = true;
+  const unsigned char* lg;
+  long long ld;  // bytes
+  const float* temperature;
+  __device__ __forceinline__ bool late(int) const { return false; }
+  __device__ __forceinline__ RowRef get(int r) const {
+    return make_row(lg + (long long)r * ld, __ldg(temperature + r), true);
+  }
+};
+
 // Workspace pieces of the row-statistics step.
 struct RsBuffers {
   Partial* part;    // [rows, tiles]
+  double* mom;      // [rows, tiles] first moments (Rows::kEntropy only)
 };
 
 // Combine a row's tile partials (warp-cooperative; result valid in lane 0).
@@ -232,6 +249,14 @@ struct CommitArgs {
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
+
+// Draft step over B rows of the drafting exit: row statistics with the first
+// moments, then one cluster per sequence for the entropy and the draw.
+cudaError_t launch_draft_step(int dtype, const unsigned char* lg, long long ld_bytes, int B, int V,
+                              const float* temperature, uint64_t seed, const int32_t* seq_id,
+                              uint32_t round, const int32_t* pos, Partial* part, double* mom,
+                              int32_t* out_tok, double* out_logq, double* out_entropy,
+                              int32_t* status, cudaStream_t st);
 
 
 

@@ -19,6 +19,8 @@
 // costs no warp shuffle and no division; the lanes are combined once per row
 // run into one Partial at the run's first tile (its other tiles get empty
 // partials).
+#include <cfloat>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -97,6 +99,37 @@ __device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, fl
       ex2x2(expo2(make_float2(__uint_as_float(w.z), __uint_as_float(w.w)), chi, clo, nM));
   return __fadd2_rn(e0, e1);
 }
+// x - a, held at -FLT_MAX for x = -inf (a masked or padded entry), whose term
+// 2^(x*c - M) = 0 must then contribute 0, not 0 * -inf.
+__device__ __forceinline__ float dev1(float x, float a) { return fmaxf(x - a, -FLT_MAX); }
+__device__ __forceinline__ float2 dev2(float2 x, float2 nA) {
+  const float2 d = __fadd2_rn(x, nA);
+  return make_float2(fmaxf(d.x, -FLT_MAX), fmaxf(d.y, -FLT_MAX));
+}
+
+// Same, also returning the pairwise sums of 2^(x*c - M) * (x - a) (nA = -a),
+// the first moment the entropy of the row's distribution needs.
+__device__ __forceinline__ float2 vec_expsum_ent(uint4 w, float2 chi, float2 clo, float2 nM,
+                                                 float2 nA, float2* mom, __nv_bfloat16*) {
+  const float2 x0 = make_float2(bf_lo(w.x), bf_hi(w.x)), x1 = make_float2(bf_lo(w.y), bf_hi(w.y));
+  const float2 x2 = make_float2(bf_lo(w.z), bf_hi(w.z)), x3 = make_float2(bf_lo(w.w), bf_hi(w.w));
+  const float2 e0 = ex2x2(expo2(x0, chi, clo, nM)), e1 = ex2x2(expo2(x1, chi, clo, nM));
+  const float2 e2 = ex2x2(expo2(x2, chi, clo, nM)), e3 = ex2x2(expo2(x3, chi, clo, nM));
+  float2 t = __fmul2_rn(e0, dev2(x0, nA));
+  t = __ffma2_rn(e1, dev2(x1, nA), t);
+  t = __ffma2_rn(e2, dev2(x2, nA), t);
+  *mom = __ffma2_rn(e3, dev2(x3, nA), t);
+  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
+}
+__device__ __forceinline__ float2 vec_expsum_ent(uint4 w, float2 chi, float2 clo, float2 nM,
+                                                 float2 nA, float2* mom, float*) {
+  const float2 x0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+  const float2 x1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+  const float2 e0 = ex2x2(expo2(x0, chi, clo, nM)), e1 = ex2x2(expo2(x1, chi, clo, nM));
+  *mom = __ffma2_rn(e1, dev2(x1, nA), __fmul2_rn(e0, dev2(x0, nA)));
+  return __fadd2_rn(e0, e1);
+}
+
 // Scalar form of one term (tail elements).
 __device__ __forceinline__ float term(float x, float chi, float clo, float nM) {
   return ex2(fmaf(x, clo, fmaf(x, chi, nM)));
@@ -147,7 +180,7 @@ template <> __device__ __forceinline__ uint4 neg_inf_vec<float>() {
 template <typename T, typename Rows>
 __global__ void __launch_bounds__(kRsWarps * 32, 1)
     row_stats_kernel(Rows rows, int row_base, int nrows, int V, Partial* __restrict__ part,
-                     int32_t* status) {
+                     double* __restrict__ mom, int32_t* status) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_wsum[kRsWarps];
   constexpr int kVec = VecOf<T>::n;
@@ -280,6 +313,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   float anchor = -INFINITY;  // the logit that set the shift
   float Msh = 0.0f;          // shift fl(anchor * chi)
   double acc = 0.0;          // sum of 2^(l*c - Msh) over the lane's elements
+  double acc1 = 0.0;         // sum of 2^(l*c - Msh) * (l - anchor) (Rows::kEntropy)
   int gidx = 0x7fffffff;     // greedy rows: first index of mrun
 
   for (; cc.left > 0; s = (s + 1 == kRsStages) ? 0 : s + 1) {
@@ -307,6 +341,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       mrun = anchor = -INFINITY;
       Msh = 0.0f;
       acc = 0.0;
+      acc1 = 0.0;
       gidx = 0x7fffffff;
     }
 
@@ -371,34 +406,73 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
         // exponents could exceed 2^kShiftSlack.
         if (!(anchor > -INFINITY) || fmaf(tm, chi, -Msh) > kShiftSlack) {
           const float Mn = __fmul_rn(tm, chi);
-          if (acc != 0.0) acc *= exp2((double)Msh - (double)Mn);
+          if (acc != 0.0) {
+            const double f = exp2((double)Msh - (double)Mn);
+            if constexpr (Rows::kEntropy) acc1 = (acc1 + ((double)anchor - (double)tm) * acc) * f;
+            acc *= f;
+          }
           anchor = tm;
           Msh = Mn;
         }
       }
       const bool has = anchor > -INFINITY;
-      float a = 0.0f;
+      float a = 0.0f, a1s = 0.0f;
       if (__all_sync(0xffffffffu, !has || fabsf(Msh) < kFarShift)) {
         if (has) {
           const float2 chi2 = make_float2(chi, chi), clo2 = make_float2(clo, clo);
           const float2 nM2 = make_float2(-Msh, -Msh);
           float2 a0 = make_float2(0.0f, 0.0f), a1 = make_float2(0.0f, 0.0f);
+          if constexpr (Rows::kEntropy) {
+            const float2 nA2 = make_float2(-anchor, -anchor);
+            float2 t0 = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int i = 0; i < kVpl; i += 2) {
-            a0 = __fadd2_rn(a0, vec_expsum(x[i], chi2, clo2, nM2, (T*)nullptr));
-            if (i + 1 < kVpl) a1 = __fadd2_rn(a1, vec_expsum(x[i + 1], chi2, clo2, nM2, (T*)nullptr));
+            for (int i = 0; i < kVpl; ++i) {
+              float2 t;
+              a0 = __fadd2_rn(a0, vec_expsum_ent(x[i], chi2, clo2, nM2, nA2, &t, (T*)nullptr));
+              t0 = __fadd2_rn(t0, t);
+            }
+            a1s = t0.x + t0.y;
+          } else {
+#pragma unroll
+            for (int i = 0; i < kVpl; i += 2) {
+              a0 = __fadd2_rn(a0, vec_expsum(x[i], chi2, clo2, nM2, (T*)nullptr));
+              if (i + 1 < kVpl)
+                a1 = __fadd2_rn(a1, vec_expsum(x[i + 1], chi2, clo2, nM2, (T*)nullptr));
+            }
           }
           const float2 a2 = __fadd2_rn(a0, a1);
           a = a2.x + a2.y;
-          if (lane < ntail) a += term(tailx, chi, clo, -Msh);
+          if (lane < ntail) {
+            const float e = term(tailx, chi, clo, -Msh);
+            a += e;
+            if constexpr (Rows::kEntropy) a1s += e * dev1(tailx, anchor);
+          }
         }
       } else if (has) {
         const float rr = fmaf(anchor, chi, -Msh) + anchor * clo;
+        if constexpr (Rows::kEntropy) {
 #pragma unroll
-        for (int i = 0; i < kVpl; ++i) a += vec_expsum_far<T>(x[i], anchor, chi, clo, rr);
-        if (lane < ntail) a += term_far(tailx, anchor, chi, clo, rr);
+          for (int i = 0; i < kVpl; ++i) {
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) {
+              const float xv = vec_elem(x[i], e, (T*)nullptr);
+              const float te = term_far(xv, anchor, chi, clo, rr);
+              a += te;
+              a1s += te * dev1(xv, anchor);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kVpl; ++i) a += vec_expsum_far<T>(x[i], anchor, chi, clo, rr);
+        }
+        if (lane < ntail) {
+          const float te = term_far(tailx, anchor, chi, clo, rr);
+          a += te;
+          if constexpr (Rows::kEntropy) a1s += te * dev1(tailx, anchor);
+        }
       }
       acc += (double)a;
+      if constexpr (Rows::kEntropy) acc1 += (double)a1s;
     }
 
     // End of the row, of a segment or of this warp's items: one Partial for
@@ -419,17 +493,25 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
         float m = mrun;
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        double sl = 0.0;
-        if (m > -INFINITY && m < INFINITY && acc != 0.0)
-          sl = acc * exp2((double)Msh - (double)__fmul_rn(m, chi));
+        double sl = 0.0, tl = 0.0;
+        if (m > -INFINITY && m < INFINITY && acc != 0.0) {
+          const double f = exp2((double)Msh - (double)__fmul_rn(m, chi));
+          sl = acc * f;
+          // moment about the run's maximum m
+          if constexpr (Rows::kEntropy) tl = (acc1 + ((double)anchor - (double)m) * acc) * f;
+        }
         p.m = m;
         p.idx = 0x7fffffff;
         p.s = warp_sum_d(sl);
+        if constexpr (Rows::kEntropy) tl = warp_sum_d(tl);
+        if (Rows::kEntropy && lane == 0) mom[(size_t)row * ntiles + run_t0] = tl;
       }
       Partial* prow = part + (size_t)row * ntiles;
       if (lane == 0) prow[run_t0] = p;
-      for (int t = run_t0 + 1 + lane; t <= t_last; t += 32)
+      for (int t = run_t0 + 1 + lane; t <= t_last; t += 32) {
         prow[t] = Partial{-INFINITY, 0x7fffffff, 0.0};
+        if constexpr (Rows::kEntropy) mom[(size_t)row * ntiles + t] = 0.0;
+      }
     }
   }
 
@@ -449,8 +531,8 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
 // Launchers
 // ----------------------------------------------------------------------------
 template <typename T, typename Rows>
-static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, int32_t* status,
-                             cudaStream_t st) {
+static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, double* mom,
+                             int32_t* status, cudaStream_t st) {
   auto kern = row_stats_kernel<T, Rows>;
   static bool smem_set = false;  // once per instantiation (same on every B200)
   if (!smem_set) {
@@ -472,7 +554,7 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
     if (grid > need) grid = need;
     if (grid < 1) grid = 1;
     const cudaError_t e = launch_pdl(kern, dim3((unsigned)grid), dim3(kRsWarps * 32),
-                                     (size_t)kRsSmemTotal, st, rows, r0, n, V, part, status);
+                                     (size_t)kRsSmemTotal, st, rows, r0, n, V, part, mom, status);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -482,8 +564,8 @@ template <typename Rows>
 cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, const RsBuffers& b,
                              int32_t* status, cudaStream_t st) {
   if (dtype == SPEC_BF16)
-    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, status, st);
-  return launch_rs<float>(rows, nrows, V, b.part, status, st);
+    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, b.mom, status, st);
+  return launch_rs<float>(rows, nrows, V, b.part, b.mom, status, st);
 }
 
 template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int,
@@ -491,6 +573,8 @@ template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int
 template cudaError_t launch_row_stats<Hier1Rows>(int, const Hier1Rows&, int, int,
                                                  const RsBuffers&, int32_t*, cudaStream_t);
 template cudaError_t launch_row_stats<Hier2Rows>(int, const Hier2Rows&, int, int,
+                                                 const RsBuffers&, int32_t*, cudaStream_t);
+template cudaError_t launch_row_stats<DraftRows>(int, const DraftRows&, int, int,
                                                  const RsBuffers&, int32_t*, cudaStream_t);
 
 }  // namespace specv

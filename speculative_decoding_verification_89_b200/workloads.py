@@ -158,6 +158,50 @@ def mixed_temperatures(B, n_greedy, t_max, gen, device):
 
 
 # ----------------------------------------------------------------------------
+# Draft-step problems
+# ----------------------------------------------------------------------------
+
+
+@dataclass
+class DraftProblem:
+    logits: torch.Tensor       # [B, V] drafting-exit rows
+    temperature: torch.Tensor  # float32 [B]
+    seq_id: torch.Tensor       # int32 [B]
+    pos: torch.Tensor          # int32 [B] slot of the drafted token
+    seed: int                  # Philox key
+    rnd: int                   # Philox round field
+
+
+def draft_problem(B, V, dtype=torch.bfloat16, *, seed=0, rnd=0, device="cpu", std=2.0,
+                  zipf_s=0.0, mask_frac=0.0, temperature=1.0, philox_seed=None,
+                  seq_id_base=0) -> DraftProblem:
+    """l_d ~ N(0, std^2) (+ Zipf log-prior), a random mask_frac of the entries
+    set to -inf; slots pos ~ U{0..15}."""
+    gen = generator(seed * 1_000_003 + rnd + 17, device)
+    lg = gaussian((B, V), std, gen, device)
+    if zipf_s:
+        lg += zipf_prior(V, zipf_s, device)
+    if mask_frac:
+        m = torch.rand((B, V), generator=gen, device=device) < mask_frac
+        lg = lg.masked_fill(m, float("-inf"))
+    lg = lg.to(dtype)
+    if isinstance(temperature, torch.Tensor):
+        T = temperature.to(device=device, dtype=torch.float32)
+    else:
+        T = torch.full((B,), float(temperature), dtype=torch.float32, device=device)
+    seq_id = torch.arange(seq_id_base, seq_id_base + B, dtype=torch.int32, device=device)
+    pos = torch.randint(0, 16, (B,), generator=gen, device=device, dtype=torch.int32)
+    return DraftProblem(lg, T, seq_id, pos, seed if philox_seed is None else philox_seed, rnd)
+
+
+def draft_batch(device="cpu", rnd=0, B=64, V=128256, seed=5):
+    """B=64, V=128256 bf16 drafting rows l_d ~ N(0, 2^2) - 1.1 ln(id + 1);
+    T = 1; Philox seed 5."""
+    return draft_problem(B, V, torch.bfloat16, seed=seed, rnd=rnd, device=device, zipf_s=1.1,
+                         temperature=1.0, philox_seed=5)
+
+
+# ----------------------------------------------------------------------------
 # Paged KV state
 # ----------------------------------------------------------------------------
 

@@ -108,3 +108,26 @@ def test_commit_host_argument_errors(lib):
     assert f(*bad) == -1                  # hidden rows without offsets
     bad = list(args); bad[3] = None
     assert f(*bad) == -1                  # no tables
+
+
+def test_draft_workspace_and_host_errors(lib):
+    P = ctypes.c_void_p
+    g = lib.spec_draft_workspace_bytes
+    g.restype = ctypes.c_size_t
+    n = g(64, 128256, 1)
+    assert n % 256 == 0 and n >= 64 * 42 * (16 + 8)
+    assert g(1, 0, 1) == 0 and g(1, 10, 9) == 0 and g(-1, 10, 0) == 0
+    f = lib.spec_draft_sample
+    f.restype = ctypes.c_int
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P,
+                  ctypes.c_uint64, P, ctypes.c_uint32, P, P, P, P, P, P, ctypes.c_size_t, P]
+    fake, odd = P(0x10000), P(0x10008)
+    base = [fake, 1024, 1, 4, 1024, fake, 0, fake, 0, fake, fake, None, None, fake, fake,
+            1 << 30, None]
+    assert f(*base[:3], 0, *base[4:]) == 0          # B = 0: nothing to do
+    for i, v, want in [(0, None, -1), (0, odd, -1), (1, 1000, -1), (2, 4, -1), (5, None, -1),
+                       (7, None, -1), (9, None, -1), (10, None, -1), (14, None, -3),
+                       (15, 64, -3)]:
+        bad = list(base)
+        bad[i] = v
+        assert f(*bad) == want, (i, v)
