@@ -344,6 +344,7 @@ def run_ours(args, dist):
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, prob, state, bufs, base, dev, dist)
     result["draft_step"] = run_draft_step(args, dev, dist, peak)
+    result["outcome_law"] = run_outcome_law(args, prob, dev, dist, peak)
     if dist.world == 1 and dist.rank == 0:
         result["parity_spot_check"] = spot_check(prob, hist[0].cpu().numpy())
         if not args.no_cpu_baseline:
@@ -391,6 +392,49 @@ def run_draft_step(args, dev, dist, peak):
             "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": nbytes / (ms * 1e-3) / 1e9 / peak,
             "gpu_launches_per_call": 2}
+
+
+def run_outcome_law(args, prob, dev, dist, peak):
+    """Outcome prediction on the benchmark's verification inputs (B=64, K=8,
+    V=128256 bf16, drafts fixed): the acceptance-length law and the 32 most
+    likely (length, token) outcomes per sequence. Algorithmic bytes: each
+    logit once (the per-position pass re-reads the row pairs)."""
+    from speculative_decoding_verification_89_b200 import capi
+    n_top = 32
+    ws = capi.outcome_workspace(B, K, V, torch.bfloat16, n_top, device=dev)
+    f64 = dict(dtype=torch.float64, device=dev)
+    p_len = torch.empty((B, K + 1), **f64)
+    tl = torch.empty((B, n_top), dtype=torch.int32, device=dev)
+    tt = torch.empty((B, n_top), dtype=torch.int32, device=dev)
+    tp = torch.empty((B, n_top), **f64)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        capi.spec_outcome_law(prob.tgt, prob.drf, prob.draft_tok, prob.temperature, n_top, p_len,
+                              status, ws, top_len=tl, top_tok=tt, top_prob=tp)
+
+    n = max(10, min(args.steps // 10, 500))
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.reduce(e0.elapsed_time(e1), "max") / n
+    if int(status.item()) != 0:
+        raise RuntimeError(f"outcome law: device status {int(status.item())}")
+    return {"workload": "outcome law: B=64, K=8, V=128256 bf16 (the verification inputs), "
+                        "32 outcomes per sequence",
+            "us_per_call": ms * 1e3, "calls": n,
+            "sequences_per_s": B * dist.world / (ms * 1e-3),
+            "algorithmic_bytes_per_call": LOGIT_BYTES,
+            "achieved_gbs": LOGIT_BYTES / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": LOGIT_BYTES / (ms * 1e-3) / 1e9 / peak,
+            "gpu_launches_per_call": 3}
 
 
 def run_e2e(args, prob, state, bufs, base, dev, dist):

@@ -82,6 +82,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 
 /* Limits checked on the host. */
 #define SPEC_MAX_K 256           /* drafts per sequence per call      */
+#define SPEC_MAX_TOP 32          /* outcomes kept per sequence        */
 #define SPEC_MAX_V (1 << 21)     /* vocabulary size                   */
 #define SPEC_MAX_COMMIT_B 16384  /* sequences per paged commit        */
 
@@ -263,6 +264,42 @@ int spec_draft_sample(const void* logits, int64_t ld, int dtype, int B, int V,
                       int32_t* out_tok, double* out_logq, double* out_entropy,
                       int32_t* dev_status, void* ws, size_t ws_bytes,
                       void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Outcome law of a chain check with the drafts fixed ([SSD] Technische
+ * Zusammenfassung 2: predict the running verification's outcome, accepted
+ * count and bonus token, and prepare continuations for the likely ones; 3.A:
+ * a budget spent mostly on short acceptance lengths; 3.B: the token after a
+ * rejection follows the residual). The pages print no interface.
+ *
+ * Same logits, dtype, sizes, drafts and temperatures as spec_verify_chain.
+ * With beta_j = min(1, p_j(x_j) / q_j(x_j)) (at T == 0: 1 iff x_j is the
+ * argmax of target row j):
+ * p_len   : out double [B, K+1]: P(a = k) = beta_0..beta_{k-1} (1 - beta_k)
+ *           for k < K, beta_0..beta_{K-1} for k = K.
+ * beta    : optional out double [B, K] (NULL to skip).
+ * mass    : optional out double [B, K+1]: sum_v max(0, p_k - q_k) for k < K,
+ *           1 for k = K (and for greedy sequences).
+ * n_top   : outcomes kept per sequence, 0 .. SPEC_MAX_TOP.
+ * top_len, top_tok, top_prob : out [B, n_top] (int32, int32, double): the
+ *           n_top most likely outcomes (k, v) by P(a = k) r_k(v), most likely
+ *           first, equal probabilities in (k, v) order, where r_k =
+ *           normalize(max(0, p_k - q_k)) for k < K, r_K = p_K (greedy: the
+ *           point mass on the argmax). Entries past the last outcome of
+ *           nonzero probability hold -1, -1, 0.
+ * dev_status : SPEC_EDEVICE for an invalid temperature, a draft id outside
+ *           [0, V) or a row without a finite maximum (outputs NaN / -1).
+ * ws, ws_bytes : spec_outcome_workspace_bytes(B, K, V, dtype, n_top) bytes,
+ *           256-byte aligned. No initial contents are needed.
+ * ------------------------------------------------------------------------- */
+size_t spec_outcome_workspace_bytes(int B, int K, int V, int dtype, int n_top);
+int spec_outcome_law(const void* tgt, int64_t ld_tgt, const void* drf,
+                     int64_t ld_drf, int dtype, int B, int K, int V,
+                     const int32_t* draft_tok, const float* temperature,
+                     int n_top, double* p_len, double* beta, double* mass,
+                     int32_t* top_len, int32_t* top_tok, double* top_prob,
+                     int32_t* dev_status, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /* ---------------------------------------------------------------------------
  * Chain verification without a caller workspace. The paper has no

@@ -13,7 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libspecverify.so")
-SOURCES = ["row_stats.cu", "decide.cu", "draft.cu", "commit.cu", "capi.cu", "noalloc.cu"]
+SOURCES = ["row_stats.cu", "decide.cu", "draft.cu", "outcome.cu", "commit.cu", "capi.cu",
+           "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh"]
 
 NVCC_FLAGS = [

@@ -47,6 +47,9 @@ _SIGS = {
     "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
                                        _u32, _p, _p, _p, _p, _p]),
     "spec_draft_workspace_bytes": (_sz, [_i, _i, _i]),
+    "spec_outcome_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "spec_outcome_law": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p,
+                              _p, _p, _p, _p, _sz, _p]),
     "spec_draft_sample": (_i, [_p, _i64, _i, _i, _i, _p, _u64, _p, _u32, _p, _p, _p, _p, _p,
                                _p, _sz, _p]),
 }
@@ -241,3 +244,29 @@ def spec_draft_sample(logits, temperature, seed, seq_id, rnd, pos, out_tok, dev_
                                 _ptr(out_tok), _ptr(logq), _ptr(entropy), _ptr(dev_status),
                                 _ptr(ws), ws.numel(), _stream(stream))
     _check("spec_draft_sample", rc)
+
+
+def spec_outcome_workspace_bytes(B, K, V, dtype, n_top):
+    code = dtype if isinstance(dtype, int) else (SPEC_BF16 if dtype == torch.bfloat16 else SPEC_F32)
+    return int(_lib.spec_outcome_workspace_bytes(B, K, V, code, n_top))
+
+
+def outcome_workspace(B, K, V, dtype, n_top, device="cuda"):
+    n = spec_outcome_workspace_bytes(B, K, V, dtype, n_top)
+    if n == 0:
+        raise ValueError("invalid sizes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def spec_outcome_law(tgt, drf, draft_tok, temperature, n_top, p_len, dev_status, ws, beta=None,
+                     mass=None, top_len=None, top_tok=None, top_prob=None, stream=None):
+    """tgt [B, K+1, V], drf [B, K, V] as for spec_verify_chain; p_len float64
+    [B, K+1]; top_* [B, n_top]."""
+    B, Kp1, V = tgt.shape
+    K = Kp1 - 1
+    rc = _lib.spec_outcome_law(
+        _ptr(tgt), _rows(tgt, Kp1), _ptr(drf) if K > 0 else None,
+        _rows(drf, K) if K > 0 else 0, _dtype_code(tgt), B, K, V, _ptr(draft_tok),
+        _ptr(temperature), n_top, _ptr(p_len), _ptr(beta), _ptr(mass), _ptr(top_len),
+        _ptr(top_tok), _ptr(top_prob), _ptr(dev_status), _ptr(ws), ws.numel(), _stream(stream))
+    _check("spec_outcome_law", rc)

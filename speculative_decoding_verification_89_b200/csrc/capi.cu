@@ -56,6 +56,23 @@ bool draft_layout(int B, int V, int dtype, DraftLayout* L) {
   return true;
 }
 
+// Outcome-law workspace: the chain layout, then the residual masses and the
+// per-(sequence, position) best weights and tokens.
+struct OutcomeLayout {
+  Layout L;
+  size_t zk, cw, cv, total;
+};
+bool outcome_layout(int B, int K, int V, int dtype, int n_top, OutcomeLayout* O) {
+  if (n_top < 0 || n_top > SPEC_MAX_TOP) return false;
+  if (!layout(B, K, V, dtype, 0, &O->L)) return false;
+  const size_t slots = (size_t)B * (K + 1);
+  O->zk = O->L.total;
+  O->cw = O->zk + align_up(slots * sizeof(double));
+  O->cv = O->cw + align_up(slots * (size_t)n_top * sizeof(float));
+  O->total = O->cv + align_up(slots * (size_t)n_top * sizeof(int));
+  return true;
+}
+
 bool rows_ok(const void* p, int64_t ld, int V, int dtype) {
   if (!p || !aligned(p, 16)) return false;
   if (ld < V) return false;
@@ -356,6 +373,63 @@ int spec_draft_sample(const void* logits, int64_t ld, int dtype, int B, int V,
       round, pos, reinterpret_cast<Partial*>((char*)ws + L.part),
       reinterpret_cast<double*>((char*)ws + L.mom), out_tok, out_logq, out_entropy, dev_status,
       (cudaStream_t)stream));
+}
+
+size_t spec_outcome_workspace_bytes(int B, int K, int V, int dtype, int n_top) {
+  OutcomeLayout O;
+  if (!outcome_layout(B, K, V, dtype, n_top, &O)) return 0;
+  return O.total;
+}
+
+int spec_outcome_law(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                     int B, int K, int V, const int32_t* draft_tok, const float* temperature,
+                     int n_top, double* p_len, double* beta, double* mass, int32_t* top_len,
+                     int32_t* top_tok, double* top_prob, int32_t* dev_status, void* ws,
+                     size_t ws_bytes, void* stream) {
+  OutcomeLayout O;
+  if (!outcome_layout(B, K, V, dtype, n_top, &O)) return SPEC_EINVAL;
+  if (B == 0) return SPEC_OK;
+  if (!rows_ok(tgt, ld_tgt, V, dtype) || !temperature || !p_len) return SPEC_EINVAL;
+  if (K > 0 && (!rows_ok(drf, ld_drf, V, dtype) || !draft_tok)) return SPEC_EINVAL;
+  if (n_top > 0 && (!top_len || !top_tok || !top_prob)) return SPEC_EINVAL;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < O.total) return SPEC_EWORKSPACE;
+  const int es = elem_size(dtype);
+  ChainRows rows;
+  rows.tgt = (const unsigned char*)tgt;
+  rows.drf = (const unsigned char*)drf;
+  rows.ld_tgt = ld_tgt * es;
+  rows.ld_drf = ld_drf * es;
+  rows.temperature = temperature;
+  rows.K = K;
+  rows.late_pos = 0;  // every target row pair is read again
+  const cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, O.L),
+                                   dev_status, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  OutcomeArgs a;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.n_top = n_top;
+  a.ntiles = stat_tiles(V, dtype);
+  a.tgt = rows.tgt;
+  a.drf = rows.drf;
+  a.ld_tgt = rows.ld_tgt;
+  a.ld_drf = rows.ld_drf;
+  a.draft_tok = draft_tok;
+  a.temperature = temperature;
+  a.part = reinterpret_cast<const Partial*>((char*)ws + O.L.part);
+  a.zk = reinterpret_cast<double*>((char*)ws + O.zk);
+  a.cw = reinterpret_cast<float*>((char*)ws + O.cw);
+  a.cv = reinterpret_cast<int*>((char*)ws + O.cv);
+  a.p_len = p_len;
+  a.beta = beta;
+  a.mass = mass;
+  a.top_len = top_len;
+  a.top_tok = top_tok;
+  a.top_prob = top_prob;
+  a.status = dev_status;
+  return cuda_status(launch_outcome(dtype, a, st));
 }
 
 const char* spec_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }

@@ -250,6 +250,28 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
 
+// Outcome law of a chain check (drafts fixed): see outcome.cu.
+struct OutcomeArgs {
+  int B, K, V, n_top, ntiles;
+  const unsigned char* tgt;
+  const unsigned char* drf;
+  long long ld_tgt, ld_drf;  // bytes
+  const int32_t* draft_tok;
+  const float* temperature;
+  const Partial* part;  // [B * (2K+1), ntiles]
+  double* zk;           // [B, K+1] residual masses
+  float* cw;            // [B, K+1, n_top] best weights
+  int* cv;              // [B, K+1, n_top] their tokens
+  double* p_len;        // out [B, K+1]
+  double* beta;         // out [B, K] or null
+  double* mass;         // out [B, K+1] or null
+  int32_t* top_len;     // out [B, n_top]
+  int32_t* top_tok;     // out [B, n_top]
+  double* top_prob;     // out [B, n_top]
+  int32_t* status;
+};
+cudaError_t launch_outcome(int dtype, const OutcomeArgs& a, cudaStream_t st);
+
 // Draft step over B rows of the drafting exit: row statistics with the first
 // moments, then one cluster per sequence for the entropy and the draw.
 cudaError_t launch_draft_step(int dtype, const unsigned char* lg, long long ld_bytes, int B, int V,

@@ -24,6 +24,9 @@ def main():
     ap.add_argument("--iters", type=int, default=6)
     ap.add_argument("--commit", action="store_true", help="also run the paged commit")
     ap.add_argument("--no-verify", action="store_true", help="commit only (random accept lengths)")
+    ap.add_argument("--outcome", type=int, default=-1,
+                    help="run the outcome law with this many outcomes instead of verifying")
+    ap.add_argument("--draft", action="store_true", help="run the draft step instead of verifying")
     args = ap.parse_args()
     B, K, V = args.B, 8, W.LLAMA3_V
     dev = torch.device("cuda")
@@ -38,6 +41,8 @@ def main():
         base = state.seq_lens.clone()
         gen = torch.Generator(device=dev)
         gen.manual_seed(0)
+    if args.outcome >= 0 or args.draft:
+        return other(args, B, K, V, dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     times = []
     for i in range(args.iters):
@@ -53,6 +58,43 @@ def main():
                                    kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
                                    hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
                                    hid_off=bufs.hid_off)
+        ev[1].record()
+        torch.cuda.synchronize()
+        times.append(ev[0].elapsed_time(ev[1]) * 1e3)
+    print(f"B={B} status={int(st.item())} us/iter median={sorted(times)[len(times) // 2]:.1f}")
+    if int(st.item()) != 0:
+        raise SystemExit(1)
+
+
+def other(args, B, K, V, dev):
+    """The outcome law (on the verification inputs) or the draft step."""
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    if args.draft:
+        prob = W.draft_batch(device=dev, B=B)
+        ws = capi.draft_workspace(B, V, torch.bfloat16, device=dev)
+        tok = torch.empty(B, dtype=torch.int32, device=dev)
+        ent = torch.empty(B, dtype=torch.float64, device=dev)
+
+        def call(i):
+            capi.spec_draft_sample(prob.logits, prob.temperature, prob.seed, prob.seq_id, i,
+                                   prob.pos, tok, st, ws, entropy=ent)
+    else:
+        prob = W.chain_batch(device=dev, B=B)
+        n = args.outcome
+        ws = capi.outcome_workspace(B, K, V, torch.bfloat16, n, device=dev)
+        p_len = torch.empty((B, K + 1), dtype=torch.float64, device=dev)
+        tl = torch.empty((B, max(n, 1)), dtype=torch.int32, device=dev)
+        tt = torch.empty((B, max(n, 1)), dtype=torch.int32, device=dev)
+        tp = torch.empty((B, max(n, 1)), dtype=torch.float64, device=dev)
+
+        def call(i):
+            capi.spec_outcome_law(prob.tgt, prob.drf, prob.draft_tok, prob.temperature, n, p_len,
+                                  st, ws, top_len=tl, top_tok=tt, top_prob=tp)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    times = []
+    for i in range(args.iters):
+        ev[0].record()
+        call(i)
         ev[1].record()
         torch.cuda.synchronize()
         times.append(ev[0].elapsed_time(ev[1]) * 1e3)
