@@ -131,3 +131,25 @@ def test_draft_workspace_and_host_errors(lib):
         bad = list(base)
         bad[i] = v
         assert f(*bad) == want, (i, v)
+
+
+def test_outcome_workspace_and_host_errors(lib):
+    P = ctypes.c_void_p
+    g = lib.spec_outcome_workspace_bytes
+    g.restype = ctypes.c_size_t
+    assert g(64, 8, 128256, 1, 32) > g(64, 8, 128256, 1, 0) > 0
+    assert g(4, 2, 100, 0, 33) == 0 and g(4, 2, 100, 0, -1) == 0
+    f = lib.spec_outcome_law
+    f.restype = ctypes.c_int
+    I, I64 = ctypes.c_int, ctypes.c_int64
+    f.argtypes = [P, I64, P, I64, I, I, I, I, P, P, I, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    fake = P(0x10000)
+    base = [fake, 1024, fake, 1024, 0, 4, 3, 1024, fake, fake, 8, fake, None, None, fake, fake,
+            fake, fake, fake, 1 << 30, None]
+    assert f(*base[:5], 0, *base[6:]) == 0          # B = 0
+    for i, v, want in [(0, None, -1), (2, None, -1), (8, None, -1), (9, None, -1),
+                       (10, 33, -1), (11, None, -1), (14, None, -1), (18, None, -3),
+                       (19, 64, -3)]:
+        bad = list(base)
+        bad[i] = v
+        assert f(*bad) == want, (i, v)
