@@ -12,7 +12,7 @@ so it rolls the previous round back and grows again: the pool stays bounded
 and every step does the same kind of work.
 
 Prints one JSON line (rank 0). ``--impl reference`` times the fp64 oracle on
-the host cores instead (the reference arm of this build).
+the host cores instead: a plain single-threaded program as the reference arm.
 """
 from __future__ import annotations
 
