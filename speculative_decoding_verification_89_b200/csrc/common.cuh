@@ -215,15 +215,21 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ----------------------------------------------------------------------------
 // Programmatic dependent launch: every kernel of the library is launched with
-// programmatic stream serialization, waits for its stream predecessors before
-// touching memory (griddepcontrol.wait returns once they have completed and
-// their writes are visible) and lets its successor start launching early.
-// ----------------------------------------------------------------------------
+// programmatic stream serialization and starts with pdl_begin(): it waits for
+// its stream predecessors before touching memory (griddepcontrol.wait returns
+// once they have completed and their writes are visible) and at once lets its
+// successor launch, so the successor's CTAs take SMs as this kernel's CTAs
+// leave them and only wait for the completion (its own griddepcontrol.wait
+// orders every memory access).
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_begin() {
+  grid_dependency_wait();
+  grid_dependents_launch();
 }
 
 // Streaming multiprocessors of the current device (148 on a B200), looked up

@@ -176,7 +176,7 @@ struct Outcome {
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecideArgs A) {
-  grid_dependency_wait();
+  pdl_begin();
   cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
@@ -241,7 +241,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
   if (rank != 0) return;
   if (o.bad) {
     fail();
-    grid_dependents_launch();
     return;
   }
   const int a = o.a;
@@ -264,7 +263,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
       if (threadIdx.x == 0) diag[4 * K + 1] = Z;
     }
   }
-  grid_dependents_launch();
 }
 
 // ---------------------------------------------------------------------------
@@ -293,7 +291,7 @@ __device__ __forceinline__ void window_append(const HierDecideArgs& A, int b, in
 // L_d; the a1 accepted drafts and the drawn token join the window.
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecideArgs A) {
-  grid_dependency_wait();
+  pdl_begin();
   cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
@@ -365,7 +363,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
   if (rank != 0) return;
   if (o.bad) {
     fail();
-    grid_dependents_launch();
     return;
   }
   const int a = o.a;
@@ -387,7 +384,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
     A.win_len[b] = w + a + 1;
     A.acc1[b] = a;
   }
-  grid_dependents_launch();
 }
 
 // Stage two: for sequences whose window holds W >= Ni tokens, the window
@@ -395,7 +391,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
 // buffered statistics; commits a2 + 1 tokens and empties the window.
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecideArgs A) {
-  grid_dependency_wait();
+  pdl_begin();
   cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
@@ -454,7 +450,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
       set_status(c.status, SPEC_EDEVICE);
       A.acc2[b] = -1;
     }
-    grid_dependents_launch();
     return;
   }
   const int a = o.a;
@@ -478,7 +473,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
     A.acc2[b] = a;
     A.win_len[b] = 0;
   }
-  grid_dependents_launch();
 }
 
 // ---------------------------------------------------------------------------

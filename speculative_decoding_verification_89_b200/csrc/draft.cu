@@ -77,7 +77,7 @@ struct DraftArgs {
 
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A) {
-  grid_dependency_wait();
+  pdl_begin();
   asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");  // waited before remote writes
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
@@ -109,7 +109,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
   const DraftStat st = s_st;
   if (!st.ok || greedy) {  // uniform over the cluster
     if (rank == 0 && threadIdx.x == 0) finish(st.amax, 0.0, 0.0, !st.ok);
-    if (rank == 0) grid_dependents_launch();
     return;
   }
   const ProbCoef kp = make_coef(st.Lt, sc);
@@ -128,7 +127,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
     const double logq = bad ? 0.0 : kLn2 * ((double)load_elem(prow + tok) * sc.d - st.Lt);
     finish(tok, logq, st.H, bad);
   }
-  grid_dependents_launch();
 }
 
 template <typename T>

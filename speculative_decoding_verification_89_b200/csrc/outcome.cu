@@ -98,7 +98,7 @@ constexpr int kPairWarps = 4;
 
 template <typename T>
 __global__ void __launch_bounds__(kPairWarps * 32, 6) outcome_pair_kernel(OutcomeArgs A) {
-  grid_dependency_wait();
+  pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y, k = blockIdx.x, K = A.K, V = A.V, n = A.n_top;
   __shared__ double s_Lt[2];
@@ -182,7 +182,6 @@ __global__ void __launch_bounds__(kPairWarps * 32, 6) outcome_pair_kernel(Outcom
     for (int w2 = 0; w2 < kPairWarps; ++w2) zt += s_z[w2];
     A.zk[slot] = zt;
   }
-  grid_dependents_launch();
 }
 
 // ---------------------------------------------------------------------------
@@ -192,7 +191,7 @@ constexpr int kFinThreads = 256;
 
 template <typename T>
 __global__ void __launch_bounds__(kFinThreads) outcome_final_kernel(OutcomeArgs A) {
-  grid_dependency_wait();
+  pdl_begin();
   const int b = blockIdx.x, K = A.K, n = A.n_top, V = A.V;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   extern __shared__ double s_dyn[];  // [2K+1] log2-partitions, then [K+1] p_len

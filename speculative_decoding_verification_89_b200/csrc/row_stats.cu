@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     for (int s = 0; s < kRsStages; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
   }
-  grid_dependency_wait();
+  pdl_begin();
 
   // The rows that need statistics: the early ones in order, then the late
   // ones in order. Each thread tests a contiguous run of at most 32 rows; a
@@ -524,7 +524,6 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       mbar_wait_bounded(&bars[q], (phase >> q) & 1u, kWaitLimitNs);
     }
   }
-  grid_dependents_launch();
 }
 
 // ----------------------------------------------------------------------------
