@@ -5,8 +5,11 @@ Workload (per GPU): batched chain verification of B=64 sequences with K=8
 drafts over a V=128256 bf16 vocabulary (targets N(0, 2^2) plus a Zipf(1.1)
 log-prior over ids, drafts = target + N(0, 1), T = 1), followed by the
 paged-KV commit of a+1 rows per sequence (block 16, contexts U[512, 4096],
-128 KiB of K/V per token, hidden rows of 4096 bf16). One step = row
-statistics + accept/residual decide + commit, through the C ABI. Each step
+128 KiB of K/V per token, hidden rows of 4096 bf16). One step = the fused
+verify-and-commit path through the C ABI: row statistics; the check and draw
+per sequence, whose last sequence to pass its accept test plans the commit,
+copying the kept K/V rows that land in held blocks; then the remaining copy --
+three launches. Each step
 verifies a fresh Philox round and commits against the same committed prefix,
 so it rolls the previous round back and grows again: the pool stays bounded
 and every step does the same kind of work.
@@ -261,13 +264,12 @@ def run_ours(args, dist):
         capi.spec_chain_row_stats(tgt, drf, T, status, ws, stream=stream)
 
     def decide_commit(i):
-        capi.spec_chain_decide(tgt, drf, dt, T, prob.seed, sid, i, hist[i], out_tok, status, ws,
-                               stream=stream)
-        capi.spec_commit_paged(state.tables, state.seq_lens, base, hist[i], 1, state.free_stack,
-                               state.free_top, K + 1, status, block_size=16,
-                               kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
-                               hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
-                               hid_off=bufs.hid_off, stream=stream)
+        capi.spec_chain_decide_commit(tgt, drf, dt, T, prob.seed, sid, i, hist[i], out_tok,
+                                      state.tables, state.seq_lens, base, state.free_stack,
+                                      state.free_top, status, ws, block_size=16,
+                                      kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
+                                      hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
+                                      hid_off=bufs.hid_off, stream=stream)
 
     clocks = Clocks(dist.local)
     clocks.start()
@@ -338,18 +340,58 @@ def run_ours(args, dist):
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": ncu_traffic(), "algorithmic_bytes_per_launch": LOGIT_BYTES,
                      "launch_ms": rs_ms},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
+    result["two_call_step"] = run_two_call_step(args, prob, state, bufs, base, dev, dist)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, prob, state, bufs, base, dev, dist)
     result["draft_step"] = run_draft_step(args, dev, dist, peak)
     result["outcome_law"] = run_outcome_law(args, prob, dev, dist, peak)
+    result["hier_step"] = run_hier_step(args, dev, dist, peak)
     if dist.world == 1 and dist.rank == 0:
         result["parity_spot_check"] = spot_check(prob, hist[0].cpu().numpy())
         if not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(prob, state)
     return result
+
+
+def run_two_call_step(args, prob, state, bufs, base, dev, dist):
+    """The same step as separate calls -- spec_verify_chain (row statistics,
+    decide) then spec_commit_paged (plan, copy): four launches, each waiting
+    for the one before."""
+    from speculative_decoding_verification_89_b200 import capi
+    n = max(10, min(args.steps, 2000))
+    acc = torch.empty((n, B), dtype=torch.int32, device=dev)
+    out = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = capi.workspace(B, K, V, torch.bfloat16, device=dev)
+
+    def step(i):
+        capi.spec_verify_chain(prob.tgt, prob.drf, prob.draft_tok, prob.temperature, prob.seed,
+                               prob.seq_id, i, acc[i], out, status, ws)
+        capi.spec_commit_paged(state.tables, state.seq_lens, base, acc[i], 1, state.free_stack,
+                               state.free_top, K + 1, status, block_size=16,
+                               kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
+                               hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
+                               hid_off=bufs.hid_off)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.reduce(e0.elapsed_time(e1), "max")
+    if int(status.item()) != 0:
+        raise RuntimeError("device status during the two-call run")
+    tokens = float((acc.cpu().numpy() + 1).sum())
+    return {"steps": n, "ms_per_step": ms / n, "tokens_per_s": tokens / (ms * 1e-3),
+            "gpu_launches_per_step": 4}
 
 
 def run_draft_step(args, dev, dist, peak):
@@ -437,6 +479,74 @@ def run_outcome_law(args, prob, dev, dist, peak):
             "gpu_launches_per_call": 3}
 
 
+def run_hier_step(args, dev, dist, peak):
+    """Two-stage verification at the large mixed-temperature shape (B=256,
+    K=N_i=4, V=151936 fp32, 51 greedy sequences), each call from an empty
+    window: stage one always, stage two for the sequences whose window then
+    holds N_i tokens. A call's algorithmic bytes are the logit rows it must
+    read once: stage one K+1 L_i rows, plus K L_d rows for a sampled
+    sequence; stage two W+1 L_f rows per firing sequence, W = a1 + 1. Each
+    call is timed alone (CUDA events around it, the window reset outside)."""
+    from speculative_decoding_verification_89_b200 import capi
+    from speculative_decoding_verification_89_b200 import workloads as W
+    hp = W.hier_mixed(device=dev)
+    Bh, Kh, Ni, Vh = hp.lg_f.shape[0], hp.K, hp.Ni, hp.lg_f.shape[2]
+    WC = Ni + Kh
+    i32 = dict(dtype=torch.int32, device=dev)
+    win_len = torch.zeros(Bh, **i32)
+    win_tok = torch.full((Bh, WC), -1, **i32)
+    win_stat = torch.zeros((Bh, WC, 2), dtype=torch.float64, device=dev)
+    acc1, acc2 = torch.empty(Bh, **i32), torch.empty(Bh, **i32)
+    ctok, cn = torch.empty((Bh, WC + 1), **i32), torch.empty(Bh, **i32)
+    status = torch.zeros(1, **i32)
+    ws = capi.workspace(Bh, Kh, Vh, hp.lg_f.dtype, Ni=Ni, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    drafts = torch.randint(0, Vh, (Bh, Kh), generator=gen, device=dev, dtype=torch.int32)
+
+    def call(i):
+        capi.spec_verify_hier(hp.lg_d, hp.lg_i, hp.lg_f, Ni, drafts, hp.temperature, hp.seed,
+                              hp.seq_id, i, win_len, win_tok, win_stat, acc1, acc2, ctok, cn,
+                              status, ws)
+
+    for i in range(max(3, args.warmup)):
+        win_len.zero_()
+        call(i)
+    n = 20
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    a1s, a2s, cns = (torch.empty((n, Bh), **i32) for _ in range(3))
+    torch.cuda.synchronize()
+    dist.barrier()
+    for i in range(n):
+        win_len.zero_()
+        ev[i][0].record()
+        call(1000 + i)
+        ev[i][1].record()
+        a1s[i].copy_(acc1)
+        a2s[i].copy_(acc2)
+        cns[i].copy_(cn)
+    torch.cuda.synchronize()
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev)
+    ms = dist.reduce(ms, "max")
+    if int(status.item()) != 0:
+        raise RuntimeError(f"two-stage verification: device status {int(status.item())}")
+    greedy = (hp.temperature == 0).cpu().numpy()
+    a1, a2 = a1s.cpu().numpy(), a2s.cpu().numpy()
+    stage1 = ((Kh + 1) + np.where(greedy, 0, Kh)).sum() * n
+    stage2 = np.where(a2 >= 0, a1 + 2, 0).sum()
+    nbytes = int(stage1 + stage2) * Vh * hp.lg_f.element_size()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "two-stage verification, B=256, K=N_i=4, V=151936 fp32, 51 greedy "
+                        "sequences, each call from an empty window",
+            "us_per_call": ms * 1e3 / n, "calls": n,
+            "stage_two_sequences_per_call": float((a2 >= 0).sum()) / n,
+            "algorithmic_bytes_per_call": nbytes / n,
+            "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / peak,
+            "committed_tokens_per_s": float(cns.sum().item()) / (ms * 1e-3),
+            "gpu_launches_per_call": 4}
+
+
 def run_e2e(args, prob, state, bufs, base, dev, dist):
     """Same step through the public API with pinned host inputs: each step
     copies its logits, drafts, temperatures, ids and staged K/V + hidden rows
@@ -460,12 +570,12 @@ def run_e2e(args, prob, state, bufs, base, dev, dist):
     def step(i):
         for k in host:
             d[k].copy_(host[k], non_blocking=True)
-        capi.spec_verify_chain(d["tgt"], d["drf"], d["dt"], d["T"], prob.seed, d["sid"], i, acc,
-                               out, status, ws, stream=stream)
-        capi.spec_commit_paged(state.tables, state.seq_lens, base, acc, 1, state.free_stack,
-                               state.free_top, K + 1, status, block_size=16,
-                               kv_stage=d["kv"], kv_pool=bufs.kv_pool, hid_stage=d["hid"],
-                               hid_out=bufs.hid_out, hid_off=bufs.hid_off, stream=stream)
+        capi.spec_verify_chain_commit(d["tgt"], d["drf"], d["dt"], d["T"], prob.seed, d["sid"],
+                                      i, acc, out, state.tables, state.seq_lens, base,
+                                      state.free_stack, state.free_top, status, ws,
+                                      block_size=16, kv_stage=d["kv"], kv_pool=bufs.kv_pool,
+                                      hid_stage=d["hid"], hid_out=bufs.hid_out,
+                                      hid_off=bufs.hid_off, stream=stream)
         acc_h[i].copy_(acc, non_blocking=True)
         out_h[i].copy_(out, non_blocking=True)
 

@@ -85,6 +85,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 #define SPEC_MAX_TOP 32          /* outcomes kept per sequence        */
 #define SPEC_MAX_V (1 << 21)     /* vocabulary size                   */
 #define SPEC_MAX_COMMIT_B 16384  /* sequences per paged commit        */
+#define SPEC_MAX_FUSED_B 4096    /* sequences per fused verify+commit */
 
 /* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
  * chain call, Ni > 0 a two-stage call. Returns 0 for invalid sizes. */
@@ -231,6 +232,68 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
                       void* kv_pool, int layers, int kv_heads, int head_dim,
                       const void* hid_stage, void* hid_out, int32_t* hid_off,
                       int hidden, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Chain verification and the paged commit of its kept rows in one call
+ * ([HS] Verlustfreie Garantie, KV-Cache reuse and batch-inference bullets).
+ *
+ * Same results as spec_verify_chain followed, on the same stream, by
+ * spec_commit_paged with keep = accept_len, keep_add = 1 and Kp1 = K + 1
+ * (a + 1 rows kept per sequence: the accepted drafts and the drawn token),
+ * in three launches instead of four: the row statistics; one cluster per
+ * sequence that runs the check and the draw, whose last sequence to finish
+ * its accept test plans the commit, and which copies the sequence's kept
+ * K/V rows that land in blocks it already holds; then the copy of the hidden
+ * rows and of the K/V rows that need a newly allocated block.
+ * Arguments: those of spec_verify_chain (the logits, drafts, temperatures,
+ * Philox key, accept_len, out_tok, diag, workspace) and of spec_commit_paged
+ * (tables, lengths, base_len, stack, pool, stage and hidden buffers), with
+ * the same layouts and ownership; B <= SPEC_MAX_FUSED_B. The workspace is
+ * spec_workspace_bytes(B, K, V, dtype, 0) bytes.
+ * Errors: host-side argument errors return without launching. On the
+ * device, a sequence that fails the check (invalid temperature, draft id
+ * or logits) sets SPEC_EDEVICE, accept_len = -1 and out_tok = -1 for it, and
+ * then nothing is committed; a commit that fails its checks sets
+ * SPEC_EINVAL or SPEC_ENOBLOCKS. In both cases no table, length, stack
+ * entry, hidden row or offset changes and the verification outputs stand,
+ * but -- unlike spec_commit_paged -- the pool slots of the kept rows of the
+ * sequences that passed the check (positions base_len .. base_len + a), in
+ * blocks those sequences already held, may hold the staged rows: they lie
+ * past the committed prefix. A status already set on entry commits nothing.
+ * ------------------------------------------------------------------------- */
+int spec_verify_chain_commit(const void* tgt, int64_t ld_tgt, const void* drf,
+                             int64_t ld_drf, int dtype, int B, int K, int V,
+                             const int32_t* draft_tok, const float* temperature,
+                             uint64_t seed, const int32_t* seq_id, uint32_t round,
+                             int32_t* accept_len, int32_t* out_tok, double* diag,
+                             int block_size, int max_blocks, int32_t* block_tables,
+                             int32_t* seq_lens, const int32_t* base_len,
+                             int32_t* free_stack, int32_t* free_top, int num_blocks,
+                             const void* kv_stage, void* kv_pool, int layers,
+                             int kv_heads, int head_dim, const void* hid_stage,
+                             void* hid_out, int32_t* hid_off, int hidden,
+                             int32_t* dev_status, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* The second half of spec_verify_chain_commit (its last two launches), for
+ * callers that time or schedule the row statistics apart: the workspace,
+ * logits and temperatures must be those of the preceding
+ * spec_chain_row_stats call on the same stream (which also clears the
+ * workspace word this call's accept launch counts finished sequences in).
+ * Arguments, results and errors as for spec_verify_chain_commit. */
+int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf,
+                             int64_t ld_drf, int dtype, int B, int K, int V,
+                             const int32_t* draft_tok, const float* temperature,
+                             uint64_t seed, const int32_t* seq_id, uint32_t round,
+                             int32_t* accept_len, int32_t* out_tok, double* diag,
+                             int block_size, int max_blocks, int32_t* block_tables,
+                             int32_t* seq_lens, const int32_t* base_len,
+                             int32_t* free_stack, int32_t* free_top, int num_blocks,
+                             const void* kv_stage, void* kv_pool, int layers,
+                             int kv_heads, int head_dim, const void* hid_stage,
+                             void* hid_out, int32_t* hid_off, int hidden,
+                             int32_t* dev_status, void* ws, size_t ws_bytes,
+                             void* stream);
 
 /* ---------------------------------------------------------------------------
  * Draft step ([HS] Kernmechanismus: the shallow exit L_d drafts the tokens the

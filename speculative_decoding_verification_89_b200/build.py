@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libspecverify.so")
 SOURCES = ["row_stats.cu", "decide.cu", "draft.cu", "outcome.cu", "commit.cu", "capi.cu",
            "noalloc.cu"]
-HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh"]
+HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh", "commit.cuh"]
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",

@@ -42,6 +42,12 @@ _SIGS = {
                               _u32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "spec_commit_paged": (_i, [_i, _i, _i, _p, _p, _p, _p, _i, _p, _p, _i, _i, _p, _p,
                                _i, _i, _i, _p, _p, _p, _i, _p, _p]),
+    "spec_verify_chain_commit": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
+                                      _u32, _p, _p, _p, _i, _i, _p, _p, _p, _p, _p, _i, _p,
+                                      _p, _i, _i, _i, _p, _p, _p, _i, _p, _p, _sz, _p]),
+    "spec_chain_decide_commit": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
+                                      _u32, _p, _p, _p, _i, _i, _p, _p, _p, _p, _p, _i, _p,
+                                      _p, _i, _i, _i, _p, _p, _p, _i, _p, _p, _sz, _p]),
     "spec_philox_uniforms": (_i, [_u64, _p, _i, _p, _p]),
     "spec_last_cuda_error": (ctypes.c_char_p, []),
     "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
@@ -195,6 +201,17 @@ def spec_commit_paged(block_tables, seq_lens, base_len, keep, keep_add, free_sta
                       stream=None):
     B, max_blocks = block_tables.shape
     num_blocks = free_stack.numel()
+    layers, kv_heads, head_dim, hidden = _kv_shapes(kv_stage, kv_pool, hid_stage, num_blocks,
+                                                    block_size)
+    rc = _lib.spec_commit_paged(
+        B, block_size, max_blocks, _ptr(block_tables), _ptr(seq_lens), _ptr(base_len),
+        _ptr(keep), keep_add, _ptr(free_stack), _ptr(free_top), num_blocks, Kp1,
+        _ptr(kv_stage), _ptr(kv_pool), layers, kv_heads, head_dim, _ptr(hid_stage),
+        _ptr(hid_out), _ptr(hid_off), hidden, _ptr(dev_status), _stream(stream))
+    _check("spec_commit_paged", rc)
+
+
+def _kv_shapes(kv_stage, kv_pool, hid_stage, num_blocks, block_size):
     layers = kv_heads = head_dim = hidden = 0
     if kv_stage is not None:
         # kv_stage [B, Kp1, layers, 2, heads, dim]; kv_pool [N, layers, 2, bs, heads, dim]
@@ -205,12 +222,41 @@ def spec_commit_paged(block_tables, seq_lens, base_len, keep, keep_add, free_sta
             raise ValueError("pool shape does not match the block pool")
     if hid_stage is not None:
         hidden = hid_stage.shape[-1]
-    rc = _lib.spec_commit_paged(
-        B, block_size, max_blocks, _ptr(block_tables), _ptr(seq_lens), _ptr(base_len),
-        _ptr(keep), keep_add, _ptr(free_stack), _ptr(free_top), num_blocks, Kp1,
-        _ptr(kv_stage), _ptr(kv_pool), layers, kv_heads, head_dim, _ptr(hid_stage),
-        _ptr(hid_out), _ptr(hid_off), hidden, _ptr(dev_status), _stream(stream))
-    _check("spec_commit_paged", rc)
+    return layers, kv_heads, head_dim, hidden
+
+
+def spec_verify_chain_commit(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
+                             out_tok, block_tables, seq_lens, base_len, free_stack, free_top,
+                             dev_status, ws, block_size=16, kv_stage=None, kv_pool=None,
+                             hid_stage=None, hid_out=None, hid_off=None, diag=None,
+                             stream=None, _entry="spec_verify_chain_commit"):
+    """spec_verify_chain, then spec_commit_paged with keep = accept_len,
+    keep_add = 1, Kp1 = K + 1, as one call (three launches)."""
+    B, Kp1, V = tgt.shape
+    K = Kp1 - 1
+    max_blocks = block_tables.shape[1]
+    num_blocks = free_stack.numel()
+    layers, kv_heads, head_dim, hidden = _kv_shapes(kv_stage, kv_pool, hid_stage, num_blocks,
+                                                    block_size)
+    rc = getattr(_lib, _entry)(
+        _ptr(tgt), _rows(tgt, Kp1), _ptr(drf) if K > 0 else None,
+        _rows(drf, K) if K > 0 else 0, _dtype_code(tgt), B, K, V, _ptr(draft_tok),
+        _ptr(temperature), seed, _ptr(seq_id), rnd, _ptr(accept_len), _ptr(out_tok),
+        _ptr(diag), block_size, max_blocks, _ptr(block_tables), _ptr(seq_lens),
+        _ptr(base_len), _ptr(free_stack), _ptr(free_top), num_blocks, _ptr(kv_stage),
+        _ptr(kv_pool), layers, kv_heads, head_dim, _ptr(hid_stage), _ptr(hid_out),
+        _ptr(hid_off), hidden, _ptr(dev_status), _ptr(ws), ws.numel(), _stream(stream))
+    _check(_entry, rc)
+
+
+def spec_chain_decide_commit(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
+                             out_tok, block_tables, seq_lens, base_len, free_stack, free_top,
+                             dev_status, ws, **kw):
+    """The accept and draw-and-copy launches of spec_verify_chain_commit,
+    after spec_chain_row_stats on the same workspace."""
+    spec_verify_chain_commit(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
+                             out_tok, block_tables, seq_lens, base_len, free_stack, free_top,
+                             dev_status, ws, _entry="spec_chain_decide_commit", **kw)
 
 
 def spec_philox_uniforms(seed, ctr, out, stream=None):

@@ -21,12 +21,13 @@ int stat_tiles(int V, int dtype) {
 }
 
 struct Layout {
-  size_t part, fin, total;
+  size_t part, fin, kv_done, ticket, total;
   long long rows;
 };
 
 // Workspace: final row statistics and tile partials for the largest row set,
-// each region 256-byte aligned.
+// then the per-sequence copied-row counts and the ticket of the fused
+// verify-and-commit path, each region 256-byte aligned.
 bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   if (B < 0 || K < 0 || K > SPEC_MAX_K || V < 1 || V > SPEC_MAX_V) return false;
   if (dtype != SPEC_F32 && dtype != SPEC_BF16) return false;
@@ -37,7 +38,9 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   L->rows = rows;
   L->fin = 0;
   L->part = align_up((size_t)rows * sizeof(RowFinal));
-  L->total = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
+  L->kv_done = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
+  L->ticket = L->kv_done + align_up((size_t)B * sizeof(int32_t));
+  L->total = L->ticket + kAlign;
   return true;
 }
 
@@ -110,6 +113,7 @@ RsBuffers rs_buffers(void* ws, const Layout& L) {
   RsBuffers b;
   b.part = reinterpret_cast<Partial*>((char*)ws + L.part);
   b.mom = nullptr;
+  b.zero = nullptr;
   return b;
 }
 
@@ -136,6 +140,59 @@ DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_to
 }
 
 }  // namespace
+
+// Host checks of a paged commit's arguments; fills *out. SPEC_OK with B == 0
+// means nothing to do.
+static int commit_args(int B, int block_size, int max_blocks, int32_t* block_tables,
+                       int32_t* seq_lens, const int32_t* base_len, const int32_t* keep,
+                       int keep_add, int32_t* free_stack, int32_t* free_top, int num_blocks,
+                       int Kp1, const void* kv_stage, void* kv_pool, int layers, int kv_heads,
+                       int head_dim, const void* hid_stage, void* hid_out, int32_t* hid_off,
+                       int hidden, int32_t* dev_status, CommitArgs* out) {
+  if (B < 0 || B > SPEC_MAX_COMMIT_B || block_size < 1 || max_blocks < 0 || num_blocks < 0 ||
+      Kp1 < 0)
+    return SPEC_EINVAL;
+  if (B == 0) return SPEC_OK;
+  if (!block_tables || !seq_lens || !keep || !free_stack || !free_top) return SPEC_EINVAL;
+  if ((long long)B * Kp1 > (1LL << 31) - 1 || (long long)B * max_blocks > (1LL << 31) - 1)
+    return SPEC_EINVAL;
+  CommitArgs& a = *out;
+  std::memset(&a, 0, sizeof(a));
+  if ((kv_stage == nullptr) != (kv_pool == nullptr)) return SPEC_EINVAL;
+  if (kv_stage) {
+    if (layers < 1 || kv_heads < 1 || head_dim < 1) return SPEC_EINVAL;
+    const long long seg = 2LL * kv_heads * head_dim;
+    if (seg % 16 != 0 || seg > (1 << 30)) return SPEC_EINVAL;
+    if (!aligned(kv_stage, 16) || !aligned(kv_pool, 16)) return SPEC_EINVAL;
+    a.layers = layers;
+    a.seg_bytes = (int)seg;
+  }
+  if ((hid_stage == nullptr) != (hid_out == nullptr)) return SPEC_EINVAL;
+  if (hid_stage) {
+    if (hidden < 1 || (2LL * hidden) % 16 != 0 || !hid_off) return SPEC_EINVAL;
+    if (!aligned(hid_stage, 16) || !aligned(hid_out, 16)) return SPEC_EINVAL;
+    a.hid_bytes = 2 * hidden;
+  }
+  a.B = B;
+  a.block_size = block_size;
+  a.max_blocks = max_blocks;
+  a.num_blocks = num_blocks;
+  a.Kp1 = Kp1;
+  a.keep_add = keep_add;
+  a.tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.base_len = base_len;
+  a.keep = keep;
+  a.free_stack = free_stack;
+  a.free_top = free_top;
+  a.kv_stage = (const unsigned char*)kv_stage;
+  a.kv_pool = (unsigned char*)kv_pool;
+  a.hid_stage = (const unsigned char*)hid_stage;
+  a.hid_out = (unsigned char*)hid_out;
+  a.hid_off = hid_off;
+  a.status = dev_status;
+  return SPEC_OK;
+}
 
 #pragma GCC visibility push(default)
 extern "C" {
@@ -193,8 +250,10 @@ int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64
   rows.temperature = temperature;
   rows.K = K;
   rows.late_pos = late_positions(B, V, dtype, 2);
-  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, ck.L),
-                                      dev_status, (cudaStream_t)stream));
+  RsBuffers rb = rs_buffers(ws, ck.L);
+  rb.zero = reinterpret_cast<int32_t*>((char*)ws + ck.L.ticket);  // for spec_chain_decide_commit
+  return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rb, dev_status,
+                                      (cudaStream_t)stream));
 }
 
 int spec_chain_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
@@ -306,49 +365,80 @@ int spec_commit_paged(int B, int block_size, int max_blocks, int32_t* block_tabl
                       const void* kv_stage, void* kv_pool, int layers, int kv_heads, int head_dim,
                       const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden,
                       int32_t* dev_status, void* stream) {
-  if (B < 0 || B > SPEC_MAX_COMMIT_B || block_size < 1 || max_blocks < 0 || num_blocks < 0 ||
-      Kp1 < 0)
-    return SPEC_EINVAL;
-  if (B == 0) return SPEC_OK;
-  if (!block_tables || !seq_lens || !keep || !free_stack || !free_top) return SPEC_EINVAL;
-  if ((long long)B * Kp1 > (1LL << 31) - 1 || (long long)B * max_blocks > (1LL << 31) - 1)
-    return SPEC_EINVAL;
   CommitArgs a;
-  std::memset(&a, 0, sizeof(a));
-  if ((kv_stage == nullptr) != (kv_pool == nullptr)) return SPEC_EINVAL;
-  if (kv_stage) {
-    if (layers < 1 || kv_heads < 1 || head_dim < 1) return SPEC_EINVAL;
-    const long long seg = 2LL * kv_heads * head_dim;
-    if (seg % 16 != 0 || seg > (1 << 30)) return SPEC_EINVAL;
-    if (!aligned(kv_stage, 16) || !aligned(kv_pool, 16)) return SPEC_EINVAL;
-    a.layers = layers;
-    a.seg_bytes = (int)seg;
-  }
-  if ((hid_stage == nullptr) != (hid_out == nullptr)) return SPEC_EINVAL;
-  if (hid_stage) {
-    if (hidden < 1 || (2LL * hidden) % 16 != 0 || !hid_off) return SPEC_EINVAL;
-    if (!aligned(hid_stage, 16) || !aligned(hid_out, 16)) return SPEC_EINVAL;
-    a.hid_bytes = 2 * hidden;
-  }
-  a.B = B;
-  a.block_size = block_size;
-  a.max_blocks = max_blocks;
-  a.num_blocks = num_blocks;
-  a.Kp1 = Kp1;
-  a.keep_add = keep_add;
-  a.tables = block_tables;
-  a.seq_lens = seq_lens;
-  a.base_len = base_len;
-  a.keep = keep;
-  a.free_stack = free_stack;
-  a.free_top = free_top;
-  a.kv_stage = (const unsigned char*)kv_stage;
-  a.kv_pool = (unsigned char*)kv_pool;
-  a.hid_stage = (const unsigned char*)hid_stage;
-  a.hid_out = (unsigned char*)hid_out;
-  a.hid_off = hid_off;
-  a.status = dev_status;
+  const int rc = commit_args(B, block_size, max_blocks, block_tables, seq_lens, base_len, keep,
+                             keep_add, free_stack, free_top, num_blocks, Kp1, kv_stage, kv_pool,
+                             layers, kv_heads, head_dim, hid_stage, hid_out, hid_off, hidden,
+                             dev_status, &a);
+  if (rc != SPEC_OK || B == 0) return rc;
   return cuda_status(launch_commit(a, (cudaStream_t)stream));
+}
+
+int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                             int dtype, int B, int K, int V, const int32_t* draft_tok,
+                             const float* temperature, uint64_t seed, const int32_t* seq_id,
+                             uint32_t round, int32_t* accept_len, int32_t* out_tok, double* diag,
+                             int block_size, int max_blocks, int32_t* block_tables,
+                             int32_t* seq_lens, const int32_t* base_len, int32_t* free_stack,
+                             int32_t* free_top, int num_blocks, const void* kv_stage,
+                             void* kv_pool, int layers, int kv_heads, int head_dim,
+                             const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 0 || B > SPEC_MAX_FUSED_B || K < 0 || K > SPEC_MAX_K) return SPEC_EINVAL;
+  FusedArgs f;
+  const int rc = commit_args(B, block_size, max_blocks, block_tables, seq_lens, base_len,
+                             accept_len, 1, free_stack, free_top, num_blocks, K + 1, kv_stage,
+                             kv_pool, layers, kv_heads, head_dim, hid_stage, hid_out, hid_off,
+                             hidden, dev_status, &f.cm);
+  if (rc != SPEC_OK) return rc;
+  const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
+                                    ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!seq_id || !out_tok || (K > 0 && !draft_tok)) return SPEC_EINVAL;
+  const int es = elem_size(dtype);
+  f.d.c = common_args(dtype, B, K, V, draft_tok, temperature, seed, seq_id, round, diag,
+                      dev_status, ws, ck.L);
+  f.d.tgt = (const unsigned char*)tgt;
+  f.d.drf = (const unsigned char*)drf;
+  f.d.ld_tgt = ld_tgt * es;
+  f.d.ld_drf = ld_drf * es;
+  f.d.accept_len = accept_len;
+  f.d.out_tok = out_tok;
+  f.kv_done = reinterpret_cast<int32_t*>((char*)ws + ck.L.kv_done);
+  f.ticket = reinterpret_cast<int32_t*>((char*)ws + ck.L.ticket);
+  return cuda_status(launch_chain_fused(f, (cudaStream_t)stream));
+}
+
+int spec_verify_chain_commit(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                             int dtype, int B, int K, int V, const int32_t* draft_tok,
+                             const float* temperature, uint64_t seed, const int32_t* seq_id,
+                             uint32_t round, int32_t* accept_len, int32_t* out_tok, double* diag,
+                             int block_size, int max_blocks, int32_t* block_tables,
+                             int32_t* seq_lens, const int32_t* base_len, int32_t* free_stack,
+                             int32_t* free_top, int num_blocks, const void* kv_stage,
+                             void* kv_pool, int layers, int kv_heads, int head_dim,
+                             const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  // Every host check of the second half first, so a refused call launches nothing.
+  if (B < 0 || B > SPEC_MAX_FUSED_B || K < 0 || K > SPEC_MAX_K) return SPEC_EINVAL;
+  CommitArgs cm;
+  int rc = commit_args(B, block_size, max_blocks, block_tables, seq_lens, base_len, accept_len,
+                       1, free_stack, free_top, num_blocks, K + 1, kv_stage, kv_pool, layers,
+                       kv_heads, head_dim, hid_stage, hid_out, hid_off, hidden, dev_status, &cm);
+  if (rc != SPEC_OK) return rc;
+  const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
+                                    ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!seq_id || !out_tok || (K > 0 && !draft_tok)) return SPEC_EINVAL;
+  rc = spec_chain_row_stats(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, dev_status,
+                            ws, ws_bytes, stream);
+  if (rc != SPEC_OK) return rc;
+  return spec_chain_decide_commit(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok,
+                                  temperature, seed, seq_id, round, accept_len, out_tok, diag,
+                                  block_size, max_blocks, block_tables, seq_lens, base_len,
+                                  free_stack, free_top, num_blocks, kv_stage, kv_pool, layers,
+                                  kv_heads, head_dim, hid_stage, hid_out, hid_off, hidden,
+                                  dev_status, ws, ws_bytes, stream);
 }
 
 size_t spec_draft_workspace_bytes(int B, int V, int dtype) {

@@ -1,0 +1,291 @@
+// Paged-commit bodies shared by the commit launches and the fused
+// verify-and-commit path: the planner (one CTA) and the row copy (many CTAs).
+// HiSpec (gist.science summary of arXiv 2510.01336), section 2: buffered KV
+// entries and hidden states of rejected tokens are dropped before the next
+// phase; block tables let every sequence keep its own number of tokens.
+#pragma once
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace specv {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kCopyThreads = 256;
+constexpr int kCopyCtasPerSm = 8;  // 64 warps per SM: one round of items for most calls
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Block-wide exclusive scan of four ints per thread (any block of up to 1024
+// threads, a multiple of 32); totals returned in tot.
+static __device__ int4 block_excl_scan4(int4 v, int4* tot) {
+  __shared__ int4 warp_sums[32];
+  __shared__ int4 s_tot;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int4 incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int yx = __shfl_up_sync(0xffffffffu, incl.x, o);
+    const int yy = __shfl_up_sync(0xffffffffu, incl.y, o);
+    const int yz = __shfl_up_sync(0xffffffffu, incl.z, o);
+    const int yw = __shfl_up_sync(0xffffffffu, incl.w, o);
+    if (lane >= o) { incl.x += yx; incl.y += yy; incl.z += yz; incl.w += yw; }
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int4 w = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : make_int4(0, 0, 0, 0);
+    int4 wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yx = __shfl_up_sync(0xffffffffu, wi.x, o);
+      const int yy = __shfl_up_sync(0xffffffffu, wi.y, o);
+      const int yz = __shfl_up_sync(0xffffffffu, wi.z, o);
+      const int yw = __shfl_up_sync(0xffffffffu, wi.w, o);
+      if (lane >= o) { wi.x += yx; wi.y += yy; wi.z += yz; wi.w += yw; }
+    }
+    warp_sums[lane] = make_int4(wi.x - w.x, wi.y - w.y, wi.z - w.z, wi.w - w.w);  // exclusive
+    if (lane == 31) s_tot = wi;
+  }
+  __syncthreads();
+  const int4 base = warp_sums[warp];
+  *tot = s_tot;
+  return make_int4(base.x + incl.x - v.x, base.y + incl.y - v.y, base.z + incl.z - v.z,
+                   base.w + incl.w - v.w);
+}
+
+// One CTA. Two rounds of global reads: (1) the per-sequence lengths and
+// counts, (2) after a block scan, every covered table entry (validation), the
+// tails to be freed and the stack entries to be popped below the old top,
+// the last two cached in shared memory. Every check is made before anything
+// is written; the writes then need no further reads while the caches hold.
+constexpr int kPushCache = 2048;   // freed entries cached in push order
+constexpr int kStackCache = 2048;  // stack entries popped from below the old top
+
+// s_seq: dynamic shared memory of 3 * B ints. Runs in any block of up to 1024
+// threads. The kept counts are read from L2: in the fused verify-and-commit
+// path they were written by other CTAs of the same grid.
+static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
+  // [3][B]: table-entry prefix, new length, kept
+  int* s_nbp = s_seq;             // blocks held before, then their exclusive prefix
+  int* s_len = s_seq + a.B;
+  int* s_kept = s_seq + 2 * a.B;
+  __shared__ int s_push[kPushCache];
+  __shared__ int s_stack[kStackCache];
+  __shared__ int s_bad, s_sbad, s_code, s_ft;
+  // The status word is read with the per-sequence inputs, not before them.
+  const int32_t st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
+  if (threadIdx.x == 0) { s_bad = 0; s_sbad = 0; s_code = 0; s_ft = *a.free_top; }
+  const int bs = a.block_size;
+  // Each thread owns a contiguous run of sequences (sequence order matters
+  // for the allocation order).
+  const int per = ceil_div(a.B, blockDim.x);
+  const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
+  int4 cnt = make_int4(0, 0, 0, 0);  // frees, allocations, kept rows, table entries
+  int bad = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int old_len = a.seq_lens[b];
+    const int base = a.base_len ? a.base_len[b] : old_len;
+    const int kept = __ldcg(a.keep + b) + a.keep_add;
+    int nbo = ceil_div(max(old_len, 0), bs), nbn = nbo;
+    bool ok = true;
+    if (kept < 0 || kept > a.Kp1 || base < 0 || base > old_len || old_len < 0) {
+      ok = false;
+    } else {
+      nbn = ceil_div(base + kept, bs);
+      if (nbo > a.max_blocks || nbn > a.max_blocks) ok = false;
+    }
+    if (!ok) bad = 1;
+    const int held = min(nbo, a.max_blocks);
+    s_nbp[b] = held;
+    s_len[b] = ok ? base + kept : 0;
+    s_kept[b] = kept;
+    cnt.x += max(0, nbo - nbn);
+    cnt.y += max(0, nbn - nbo);
+    cnt.z += kept;
+    cnt.w += held;
+  }
+  if (st0 != SPEC_OK) return;  // sticky error: the same in every thread
+  if (bad) atomicOr(&s_bad, 1);
+  int4 tot;
+  const int4 pre = block_excl_scan4(cnt, &tot);  // its barriers also publish s_ft, s_bad
+  {
+    int q = pre.w;  // blocks held -> their exclusive prefix, over this thread's run
+    for (int b = b0; b < b1; ++b) {
+      const int h = s_nbp[b];
+      s_nbp[b] = q;
+      q += h;
+    }
+  }
+  const int F = tot.x, A = tot.y, KT = tot.z, NE = tot.w, ft = s_ft;
+  auto held = [&](int b) { return (b + 1 < a.B ? s_nbp[b + 1] : NE) - s_nbp[b]; };
+  __syncthreads();
+  const bool sizes_ok = !s_bad && ft >= 0 && ft <= a.num_blocks && ft + F <= a.num_blocks;
+  // Pops come from stack positions [lo, ft + F): those at or above ft are the
+  // entries pushed by this call, those below ft are read here.
+  const int lo = max(0, ft + F - A);
+  const bool cached = F <= kPushCache && ft - lo <= kStackCache;
+  if (sizes_ok) {
+    // Every covered table entry must be a valid block id: 1, 2 or 4
+    // sequences per warp (32, 16 or 8 lanes each), 16 loads in flight per lane.
+    {
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+      const int need = ceil_div(a.B, nwarps);
+      const int spw = need <= 1 ? 1 : (need <= 2 ? 2 : 4);
+      const int lps = 32 / spw, sub = lane / lps, sl = lane % lps;
+      constexpr int kBatch = 16;
+      for (int bb = warp * spw; bb < a.B; bb += nwarps * spw) {
+        const int b = bb + sub;
+        const int nb = b < a.B ? held(b) : 0;
+        const int32_t* tab = a.tables + (size_t)(b < a.B ? b : 0) * a.max_blocks;
+        for (int i0 = sl; i0 < nb; i0 += lps * kBatch) {
+          int v[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) v[k] = (i0 + lps * k < nb) ? tab[i0 + lps * k] : 0;
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k)
+            if (i0 + lps * k < nb && (v[k] < 0 || v[k] >= a.num_blocks)) bad = 1;
+        }
+      }
+    }
+    // Tails to be freed, cached in push order (same round of reads).
+    if (cached) {
+      int fpos = pre.x;
+      for (int b = b0; b < b1; ++b) {
+        const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+        for (int i = ceil_div(s_len[b], bs); i < held(b); ++i) s_push[fpos++] = tab[i];
+      }
+    }
+    if (bad) atomicOr(&s_bad, 1);
+    // Stack entries popped from below the old top must be valid ids.
+    int sbad = 0;
+    for (int p = lo + threadIdx.x; p < ft; p += blockDim.x) {
+      const int x = a.free_stack[p];
+      if (x < 0 || x >= a.num_blocks) sbad = 1;
+      if (cached) s_stack[p - lo] = x;
+    }
+    if (sbad) atomicOr(&s_sbad, 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // the order of the checks fixes which status wins
+    if (!sizes_ok || s_bad) s_code = SPEC_EINVAL;
+    else if (ft + F < A) s_code = SPEC_ENOBLOCKS;
+    else if (s_sbad) s_code = SPEC_EINVAL;
+  }
+  __syncthreads();
+  if (s_code != 0) {
+    if (threadIdx.x == 0) set_status(a.status, s_code);
+    return;
+  }
+  // Frees: push table tails in sequence order.
+  int fpos = pre.x;
+  for (int b = b0; b < b1; ++b) {
+    int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+    for (int i = ceil_div(s_len[b], bs); i < held(b); ++i) {
+      a.free_stack[ft + fpos] = cached ? s_push[fpos] : tab[i];
+      ++fpos;
+      tab[i] = -1;
+    }
+  }
+  if (!cached) __syncthreads();  // pops below read the pushed entries back
+  // Allocations: pop from the top in sequence order; lengths and offsets.
+  const int top = ft + F;
+  int k = pre.y, off = pre.z;
+  for (int b = b0; b < b1; ++b) {
+    int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+    const int nbn = ceil_div(s_len[b], bs);
+    for (int i = held(b); i < nbn; ++i) {
+      const int p = top - 1 - (k++);
+      tab[i] = !cached ? a.free_stack[p] : (p >= ft ? s_push[p - ft] : s_stack[p - lo]);
+    }
+    if (a.hid_off) a.hid_off[b] = off;
+    off += s_kept[b];
+    a.seq_lens[b] = s_len[b];
+  }
+  if (threadIdx.x == 0) {
+    *a.free_top = top - A;
+    if (a.hid_off) a.hid_off[a.B] = KT;
+  }
+}
+
+// Copy of kept token rows. Every CTA scans the kept counts (the planner has
+// checked them) so kept rows are numbered 0..KT-1; warps then stride over
+// (kept row, segment) items. A segment is one (layer, K|V) slice of a token's
+// staged row (kv_heads * head_dim * 2 bytes, contiguous in both stage and
+// pool); the hidden row is cut into pieces of the same size after them.
+// s_off: dynamic shared memory of 2 * B + 1 ints. CTA `cta` of `ncta` taking
+// part; any block size that is a multiple of 32 and at least 64.
+static __device__ void copy_body(const CommitArgs& a, int cta, int ncta, int* s_off) {
+  // [B + 1] exclusive scan of kept rows, then [B] new lengths
+  int* s_len = s_off + a.B + 1;
+  // The status word is read with the counts, and checked once they are in.
+  const int32_t st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int b = (int)threadIdx.x - 32; b >= 0 && b < a.B; b += blockDim.x - 32)
+    s_len[b] = a.seq_lens[b];  // the other warps, while warp 0 scans
+  if (warp == 0) {
+    int carry = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < a.B ? a.keep[b] + a.keep_add : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b < a.B) s_off[b] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_off[a.B] = carry;
+  }
+  __syncthreads();
+  if (st0 != SPEC_OK) return;  // sticky error: the same in every thread
+  const int KT = s_off[a.B];
+  const int nseg = a.kv_stage ? a.layers * 2 : 0;
+  const int piece = a.kv_stage ? a.seg_bytes : 2048;
+  const int nhid = a.hid_stage ? (a.hid_bytes + piece - 1) / piece : 0;
+  const int per_tok = nseg + nhid;
+  const int nitems = KT * per_tok;
+  const int nw = ncta * (blockDim.x >> 5);
+  for (int item = cta * (blockDim.x >> 5) + warp; item < nitems; item += nw) {
+    const int k = item / per_tok, sidx = item - k * per_tok;
+    int lo = 0, hi = a.B - 1;  // the sequence b with s_off[b] <= k < s_off[b + 1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= k) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo, i = k - s_off[b];
+    const int kept = s_off[b + 1] - s_off[b];
+    const uint4* src;
+    uint4* dst;
+    int nvec;
+    if (sidx < nseg) {
+      if (a.kv_done && i < a.kv_done[b]) continue;  // copied by the decide launch
+      const int pos = s_len[b] - kept + i;  // base_len + i
+      const int blk = a.tables[(size_t)b * a.max_blocks + pos / a.block_size];
+      const int slot = pos % a.block_size;
+      src = reinterpret_cast<const uint4*>(a.kv_stage +
+                                           (((size_t)b * a.Kp1 + i) * nseg + sidx) * a.seg_bytes);
+      dst = reinterpret_cast<uint4*>(
+          a.kv_pool + (((size_t)blk * nseg + sidx) * a.block_size + slot) * (size_t)a.seg_bytes);
+      nvec = a.seg_bytes / 16;
+    } else {
+      const int h = sidx - nseg;
+      const int off = h * piece, len = min(piece, a.hid_bytes - off);
+      src = reinterpret_cast<const uint4*>(a.hid_stage + ((size_t)b * a.Kp1 + i) * a.hid_bytes + off);
+      dst = reinterpret_cast<uint4*>(a.hid_out + (size_t)(s_off[b] + i) * a.hid_bytes + off);
+      nvec = len / 16;
+    }
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) r[u] = __ldcs(src + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) __stcs(dst + v0 + 32 * u, r[u]);
+    }
+  }
+}
+
+}  // namespace specv

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/spec_verify.h"
 
 namespace specv {
@@ -246,6 +248,39 @@ static inline int sm_count() {
     sms = v > 0 ? v : 148;
   }
   return sms;
+}
+
+// Lets kernel `fn` launch with `bytes` of dynamic shared memory: a kernel
+// whose static plus dynamic shared memory passes 48 KB needs the opt-in. The
+// largest size granted so far is kept per kernel, so the attribute is set
+// only when a launch needs more than before (and never lowered under a
+// concurrent caller).
+static cudaError_t reserve_dyn_smem(const void* fn, size_t bytes) {
+  static std::mutex mu;
+  static const void* fns[64];
+  static size_t granted[64];
+  static int n = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int i = 0;
+  while (i < n && fns[i] != fn) ++i;
+  if (i < n && granted[i] >= bytes) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e;
+  }
+  if (i < n) {
+    granted[i] = bytes;
+  } else if (n < 64) {
+    fns[n] = fn;
+    granted[n++] = bytes;
+  }
+  return cudaSuccess;
+}
+template <typename Kern>
+static cudaError_t reserve_dyn_smem(Kern* fn, size_t bytes) {
+  return reserve_dyn_smem(reinterpret_cast<const void*>(fn), bytes);
 }
 
 template <typename Kern, typename... Args>

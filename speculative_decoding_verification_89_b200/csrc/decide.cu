@@ -20,6 +20,7 @@
 // leader prefixes the tile sums, finds the tile holding u' * Z, rescans that
 // one tile and writes the outputs. No atomics, no spinning, no second launch.
 #include "draw.cuh"
+#include "commit.cuh"
 
 namespace specv {
 
@@ -476,21 +477,196 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
 }
 
 // ---------------------------------------------------------------------------
+// Chain verification fused with the paged commit
+// ---------------------------------------------------------------------------
+// chain_decide_kernel's cluster per sequence, which also commits. Once its
+// accept test is done the leader writes the kept count (a + 1) and takes a
+// ticket (one atomic, never awaited): the CTA that takes the B-th ticket has
+// seen every kept count and runs the commit planner (tables, free stack,
+// lengths, hidden offsets) before its share of the residual tiles. Beside the
+// draw, every CTA copies its share of the sequence's kept K/V rows that land
+// in blocks the sequence already holds (their pool slots are known without the
+// planner: blocks below ceil(old length / block) stay, the new length being
+// at least the base); kv_done[b] records how many leading rows were copied.
+// The launch after this one copies the hidden rows and the K/V rows that need
+// a newly allocated block.
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(FusedArgs F) {
+  pdl_begin();
+  cluster_arrive_relaxed();  // paired with the wait in cluster_rows
+  cg::cluster_group cl = cg::this_cluster();
+  const unsigned rank = cl.block_rank();
+  __shared__ SeqShared sh;
+  __shared__ Outcome s_out;
+  __shared__ int s_last;
+  extern __shared__ double dyn[];  // leader: [nrt] tile sums, [nrt] prefixes; planner: 3B ints
+  SeqShared* lsh = cl.map_shared_rank(&sh, 0);
+  double* ltsum = cl.map_shared_rank(dyn, 0);
+  const ChainDecideArgs& A = F.d;
+  const DecideCommon& c = A.c;
+  const CommitArgs& cm = F.cm;
+  const int b = blockIdx.y, K = c.K, V = c.V, per = 2 * K + 1;
+  const int nrt = residual_tiles(V);
+  // This sequence's commit inputs, read before any CTA can take the last
+  // ticket (the planner rewrites the length).
+  const int32_t st0 = c.status ? *(volatile int32_t*)c.status : SPEC_OK;
+  const int old_len = cm.seq_lens[b];
+  const int base = cm.base_len ? cm.base_len[b] : old_len;
+  const float Tb = c.temperature[b];
+  const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
+  double* diag = (rank == 0 && c.diag) ? c.diag + (size_t)b * (4 * K + 2) : nullptr;
+  const int32_t* drafts = c.draft_tok + (size_t)b * K;
+  int32_t* out = A.out_tok + (size_t)b * (K + 1);
+  auto tp = [&](int j) { return row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
+  auto dp = [&](int j) { return row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + j); };
+  auto dl = [&](int j) { return lsh->M[K + 1 + j] + lsh->L[K + 1 + j]; };
+  const Scale sc = (greedy || !tvalid) ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+  if (tvalid) {
+    const bool accept_warp = (threadIdx.x >> 5) == kDecWarps - 1;
+    AcceptPre pre{-1, 0.f, 0.f};
+    if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp, c, b, 0, 1);
+    cluster_rows(lsh, rank, c.part, c.ntiles, b * per, per,
+                 [&](int r) { return r <= K || !greedy; }, greedy, sc.hi, c.fin);
+    cl.sync();  // the leader holds every row's statistics
+    if (accept_warp) {
+      int bad;
+      float ud;
+      const int a = accept_scan<T>(lsh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
+                                   diag && !greedy ? diag + 2 * K + 1 : nullptr,
+                                   diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad, &ud);
+      if ((threadIdx.x & 31) == 0) s_out = Outcome{a, bad || !rows_ok(lsh, per), ud};
+    }
+  } else {
+    cluster_wait();  // completes the entry barrier: no rows to combine
+    if (threadIdx.x == 0) s_out = Outcome{0, 1, 0.f};
+  }
+  __syncthreads();
+  const Outcome o = s_out;
+  const int a = o.a;
+  // Leader: every output but a sampled sequence's drawn token, then the ticket.
+  if (rank == 0) {
+    if (o.bad) {
+      if (threadIdx.x == 0) {
+        set_status(c.status, SPEC_EDEVICE);
+        A.accept_len[b] = -1;
+      }
+      for (int j = threadIdx.x; j <= K; j += blockDim.x) out[j] = -1;
+      if (diag)
+        for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
+    } else {
+      for (int j = threadIdx.x; j <= K; j += blockDim.x)
+        if (j != a || greedy) out[j] = j < a ? drafts[j] : (j == a ? sh.amax[a] : -1);
+      if (threadIdx.x == 0) A.accept_len[b] = a;
+      if (diag) {
+        if (greedy)
+          for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
+        else
+          for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicAdd(F.ticket, 1) == c.B - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();  // every other sequence's kept count and status are visible
+      plan_body(cm, reinterpret_cast<int*>(dyn + 2 * nrt));
+    }
+  }
+  // Residual tile sums of a sampled sequence, a quarter per CTA.
+  const bool draw = !o.bad && !greedy;
+  const T* prow = nullptr;
+  const T* qrow = nullptr;
+  ProbCoef kp{}, kq{};
+  if (draw) {
+    prow = tp(a);
+    qrow = a < K ? dp(a) : nullptr;
+    kp = make_coef(lsh->M[a] + lsh->L[a], sc);
+    kq = make_coef(a < K ? dl(a) : 0.0, sc);
+    const int chunk = (nrt + kCluster - 1) / kCluster;
+    residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
+                          min(nrt, ((int)rank + 1) * chunk), ltsum);
+  }
+  // The tile sums are in the leader once every CTA has arrived; only the
+  // leader waits, the others go on to their copies.
+  asm volatile("barrier.cluster.arrive;" ::: "memory");
+  if (rank == 0) {
+    asm volatile("barrier.cluster.wait;" ::: "memory");
+    if (draw) {
+      double Z;
+      const int tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, o.u_draw, &Z);
+      if (threadIdx.x == 0) {
+        out[a] = tok;
+        if (diag) diag[4 * K + 1] = Z;
+      }
+    }
+  }
+  // Kept rows whose pool block the sequence already holds: i < n_early.
+  int n_early = 0;
+  if (st0 == SPEC_OK && !o.bad && cm.kv_stage && old_len >= 0 && base >= 0 && base <= old_len) {
+    const int held = min((old_len + cm.block_size - 1) / cm.block_size, cm.max_blocks);
+    n_early = max(0, min(a + 1, held * cm.block_size - base));
+  }
+  if (rank == 0 && threadIdx.x == 0) F.kv_done[b] = n_early;
+  const int nseg = cm.layers * 2, nvec = cm.seg_bytes / 16;
+  const int lane = threadIdx.x & 31, gw = (int)rank * kDecWarps + (threadIdx.x >> 5);
+  for (int item = gw; item < n_early * nseg; item += kCluster * kDecWarps) {
+    const int i = item / nseg, sidx = item - i * nseg;
+    const int pos = base + i;
+    const int blk = cm.tables[(size_t)b * cm.max_blocks + pos / cm.block_size];
+    if (blk < 0 || blk >= cm.num_blocks) continue;  // the planner refuses the call
+    const int slot = pos % cm.block_size;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        cm.kv_stage + (((size_t)b * cm.Kp1 + i) * nseg + sidx) * cm.seg_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(
+        cm.kv_pool + (((size_t)blk * nseg + sidx) * cm.block_size + slot) * (size_t)cm.seg_bytes);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) r[u] = __ldcs(src + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nvec) __stcs(dst + v0 + 32 * u, r[u]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Launchers: grid (kCluster, B), clusters of kCluster CTAs along x.
 // ---------------------------------------------------------------------------
 template <typename Kern, typename Args>
 static cudaError_t launch_decide(Kern k, const Args& a, cudaStream_t st) {
   const size_t smem = 2 * (size_t)residual_tiles(a.c.V) * sizeof(double);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-    return cudaGetLastError();
+  const cudaError_t e = reserve_dyn_smem(k, smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl_cluster(k, dim3(kCluster, a.c.B), dim3(kDecThreads), smem, st, kCluster, a);
 }
 
 cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st) {
   return a.c.dtype == SPEC_BF16 ? launch_decide(chain_decide_kernel<__nv_bfloat16>, a, st)
                                 : launch_decide(chain_decide_kernel<float>, a, st);
+}
+template <typename T>
+static cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st) {
+  auto k = chain_decide_commit_kernel<T>;
+  const size_t smem = 2 * (size_t)residual_tiles(a.d.c.V) * sizeof(double) +
+                      3 * (size_t)a.d.c.B * sizeof(int);
+  cudaError_t e = reserve_dyn_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl_cluster(k, dim3(kCluster, a.d.c.B), dim3(kDecThreads), smem, st, kCluster, a);
+  if (e != cudaSuccess) return e;
+  CommitArgs rest = a.cm;
+  rest.kv_done = a.kv_done;
+  return launch_commit_copy(rest, st);
+}
+
+cudaError_t launch_chain_fused(const FusedArgs& a, cudaStream_t st) {
+  return a.d.c.dtype == SPEC_BF16 ? launch_fused<__nv_bfloat16>(a, st)
+                                  : launch_fused<float>(a, st);
 }
 cudaError_t launch_hier1_decide(const HierDecideArgs& a, cudaStream_t st) {
   return a.c.dtype == SPEC_BF16 ? launch_decide(hier1_decide_kernel<__nv_bfloat16>, a, st)

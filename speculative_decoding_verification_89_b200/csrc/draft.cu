@@ -133,10 +133,8 @@ template <typename T>
 static cudaError_t launch_draw(const DraftArgs& a, cudaStream_t st) {
   auto k = draft_draw_kernel<T>;
   const size_t smem = 2 * (size_t)residual_tiles(a.V) * sizeof(double);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-    return cudaGetLastError();
+  const cudaError_t e = reserve_dyn_smem(k, smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl_cluster(k, dim3(kCluster, a.B), dim3(kDecThreads), smem, st, kCluster, a);
 }
 
@@ -152,6 +150,7 @@ cudaError_t launch_draft_step(int dtype, const unsigned char* lg, long long ld_b
   RsBuffers rb;
   rb.part = part;
   rb.mom = mom;
+  rb.zero = nullptr;
   cudaError_t e = launch_row_stats(dtype, rows, B, V, rb, status, st);
   if (e != cudaSuccess) return e;
   DraftArgs a;

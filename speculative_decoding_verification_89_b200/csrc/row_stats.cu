@@ -180,7 +180,7 @@ template <> __device__ __forceinline__ uint4 neg_inf_vec<float>() {
 template <typename T, typename Rows>
 __global__ void __launch_bounds__(kRsWarps * 32, 1)
     row_stats_kernel(Rows rows, int row_base, int nrows, int V, Partial* __restrict__ part,
-                     double* __restrict__ mom, int32_t* status) {
+                     double* __restrict__ mom, int32_t* status, int32_t* zero_word) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_wsum[kRsWarps];
   constexpr int kVec = VecOf<T>::n;
@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
     fence_barrier_init();
   }
   pdl_begin();
+  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
 
   // The rows that need statistics: the early ones in order, then the late
   // ones in order. Each thread tests a contiguous run of at most 32 rows; a
@@ -531,7 +532,7 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
 // ----------------------------------------------------------------------------
 template <typename T, typename Rows>
 static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, double* mom,
-                             int32_t* status, cudaStream_t st) {
+                             int32_t* zero_word, int32_t* status, cudaStream_t st) {
   auto kern = row_stats_kernel<T, Rows>;
   static bool smem_set = false;  // once per instantiation (same on every B200)
   if (!smem_set) {
@@ -553,7 +554,8 @@ static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, 
     if (grid > need) grid = need;
     if (grid < 1) grid = 1;
     const cudaError_t e = launch_pdl(kern, dim3((unsigned)grid), dim3(kRsWarps * 32),
-                                     (size_t)kRsSmemTotal, st, rows, r0, n, V, part, mom, status);
+                                     (size_t)kRsSmemTotal, st, rows, r0, n, V, part, mom, status,
+                                     zero_word);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -563,8 +565,8 @@ template <typename Rows>
 cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, const RsBuffers& b,
                              int32_t* status, cudaStream_t st) {
   if (dtype == SPEC_BF16)
-    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, b.mom, status, st);
-  return launch_rs<float>(rows, nrows, V, b.part, b.mom, status, st);
+    return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, b.mom, b.zero, status, st);
+  return launch_rs<float>(rows, nrows, V, b.part, b.mom, b.zero, status, st);
 }
 
 template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int,

@@ -110,6 +110,47 @@ def test_commit_host_argument_errors(lib):
     assert f(*bad) == -1                  # no tables
 
 
+def test_fused_host_argument_errors(lib):
+    """spec_verify_chain_commit and spec_chain_decide_commit refuse bad chain
+    or commit arguments before any launch (fake device pointers are never
+    dereferenced)."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    fns = [lib.spec_verify_chain_commit, lib.spec_chain_decide_commit]
+    for f in fns:
+        f.restype = I
+        f.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, I, I, I, I, P, P, ctypes.c_uint64,
+                      P, ctypes.c_uint32, P, P, P, I, I, P, P, P, P, P, I, P, P, I, I, I, P, P,
+                      P, I, P, P, ctypes.c_size_t, P]
+    fake = P(0x10000)
+    odd = P(0x10008)
+    args = [fake, 1024, fake, 1024, 0, 4, 3, 1024, fake, fake, 0, fake, 0, fake, fake, None,
+            16, 8, fake, fake, None, fake, fake, 64, fake, fake, 32, 8, 128, None, None, None, 0,
+            fake, fake, 1 << 30, None]
+    for f in fns:   # B = 0: nothing to do
+        assert f(*[0 if i == 5 else a for i, a in enumerate(args)]) == 0
+    cases = [
+        (5, 4097, -1),          # B above the fused limit
+        (6, 300, -1),           # K above the limit
+        (16, 0, -1),            # block size
+        (25, None, -1),         # K/V stage without a pool
+        ((27, 28), (1, 3), -1),  # segment (2 * heads * dim bytes) not a multiple of 16
+        (18, None, -1),         # no tables
+        (13, None, -1),         # no accept_len (the commit's kept counts)
+        (14, None, -1),         # no out_tok
+        (4, 7, -1),             # unknown dtype
+        (0, odd, -1),           # rows not 16-byte aligned
+        (34, odd, -3),          # workspace misaligned
+        (35, 64, -3),           # workspace too small
+    ]
+    for i, v, code in cases:
+        bad = list(args)
+        for j, x in zip(*((i, v) if isinstance(i, tuple) else ((i,), (v,)))):
+            bad[j] = x
+        for f in fns:
+            assert f(*bad) == code, (i, v)
+
+
 def test_draft_workspace_and_host_errors(lib):
     P = ctypes.c_void_p
     g = lib.spec_draft_workspace_bytes
