@@ -241,10 +241,8 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
  * spec_commit_paged with keep = accept_len, keep_add = 1 and Kp1 = K + 1
  * (a + 1 rows kept per sequence: the accepted drafts and the drawn token),
  * in three launches instead of four: the row statistics; one cluster per
- * sequence that runs the check and the draw, whose last sequence to finish
- * its accept test plans the commit, and which copies the sequence's kept
- * K/V rows that land in blocks it already holds; then the copy of the hidden
- * rows and of the K/V rows that need a newly allocated block.
+ * sequence for the check and the draw, whose last sequence to finish its
+ * accept test plans the commit; the copy of the kept K/V and hidden rows.
  * Arguments: those of spec_verify_chain (the logits, drafts, temperatures,
  * Philox key, accept_len, out_tok, diag, workspace) and of spec_commit_paged
  * (tables, lengths, base_len, stack, pool, stage and hidden buffers), with
@@ -254,12 +252,8 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
  * device, a sequence that fails the check (invalid temperature, draft id
  * or logits) sets SPEC_EDEVICE, accept_len = -1 and out_tok = -1 for it, and
  * then nothing is committed; a commit that fails its checks sets
- * SPEC_EINVAL or SPEC_ENOBLOCKS. In both cases no table, length, stack
- * entry, hidden row or offset changes and the verification outputs stand,
- * but -- unlike spec_commit_paged -- the pool slots of the kept rows of the
- * sequences that passed the check (positions base_len .. base_len + a), in
- * blocks those sequences already held, may hold the staged rows: they lie
- * past the committed prefix. A status already set on entry commits nothing.
+ * SPEC_EINVAL or SPEC_ENOBLOCKS and changes no table, length, stack entry,
+ * pool slot, hidden row or offset, while the verification outputs stand.
  * ------------------------------------------------------------------------- */
 int spec_verify_chain_commit(const void* tgt, int64_t ld_tgt, const void* drf,
                              int64_t ld_drf, int dtype, int B, int K, int V,

@@ -21,13 +21,13 @@ int stat_tiles(int V, int dtype) {
 }
 
 struct Layout {
-  size_t part, fin, kv_done, ticket, total;
+  size_t part, fin, ticket, total;
   long long rows;
 };
 
 // Workspace: final row statistics and tile partials for the largest row set,
-// then the per-sequence copied-row counts and the ticket of the fused
-// verify-and-commit path, each region 256-byte aligned.
+// then the ticket word of the fused verify-and-commit path, each region
+// 256-byte aligned.
 bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   if (B < 0 || K < 0 || K > SPEC_MAX_K || V < 1 || V > SPEC_MAX_V) return false;
   if (dtype != SPEC_F32 && dtype != SPEC_BF16) return false;
@@ -38,8 +38,7 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   L->rows = rows;
   L->fin = 0;
   L->part = align_up((size_t)rows * sizeof(RowFinal));
-  L->kv_done = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
-  L->ticket = L->kv_done + align_up((size_t)B * sizeof(int32_t));
+  L->ticket = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
   L->total = L->ticket + kAlign;
   return true;
 }
@@ -404,7 +403,6 @@ int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf, i
   f.d.ld_drf = ld_drf * es;
   f.d.accept_len = accept_len;
   f.d.out_tok = out_tok;
-  f.kv_done = reinterpret_cast<int32_t*>((char*)ws + ck.L.kv_done);
   f.ticket = reinterpret_cast<int32_t*>((char*)ws + ck.L.ticket);
   return cuda_status(launch_chain_fused(f, (cudaStream_t)stream));
 }

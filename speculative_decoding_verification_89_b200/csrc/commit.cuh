@@ -260,7 +260,6 @@ static __device__ void copy_body(const CommitArgs& a, int cta, int ncta, int* s_
     uint4* dst;
     int nvec;
     if (sidx < nseg) {
-      if (a.kv_done && i < a.kv_done[b]) continue;  // copied by the decide launch
       const int pos = s_len[b] - kept + i;  // base_len + i
       const int blk = a.tables[(size_t)b * a.max_blocks + pos / a.block_size];
       const int slot = pos % a.block_size;

@@ -479,17 +479,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
 // ---------------------------------------------------------------------------
 // Chain verification fused with the paged commit
 // ---------------------------------------------------------------------------
-// chain_decide_kernel's cluster per sequence, which also commits. Once its
-// accept test is done the leader writes the kept count (a + 1) and takes a
-// ticket (one atomic, never awaited): the CTA that takes the B-th ticket has
-// seen every kept count and runs the commit planner (tables, free stack,
-// lengths, hidden offsets) before its share of the residual tiles. Beside the
-// draw, every CTA copies its share of the sequence's kept K/V rows that land
-// in blocks the sequence already holds (their pool slots are known without the
-// planner: blocks below ceil(old length / block) stay, the new length being
-// at least the base); kv_done[b] records how many leading rows were copied.
-// The launch after this one copies the hidden rows and the K/V rows that need
-// a newly allocated block.
+// chain_decide_kernel's cluster per sequence, which also plans the commit.
+// Once its accept test is done the leader writes the kept count (a + 1) and
+// takes a ticket (one atomic, never awaited): the CTA that takes the B-th
+// ticket has seen every kept count and runs the commit planner (tables, free
+// stack, lengths, hidden offsets). The leader takes no residual tiles -- the
+// other kCluster - 1 CTAs sum them -- so the planner, which overlaps the
+// other sequences' draws, delays nothing but its own sequence's draw. The
+// copy launch after this one moves the kept K/V and hidden rows.
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(FusedArgs F) {
   pdl_begin();
@@ -507,11 +504,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
   const CommitArgs& cm = F.cm;
   const int b = blockIdx.y, K = c.K, V = c.V, per = 2 * K + 1;
   const int nrt = residual_tiles(V);
-  // This sequence's commit inputs, read before any CTA can take the last
-  // ticket (the planner rewrites the length).
-  const int32_t st0 = c.status ? *(volatile int32_t*)c.status : SPEC_OK;
-  const int old_len = cm.seq_lens[b];
-  const int base = cm.base_len ? cm.base_len[b] : old_len;
+  if (rank == 0) {  // the planner reads every held table entry: bring this row's into L2
+    const int old_len = max(cm.seq_lens[b], 0);
+    const int held = min((old_len + cm.block_size - 1) / cm.block_size, cm.max_blocks);
+    const int32_t* row = cm.tables + (size_t)b * cm.max_blocks;
+    for (int i = threadIdx.x * 32; i < held; i += blockDim.x * 32)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(row + i));
+  }
   const float Tb = c.temperature[b];
   const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
   double* diag = (rank == 0 && c.diag) ? c.diag + (size_t)b * (4 * K + 2) : nullptr;
@@ -576,61 +575,33 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
       plan_body(cm, reinterpret_cast<int*>(dyn + 2 * nrt));
     }
   }
-  // Residual tile sums of a sampled sequence, a quarter per CTA.
+  // Residual tile sums of a sampled sequence, split over the CTAs but the leader.
   const bool draw = !o.bad && !greedy;
   const T* prow = nullptr;
   const T* qrow = nullptr;
   ProbCoef kp{}, kq{};
+  constexpr int kWorkers = kCluster - 1;
   if (draw) {
     prow = tp(a);
     qrow = a < K ? dp(a) : nullptr;
     kp = make_coef(lsh->M[a] + lsh->L[a], sc);
     kq = make_coef(a < K ? dl(a) : 0.0, sc);
-    const int chunk = (nrt + kCluster - 1) / kCluster;
-    residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
-                          min(nrt, ((int)rank + 1) * chunk), ltsum);
+    const int chunk = (nrt + kWorkers - 1) / kWorkers, wr = (int)rank - 1;
+    if (wr >= 0)
+      residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, wr * chunk),
+                            min(nrt, (wr + 1) * chunk), ltsum);
   }
   // The tile sums are in the leader once every CTA has arrived; only the
-  // leader waits, the others go on to their copies.
+  // leader waits.
   asm volatile("barrier.cluster.arrive;" ::: "memory");
-  if (rank == 0) {
-    asm volatile("barrier.cluster.wait;" ::: "memory");
-    if (draw) {
-      double Z;
-      const int tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, o.u_draw, &Z);
-      if (threadIdx.x == 0) {
-        out[a] = tok;
-        if (diag) diag[4 * K + 1] = Z;
-      }
-    }
-  }
-  // Kept rows whose pool block the sequence already holds: i < n_early.
-  int n_early = 0;
-  if (st0 == SPEC_OK && !o.bad && cm.kv_stage && old_len >= 0 && base >= 0 && base <= old_len) {
-    const int held = min((old_len + cm.block_size - 1) / cm.block_size, cm.max_blocks);
-    n_early = max(0, min(a + 1, held * cm.block_size - base));
-  }
-  if (rank == 0 && threadIdx.x == 0) F.kv_done[b] = n_early;
-  const int nseg = cm.layers * 2, nvec = cm.seg_bytes / 16;
-  const int lane = threadIdx.x & 31, gw = (int)rank * kDecWarps + (threadIdx.x >> 5);
-  for (int item = gw; item < n_early * nseg; item += kCluster * kDecWarps) {
-    const int i = item / nseg, sidx = item - i * nseg;
-    const int pos = base + i;
-    const int blk = cm.tables[(size_t)b * cm.max_blocks + pos / cm.block_size];
-    if (blk < 0 || blk >= cm.num_blocks) continue;  // the planner refuses the call
-    const int slot = pos % cm.block_size;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        cm.kv_stage + (((size_t)b * cm.Kp1 + i) * nseg + sidx) * cm.seg_bytes);
-    uint4* dst = reinterpret_cast<uint4*>(
-        cm.kv_pool + (((size_t)blk * nseg + sidx) * cm.block_size + slot) * (size_t)cm.seg_bytes);
-    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-      uint4 r[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (v0 + 32 * u < nvec) r[u] = __ldcs(src + v0 + 32 * u);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (v0 + 32 * u < nvec) __stcs(dst + v0 + 32 * u, r[u]);
+  if (rank != 0) return;
+  asm volatile("barrier.cluster.wait;" ::: "memory");
+  if (draw) {
+    double Z;
+    const int tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, o.u_draw, &Z);
+    if (threadIdx.x == 0) {
+      out[a] = tok;
+      if (diag) diag[4 * K + 1] = Z;
     }
   }
 }
@@ -659,9 +630,7 @@ static cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   e = launch_pdl_cluster(k, dim3(kCluster, a.d.c.B), dim3(kDecThreads), smem, st, kCluster, a);
   if (e != cudaSuccess) return e;
-  CommitArgs rest = a.cm;
-  rest.kv_done = a.kv_done;
-  return launch_commit_copy(rest, st);
+  return launch_commit_copy(a.cm, st);
 }
 
 cudaError_t launch_chain_fused(const FusedArgs& a, cudaStream_t st) {

@@ -245,7 +245,6 @@ struct CommitArgs {
   int32_t* hid_off;
   int hid_bytes;                   // hidden * 2
   int32_t* status;
-  const int32_t* kv_done;          // optional [B]: leading kept rows whose K/V rows are in place
 };
 
 // The planner launch, then the copy launch; the copy launch alone.
@@ -259,11 +258,10 @@ struct FusedArgs {
   ChainDecideArgs d;
   CommitArgs cm;       // keep = d.accept_len, keep_add = 1, Kp1 = K + 1
   int32_t* ticket;     // zeroed by the row-statistics launch that precedes this call
-  int32_t* kv_done;    // [B] leading kept rows whose K/V rows the decide launch copied
 };
 
-// The decide-and-commit launch (check, draw, plan, K/V rows into held
-// blocks), then the copy of the remaining rows; the row statistics precede.
+// The decide launch that also plans the commit, then the copy launch; the
+// row statistics precede.
 cudaError_t launch_chain_fused(const FusedArgs& a, cudaStream_t st);
 
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
