@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a)
   plan_body(a, s_seq);
 }
 
-__global__ void __launch_bounds__(kCopyThreads, kCopyCtasPerSm) commit_copy_kernel(CommitArgs a) {
+__global__ void __launch_bounds__(kCopyThreads) commit_copy_kernel(CommitArgs a) {
   pdl_begin();
   extern __shared__ int s_off[];
   copy_body(a, blockIdx.x, gridDim.x, s_off);
