@@ -175,6 +175,8 @@ SMALL = [
     (2, 40, 3000, torch.bfloat16, 1.0),          # K > 32
     (3, 5, 777, torch.bfloat16, 0.0),            # all greedy
     (37, 4, 5000, torch.bfloat16, 0.9),          # more sequences than draw clusters of 4 fit
+    (300, 3, 2000, torch.float32, 1.0),          # clusters in several waves: late tickets
+    (4096, 1, 64, torch.float32, 0.8),           # the largest batch of the fused call
 ]
 
 
