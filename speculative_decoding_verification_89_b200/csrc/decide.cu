@@ -18,7 +18,9 @@
 // position, ballot for the first rejection), split the residual row pair
 // between them and write their tile sums into the leader, meet again, and the
 // leader prefixes the tile sums, finds the tile holding u' * Z, rescans that
-// one tile and writes the outputs. No atomics, no spinning, no second launch.
+// one tile and writes the outputs. No spinning and no second launch; the
+// variant that also plans a paged commit (chain_decide_commit_kernel, at the
+// end of this file) adds one atomic ticket per sequence.
 #include "draw.cuh"
 #include "commit.cuh"
 
