@@ -569,7 +569,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      s_last = atomicAdd(F.ticket, 1) == c.B - 1;
+      // The B-th ticket of this call (modulo B: a repeated call after one
+      // row-statistics launch counts on from B).
+      s_last = (atomicAdd(F.ticket, 1) + 1) % c.B == 0;
     }
     __syncthreads();
     if (s_last) {

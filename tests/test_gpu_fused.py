@@ -19,7 +19,7 @@ FIELDS = ("acc", "out", "diag", "status", "tables", "seq_lens", "free_stack", "f
           "kv_pool", "hid_out", "hid_off")
 
 
-def _run(prob, state, bufs, fused, base=None):
+def _run(prob, state, bufs, fused, base=None, status0=0):
     from speculative_decoding_verification_89_b200 import capi
     dev = "cuda"
     tgt = padded(prob.tgt.to(dev))
@@ -41,7 +41,7 @@ def _run(prob, state, bufs, fused, base=None):
     acc = torch.full((B,), -7, dtype=torch.int32, device=dev)
     out = torch.full((B, K + 1), -7, dtype=torch.int32, device=dev)
     dg = torch.full((B, 4 * K + 2), -7.0, dtype=torch.float64, device=dev)
-    s = torch.zeros(1, dtype=torch.int32, device=dev)
+    s = torch.full((1,), status0, dtype=torch.int32, device=dev)
     if fused:
         capi.spec_verify_chain_commit(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, t, l,
                                       b_len, f, top, s, ws, block_size=state.block_size,
@@ -242,3 +242,65 @@ def test_fused_failures():
     _same(fused, two, "pool2")
     _check_oracle(prob, state, bufs, fused, "pool2", tally)
     tally.check_share()
+
+
+def test_fused_pending_status_commits_nothing():
+    """A status word that already holds an error on entry: the check still
+    runs and writes its outputs, the commit changes nothing -- as for the two
+    calls."""
+    prob, state, bufs = _small_case(5, 4, 3000, torch.bfloat16, 0.9, seed=51)
+    fused = _run(prob, state, bufs, True, status0=-6)
+    two = _run(prob, state, bufs, False, status0=-6)
+    assert fused["status"] == -6
+    _same(fused, two, "pending")
+    assert torch.equal(fused["tables"], state.tables)
+    assert torch.equal(fused["seq_lens"], state.seq_lens)
+    assert torch.equal(fused["free_stack"], state.free_stack)
+    assert torch.equal(fused["kv_pool"].cpu(), bufs.kv_pool)
+    assert torch.equal(fused["hid_out"].cpu(), bufs.hid_out)
+
+
+def test_split_entry_points_repeat_after_one_row_pass():
+    """spec_chain_row_stats once, then spec_chain_decide_commit for two rounds
+    on the same rows: each round equals spec_chain_decide + spec_commit_paged
+    (the accept launch's tickets keep counting past B)."""
+    from speculative_decoding_verification_89_b200 import capi
+    dev = "cuda"
+    prob, state, bufs = _small_case(6, 3, 4000, torch.bfloat16, 1.1, seed=61, spare=24)
+    tgt, drf = padded(prob.tgt.to(dev)), padded(prob.drf.to(dev))
+    dt, T, sid = prob.draft_tok.to(dev), prob.temperature.to(dev), prob.seq_id.to(dev)
+    B, K, V = 6, 3, 4000
+    res = []
+    for fused in (True, False):
+        st = state.clone()
+        t, l, f, top = (st.tables.to(dev), st.seq_lens.to(dev), st.free_stack.to(dev),
+                        st.free_top.to(dev))
+        pool, hout, hoff = bufs.kv_pool.clone().to(dev), bufs.hid_out.clone().to(dev), \
+            bufs.hid_off.clone().to(dev)
+        kw = dict(kv_stage=bufs.kv_stage.to(dev), kv_pool=pool, hid_stage=bufs.hid_stage.to(dev),
+                  hid_out=hout, hid_off=hoff)
+        ws = capi.workspace(B, K, V, tgt.dtype, device=dev)
+        s = torch.zeros(1, dtype=torch.int32, device=dev)
+        capi.spec_chain_row_stats(tgt, drf, T, s, ws)
+        outs = []
+        for rnd in (7, 8):
+            acc = torch.empty(B, dtype=torch.int32, device=dev)
+            out = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+            if fused:
+                capi.spec_chain_decide_commit(tgt, drf, dt, T, prob.seed, sid, rnd, acc, out, t, l,
+                                              None, f, top, s, ws, block_size=state.block_size,
+                                              **kw)
+            else:
+                capi.spec_chain_decide(tgt, drf, dt, T, prob.seed, sid, rnd, acc, out, s, ws)
+                capi.spec_commit_paged(t, l, None, acc, 1, f, top, K + 1, s,
+                                       block_size=state.block_size, **kw)
+            torch.cuda.synchronize()
+            outs.append((acc.cpu(), out.cpu(), t.cpu().clone(), l.cpu().clone(),
+                         top.cpu().clone(), hoff.cpu().clone()))
+        res.append((outs, pool.cpu(), hout.cpu(), int(s.item())))
+    assert res[0][3] == res[1][3]
+    for (a, b) in zip(res[0][0], res[1][0]):
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
+    assert torch.equal(res[0][1].view(torch.int16), res[1][1].view(torch.int16))
+    assert torch.equal(res[0][2].view(torch.int16), res[1][2].view(torch.int16))
