@@ -82,7 +82,8 @@ CASES = [
     (8, 32000, torch.bfloat16, 0.7, {"mask_frac": 0.3}),   # masked entries
     (4, 50000, torch.float32, 1e-3, {}),                   # near-greedy
     (4, 50000, torch.bfloat16, 50.0, {}),                  # flat laws
-    (6, 151936, torch.float32, 1.0, {"zipf_s": 1.1}),      # Qwen-size fp32 rows
+    (6, 151936, torch.float32, 1.0, {"zipf_s": 1.1}),      # Qwen-size fp32 rows (8-CTA slices)
+    (2, 262144, torch.float32, 0.9, {}),                   # too large to stage: two launches
 ]
 
 
