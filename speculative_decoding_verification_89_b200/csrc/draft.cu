@@ -9,12 +9,18 @@
 // mind-verse.de, SVIP paragraphs), from which a draft-length policy decides
 // whether to keep drafting.
 //
-// Two launches: the row-statistics kernel over the B rows (DraftRows, which
-// also gathers the first moment sum 2^(l*c - M) * (l - m)), then one
-// thread-block cluster per sequence that combines its row, and -- unless the
-// sequence is greedy -- splits the row's 256-element tiles of p over the
-// cluster, prefixes their sums in the leader and draws by inverse CDF with the
-// lane-1 uniform of the Philox counter (seq_id, round, pos, 0).
+// One launch when a cluster of 4 (or 8) CTAs can hold a row in shared memory
+// (draft_fused_kernel: every logit read from HBM once, statistics and draw
+// from shared memory). Larger rows take two launches: the row-statistics
+// kernel over the B rows (DraftRows, which also gathers the first moment sum
+// 2^(l*c - M) * (l - m)), then one thread-block cluster per sequence that
+// combines its row, and -- unless the sequence is greedy -- splits the row's
+// 256-element tiles of p over the cluster, prefixes their sums in the leader
+// and draws. Either way the draw is by inverse CDF with the lane-1 uniform of
+// the Philox counter (seq_id, round, pos, 0).
+#include <cfloat>
+#include <climits>
+
 #include "draw.cuh"
 
 namespace specv {
@@ -129,6 +135,275 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
   }
 }
 
+// ---------------------------------------------------------------------------
+// One launch for rows that fit the cluster's shared memory
+// ---------------------------------------------------------------------------
+// A cluster of cs CTAs per row. CTA r stages its slice of the row -- whole
+// 256-element tiles [r*tc, (r+1)*tc) -- in shared memory with bulk copies, so
+// the row is read from HBM once, and finds its largest logit m_r with its
+// first index, then per tile the sum of 2^(x*c - M_r) with its own exact
+// shift M_r = fl(m_r * c_hi), and the first moment sum 2^(x*c - M_r) (x - m_r).
+// Every CTA sends (m_r, argmax, S_r, T_r) to every other CTA of the cluster
+// (distributed shared memory); after a cluster barrier each combines them in
+// the same order -- the row's max and shift M, partition, entropy and the draw
+// target u * S -- and the CTA whose slice holds the target prefixes its tile
+// sums and rescans one tile in shared memory for the token. Results equal the
+// two-launch path's up to the summation order of the partition.
+constexpr int kDfMaxCluster = 8;
+constexpr int kDfSliceBytes = 100 * 1024;  // staged slice per CTA, at most
+constexpr uint32_t kDfChunk = 32768;        // bytes per bulk copy
+
+struct DfPart {
+  float m;
+  int amax;
+  double S, T;
+};
+
+// One staged element (shared memory: plain loads, not the read-only path).
+__device__ __forceinline__ float smem_elem(const float* p) { return *p; }
+__device__ __forceinline__ float smem_elem(const __nv_bfloat16* p) {
+  return __uint_as_float(((unsigned)*reinterpret_cast<const unsigned short*>(p)) << 16);
+}
+template <typename T>
+__device__ __forceinline__ void smem8(const T* xs, int i0, int n, float x[8]) {
+  if (i0 + 8 <= n) {
+    Raw8<T> r;
+    const uint4* p = reinterpret_cast<const uint4*>(xs + i0);
+#pragma unroll
+    for (int k = 0; k < (int)(sizeof(T) / 2); ++k) r.v[k] = p[k];
+    unpack8(r, x);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = i0 + e < n ? smem_elem(xs + i0 + e) : -INFINITY;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A, int tc) {
+  pdl_begin();
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");  // waited before remote writes
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank(), cs = (int)cl.num_blocks();
+  extern __shared__ __align__(128) unsigned char dsm[];
+  T* xs = reinterpret_cast<T*>(dsm);
+  double* tsum = reinterpret_cast<double*>(dsm + (size_t)tc * kResTile * sizeof(T));
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ DfPart s_part[kDfMaxCluster];
+  __shared__ float s_wm[kDecWarps];
+  __shared__ int s_wi[kDecWarps];
+  __shared__ double s_ws[kDecWarps], s_wt[kDecWarps];
+  const int b = blockIdx.y, V = A.V, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nrt = residual_tiles(V);
+  const int t0 = min(nrt, rank * tc), t1 = min(nrt, t0 + tc), nt = t1 - t0;
+  const int e0 = t0 * kResTile, n = max(0, min(V, t1 * kResTile) - e0);
+  const float Tb = A.temperature[b];
+  const bool greedy = (Tb == 0.0f);
+  const T* row = row_ptr<T>(A.lg, A.ld, b);
+  auto finish = [&](int tok, double logq, double H, bool bad) {
+    if (bad) set_status(A.status, SPEC_EDEVICE);
+    A.out_tok[b] = bad ? -1 : tok;
+    if (A.out_logq) A.out_logq[b] = bad ? dnan() : logq;
+    if (A.out_entropy) A.out_entropy[b] = bad ? dnan() : H;
+  };
+  if (!temp_valid(Tb)) {  // the same verdict in every CTA of the cluster
+    if (rank == 0 && threadIdx.x == 0) finish(-1, 0.0, 0.0, true);
+    return;
+  }
+  const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+
+  // Stage the slice: bulk copies of its 16-byte part, plain loads of the rest.
+  const uint32_t bytes = ((uint32_t)n * (uint32_t)sizeof(T)) & ~15u;
+  const int nbulk = (int)(bytes / sizeof(T));
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && bytes) {
+    mbar_arrive_expect_tx(&s_bar, bytes);
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(row + e0);
+    for (uint32_t o = 0; o < bytes; o += kDfChunk)
+      bulk_g2s(dsm + o, src + o, min(kDfChunk, bytes - o), &s_bar);
+  }
+  for (int i = nbulk + (int)threadIdx.x; i < n; i += blockDim.x) xs[i] = row[e0 + i];
+  if (bytes && !mbar_wait_bounded(&s_bar, 0, kWaitLimitNs)) {
+    set_status(A.status, SPEC_ETIMEOUT);
+    mbar_wait_bounded(&s_bar, 0, kWaitLimitNs);  // let the copies land before going on
+  }
+  __syncthreads();
+
+  // Largest logit of the slice and its first index.
+  float mv = -INFINITY;
+  int mi = 0x7fffffff;
+  for (int i0 = (int)threadIdx.x * 8; i0 < n; i0 += blockDim.x * 8) {
+    float x[8];
+    smem8(xs, i0, n, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (x[e] > mv) { mv = x[e]; mi = e0 + i0 + e; }
+  }
+  warp_argmax(mv, mi);
+  if (lane == 0) { s_wm[warp] = mv; s_wi[warp] = mi; }
+  __syncthreads();
+  float m_r = -INFINITY;
+  int a_r = 0x7fffffff;
+  for (int w = 0; w < kDecWarps; ++w)
+    if (s_wm[w] > m_r || (s_wm[w] == m_r && s_wi[w] < a_r)) { m_r = s_wm[w]; a_r = s_wi[w]; }
+
+  // Tile sums of 2^(x*c - M_r) and the first moment about m_r.
+  double S_r = 0.0, T_r = 0.0;
+  const bool fin = m_r > -INFINITY && m_r < INFINITY;
+  if (!greedy && fin) {
+    const float Mr = __fmul_rn(m_r, sc.hi);
+    const ProbCoef kr = make_coef((double)Mr, sc);
+    double ws = 0.0, wt = 0.0;
+    for (int t = warp; t < nt; t += kDecWarps) {
+      float x[8], w[8];
+      smem8(xs, t * kResTile + lane * 8, n, x);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float2 pr = prob2(make_float2(x[e], x[e + 1]), kr);
+        w[e] = pr.x;
+        w[e + 1] = pr.y;
+      }
+      float mom = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mom += w[e] * fmaxf(x[e] - m_r, -FLT_MAX);
+      const double st = warp_sum_d(lane_sum8(w));
+      if (lane == 0) tsum[t] = st;
+      ws += st;
+      wt += (double)mom;
+    }
+    wt = warp_sum_d(wt);
+    if (lane == 0) { s_ws[warp] = ws; s_wt[warp] = wt; }
+    __syncthreads();
+    for (int w = 0; w < kDecWarps; ++w) { S_r += s_ws[w]; T_r += s_wt[w]; }
+  }
+
+  // Every CTA's summary to every CTA, then the same combine everywhere.
+  asm volatile("barrier.cluster.wait;" ::: "memory");
+  if (threadIdx.x < cs) {
+    DfPart* dst = cl.map_shared_rank(s_part, (unsigned)threadIdx.x);
+    dst[rank] = DfPart{m_r, a_r, S_r, T_r};
+  }
+  cl.sync();
+  float m = -INFINITY;
+  int amax = 0x7fffffff;
+  for (int r = 0; r < cs; ++r)
+    if (s_part[r].m > m || (s_part[r].m == m && s_part[r].amax < amax)) {
+      m = s_part[r].m;
+      amax = s_part[r].amax;
+    }
+  const bool ok = m > -INFINITY && m < INFINITY;
+  if (!ok || greedy) {
+    if (rank == 0 && threadIdx.x == 0) finish(amax, 0.0, 0.0, !ok);
+    return;
+  }
+  const double M = (double)__fmul_rn(m, sc.hi);
+  double S = 0.0, Tm = 0.0;
+  for (int r = 0; r < cs; ++r) {
+    if (s_part[r].S > 0.0) {
+      const float mr = s_part[r].m;
+      const double f = exp2((double)__fmul_rn(mr, sc.hi) - M);
+      S += s_part[r].S * f;
+      Tm += (s_part[r].T + ((double)mr - (double)m) * s_part[r].S) * f;
+    }
+  }
+  const double Lt = M + log2(S);
+  const double Mcm = (M - (double)m * (double)sc.hi) - (double)m * (double)sc.lo;
+  const double H = kLn2 * (Mcm + log2(S) - sc.d * (Tm / S));
+  const float u = spec_uniforms(A.seed, (uint32_t)A.seq_id[b], A.round, (uint32_t)A.pos[b], 0u).y;
+  const double target = (double)u * S;
+  // The CTA whose slice holds the target: the first whose running total passes it.
+  int owner = -1;
+  double local = 0.0, cum = 0.0;
+  for (int r = 0; r < cs; ++r) {
+    if (s_part[r].S > 0.0) {
+      const double f = exp2((double)__fmul_rn(s_part[r].m, sc.hi) - M);
+      const double c_r = s_part[r].S * f;
+      owner = r;  // the last with mass, if rounding leaves the target past the end
+      local = (target - cum) / f;
+      if (cum + c_r > target) break;
+      cum += c_r;
+    }
+  }
+  if (owner < 0) {  // no mass anywhere: cannot happen for a row with a finite maximum
+    if (rank == 0 && threadIdx.x == 0) finish(-1, 0.0, 0.0, true);
+    return;
+  }
+  if (rank != owner) return;
+
+  // Owner: the tile (warp 0 prefixes the tile sums: a contiguous run per
+  // lane, then a scan over the lanes), then the element.
+  if (warp == 0) {
+    const int per = (nt + 31) / 32;
+    const int a0 = min(nt, lane * per), a1 = min(nt, a0 + per);
+    double run = 0.0;
+    for (int t = a0; t < a1; ++t) run += tsum[t];
+    double incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    // The last tile with mass whose prefix does not pass the target.
+    double c = incl - run, c_cand = 0.0;
+    int cand = -1;
+    for (int t = a0; t < a1; ++t) {
+      if (c <= local && tsum[t] > 0.0) { cand = t; c_cand = c; }
+      c += tsum[t];
+    }
+    int best = cand;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    const int tile = best < 0 ? 0 : best;
+    const unsigned holder = __ballot_sync(0xffffffffu, cand == best && best >= 0);
+    const double pre = holder ? __shfl_sync(0xffffffffu, c_cand, __ffs(holder) - 1) : 0.0;
+    const float Mr = __fmul_rn(s_part[owner].m, sc.hi);
+    const ProbCoef kr = make_coef((double)Mr, sc);
+    float x[8], w[8];
+    smem8(xs, tile * kResTile + lane * 8, n, x);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float2 pr = prob2(make_float2(x[e], x[e + 1]), kr);
+      w[e] = pr.x;
+      w[e + 1] = pr.y;
+    }
+    const double ls = lane_sum8(w);
+    double li = ls;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, li, o);
+      if (lane >= o) li += y;
+    }
+    const double start = pre + (li - ls);
+    int found = INT_MAX;
+    if (start <= local) {
+      double acc = start;
+      for (int e = 0; e < 8; ++e) {
+        acc += (double)w[e];
+        if (acc > local && w[e] > 0.0f) { found = tile * kResTile + lane * 8 + e; break; }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) found = min(found, __shfl_xor_sync(0xffffffffu, found, o));
+    if (found == INT_MAX) {  // the target sits at the tile's end by rounding
+      int last = -1;
+      for (int e = 7; e >= 0; --e)
+        if (w[e] > 0.0f) { last = tile * kResTile + lane * 8 + e; break; }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+      found = last;
+    }
+    if (lane == 0) {
+      const bool bad = found < 0 || found >= n;
+      const int tok = bad ? -1 : e0 + found;
+      const double logq = bad ? 0.0 : kLn2 * ((double)smem_elem(xs + found) * sc.d - Lt);
+      finish(tok, logq, H, bad);
+    }
+  }
+}
+
 template <typename T>
 static cudaError_t launch_draw(const DraftArgs& a, cudaStream_t st) {
   auto k = draft_draw_kernel<T>;
@@ -138,11 +413,43 @@ static cudaError_t launch_draw(const DraftArgs& a, cudaStream_t st) {
   return launch_pdl_cluster(k, dim3(kCluster, a.B), dim3(kDecThreads), smem, st, kCluster, a);
 }
 
+template <typename T>
+static cudaError_t launch_fused_draw(const DraftArgs& a, int cs, int tc, cudaStream_t st) {
+  auto k = draft_fused_kernel<T>;
+  const size_t smem = (size_t)tc * kResTile * sizeof(T) + (size_t)tc * sizeof(double);
+  const cudaError_t e = reserve_dyn_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl_cluster(k, dim3(cs, a.B), dim3(kDecThreads), smem, st, (unsigned)cs, a, tc);
+}
+
 cudaError_t launch_draft_step(int dtype, const unsigned char* lg, long long ld_bytes, int B, int V,
                               const float* temperature, uint64_t seed, const int32_t* seq_id,
                               uint32_t round, const int32_t* pos, Partial* part, double* mom,
                               int32_t* out_tok, double* out_logq, double* out_entropy,
                               int32_t* status, cudaStream_t st) {
+  // One launch when a cluster of 4 (or 8) CTAs holds the row in shared memory.
+  const int esz = dtype == SPEC_BF16 ? 2 : 4, nrt = residual_tiles(V);
+  for (int cs = 4; cs <= kDfMaxCluster; cs *= 2) {
+    const int tc = (nrt + cs - 1) / cs;
+    if ((size_t)tc * kResTile * esz + (size_t)tc * sizeof(double) > (size_t)kDfSliceBytes) continue;
+    DraftArgs a{};
+    a.B = B;
+    a.V = V;
+    a.lg = lg;
+    a.ld = ld_bytes;
+    a.temperature = temperature;
+    a.seed = seed;
+    a.seq_id = seq_id;
+    a.round = round;
+    a.pos = pos;
+    a.out_tok = out_tok;
+    a.out_logq = out_logq;
+    a.out_entropy = out_entropy;
+    a.status = status;
+    return dtype == SPEC_BF16 ? launch_fused_draw<__nv_bfloat16>(a, cs, tc, st)
+                              : launch_fused_draw<float>(a, cs, tc, st);
+  }
+  // Larger rows: the row statistics, then the draw re-reading one row.
   DraftRows rows;
   rows.lg = lg;
   rows.ld = ld_bytes;
