@@ -232,15 +232,24 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
   }
   __syncthreads();
 
-  // Largest logit of the slice and its first index.
+  // Largest logit of the slice, and for a greedy row its first index.
   float mv = -INFINITY;
   int mi = 0x7fffffff;
-  for (int i0 = (int)threadIdx.x * 8; i0 < n; i0 += blockDim.x * 8) {
-    float x[8];
-    smem8(xs, i0, n, x);
+  if (greedy) {
+    for (int i0 = (int)threadIdx.x * 8; i0 < n; i0 += blockDim.x * 8) {
+      float x[8];
+      smem8(xs, i0, n, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (x[e] > mv) { mv = x[e]; mi = e0 + i0 + e; }
+      for (int e = 0; e < 8; ++e)
+        if (x[e] > mv) { mv = x[e]; mi = e0 + i0 + e; }
+    }
+  } else {
+    for (int i0 = (int)threadIdx.x * 8; i0 < n; i0 += blockDim.x * 8) {
+      float x[8];
+      smem8(xs, i0, n, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mv = fmaxf(mv, x[e]);
+    }
   }
   warp_argmax(mv, mi);
   if (lane == 0) { s_wm[warp] = mv; s_wi[warp] = mi; }
@@ -269,12 +278,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
       float mom = 0.0f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) mom += w[e] * fmaxf(x[e] - m_r, -FLT_MAX);
-      const double st = warp_sum_d(lane_sum8(w));
-      if (lane == 0) tsum[t] = st;
-      ws += st;
+      float ls = (float)lane_sum8(w);  // fp32 over the tile: values <= 1, 256 terms
+#pragma unroll
+      for (int o = 16; o; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+      if (lane == 0) tsum[t] = (double)ls;
+      ws += (double)ls;
       wt += (double)mom;
     }
-    wt = warp_sum_d(wt);
+    wt = warp_sum_d(wt);  // ws is the same in every lane
     if (lane == 0) { s_ws[warp] = ws; s_wt[warp] = wt; }
     __syncthreads();
     for (int w = 0; w < kDecWarps; ++w) { S_r += s_ws[w]; T_r += s_wt[w]; }
@@ -287,46 +298,63 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     dst[rank] = DfPart{m_r, a_r, S_r, T_r};
   }
   cl.sync();
-  float m = -INFINITY;
-  int amax = 0x7fffffff;
-  for (int r = 0; r < cs; ++r)
-    if (s_part[r].m > m || (s_part[r].m == m && s_part[r].amax < amax)) {
-      m = s_part[r].m;
-      amax = s_part[r].amax;
+  // The combine, by one thread (the same arithmetic in every CTA).
+  __shared__ float s_m;
+  __shared__ int s_amax, s_owner;
+  __shared__ double s_Lt, s_H, s_local;
+  if (threadIdx.x == 0) {
+    float m = -INFINITY;
+    int amax = 0x7fffffff;
+    for (int r = 0; r < cs; ++r)
+      if (s_part[r].m > m || (s_part[r].m == m && s_part[r].amax < amax)) {
+        m = s_part[r].m;
+        amax = s_part[r].amax;
+      }
+    s_m = m;
+    s_amax = amax;
+    s_owner = -1;
+    const bool ok = m > -INFINITY && m < INFINITY;
+    if (ok && !greedy) {
+      const double M = (double)__fmul_rn(m, sc.hi);
+      double f[kDfMaxCluster];
+      double S = 0.0, Tm = 0.0;
+      for (int r = 0; r < cs; ++r) {
+        f[r] = 0.0;
+        if (s_part[r].S > 0.0) {
+          const float mr = s_part[r].m;
+          f[r] = exp2((double)__fmul_rn(mr, sc.hi) - M);
+          S += s_part[r].S * f[r];
+          Tm += (s_part[r].T + ((double)mr - (double)m) * s_part[r].S) * f[r];
+        }
+      }
+      const double Mcm = (M - (double)m * (double)sc.hi) - (double)m * (double)sc.lo;
+      s_Lt = M + log2(S);
+      s_H = kLn2 * (Mcm + log2(S) - sc.d * (Tm / S));
+      const float u =
+          spec_uniforms(A.seed, (uint32_t)A.seq_id[b], A.round, (uint32_t)A.pos[b], 0u).y;
+      const double target = (double)u * S;
+      // The CTA whose slice holds the target: the first whose running total passes it.
+      double cum = 0.0;
+      for (int r = 0; r < cs; ++r) {
+        if (s_part[r].S > 0.0) {
+          const double c_r = s_part[r].S * f[r];
+          s_owner = r;  // the last with mass, if rounding leaves the target past the end
+          s_local = (target - cum) / f[r];
+          if (cum + c_r > target) break;
+          cum += c_r;
+        }
+      }
     }
+  }
+  __syncthreads();
+  const float m = s_m;
+  const int amax = s_amax, owner = s_owner;
   const bool ok = m > -INFINITY && m < INFINITY;
   if (!ok || greedy) {
     if (rank == 0 && threadIdx.x == 0) finish(amax, 0.0, 0.0, !ok);
     return;
   }
-  const double M = (double)__fmul_rn(m, sc.hi);
-  double S = 0.0, Tm = 0.0;
-  for (int r = 0; r < cs; ++r) {
-    if (s_part[r].S > 0.0) {
-      const float mr = s_part[r].m;
-      const double f = exp2((double)__fmul_rn(mr, sc.hi) - M);
-      S += s_part[r].S * f;
-      Tm += (s_part[r].T + ((double)mr - (double)m) * s_part[r].S) * f;
-    }
-  }
-  const double Lt = M + log2(S);
-  const double Mcm = (M - (double)m * (double)sc.hi) - (double)m * (double)sc.lo;
-  const double H = kLn2 * (Mcm + log2(S) - sc.d * (Tm / S));
-  const float u = spec_uniforms(A.seed, (uint32_t)A.seq_id[b], A.round, (uint32_t)A.pos[b], 0u).y;
-  const double target = (double)u * S;
-  // The CTA whose slice holds the target: the first whose running total passes it.
-  int owner = -1;
-  double local = 0.0, cum = 0.0;
-  for (int r = 0; r < cs; ++r) {
-    if (s_part[r].S > 0.0) {
-      const double f = exp2((double)__fmul_rn(s_part[r].m, sc.hi) - M);
-      const double c_r = s_part[r].S * f;
-      owner = r;  // the last with mass, if rounding leaves the target past the end
-      local = (target - cum) / f;
-      if (cum + c_r > target) break;
-      cum += c_r;
-    }
-  }
+  const double Lt = s_Lt, H = s_H, local = s_local;
   if (owner < 0) {  // no mass anywhere: cannot happen for a row with a finite maximum
     if (rank == 0 && threadIdx.x == 0) finish(-1, 0.0, 0.0, true);
     return;
