@@ -314,7 +314,7 @@ int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf,
  * ws, ws_bytes: spec_draft_workspace_bytes(B, V, dtype) bytes, 256-byte
  *               aligned. No initial contents are needed.
  * One launch when a row fits the shared memory of a cluster of 8 CTAs
- * (V * element size up to 800 KiB; the workspace is then unused), else two.
+ * (V * element size up to about 790 KiB; the workspace is then unused), else two.
  * ------------------------------------------------------------------------- */
 size_t spec_draft_workspace_bytes(int B, int V, int dtype);
 int spec_draft_sample(const void* logits, int64_t ld, int dtype, int B, int V,
