@@ -58,7 +58,34 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--plan-only", action="store_true",
+                    help="print each rank's device and sequence assignment (gloo, no GPU work)")
     return ap.parse_args()
+
+
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch(args):
+    """`--gpus N` with N > 1 outside a launcher: run this script again as N
+    ranks (one process per GPU) under torch.distributed.run on this node,
+    bounded by a timeout, and return its exit status."""
+    cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run",
+           "--nnodes=1", f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def rank_plan(dist):
+    """What rank `dist.rank` works on: its own GPU (LOCAL_RANK), its own B
+    sequences (ids B*rank ..), its own logits and block pool (seeds)."""
+    return {"rank": dist.rank, "world": dist.world, "device": dist.local,
+            "seq_id_base": B * dist.rank, "logit_seed": 2 + 1000 * dist.rank,
+            "pool_seed": 2 + dist.rank}
 
 
 # ----------------------------------------------------------------------------
@@ -247,11 +274,12 @@ def run_ours(args, dist):
     from speculative_decoding_verification_89_b200 import capi
     from speculative_decoding_verification_89_b200 import workloads as W
 
-    dev = torch.device("cuda", dist.local)
+    plan = rank_plan(dist)
+    dev = torch.device("cuda", plan["device"])
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    prob = W.chain_batch(device=dev, seed=2 + 1000 * dist.rank, seq_id_base=B * dist.rank)
-    state, bufs = W.commit_setup(B, K, device=dev, seed=2 + dist.rank)
+    prob = W.chain_batch(device=dev, seed=plan["logit_seed"], seq_id_base=plan["seq_id_base"])
+    state, bufs = W.commit_setup(B, K, device=dev, seed=plan["pool_seed"])
     base = state.seq_lens.clone()
     total = args.warmup + args.steps
     hist = torch.zeros((total, B), dtype=torch.int32, device=dev)
@@ -630,7 +658,22 @@ def run_reference(args, dist):
 
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(args)
     dist = Dist()
+    if dist.world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={dist.world}; running "
+              f"{dist.world} rank(s)", file=sys.stderr)
+    if args.plan_only:
+        dist.init("gloo")
+        plans = [rank_plan(dist)]
+        if dist.pg:
+            plans = [None] * dist.world
+            dist.pg.all_gather_object(plans, rank_plan(dist))
+        if dist.rank == 0:
+            print(json.dumps({"plans": plans}), flush=True)
+        dist.close()
+        return 0
     if args.impl == "reference":
         if dist.rank == 0:
             print(json.dumps(run_reference(args, dist)), flush=True)

@@ -371,8 +371,12 @@ int spec_outcome_law(const void* tgt, int64_t ld_tgt, const void* drf,
  * process exits. It calls no allocating routine.
  *   - Sizes whose workspace (spec_workspace_bytes(B, K, V, dtype, 0)) would
  *     exceed the array return SPEC_EWORKSPACE and launch nothing.
- *   - The first call on a device looks the array's device address up with
- *     that device current; make that first call outside any stream capture.
+ *   - A call looks the array's device address up with the device current
+ *     (cudaGetSymbolAddress) and keeps it per device and CUDA context, so the
+ *     lookup runs on the first call on a device (and again only after that
+ *     device's context was destroyed and re-created); make that first call
+ *     outside any stream capture. A failed lookup returns SPEC_ECUDA (text
+ *     from spec_last_cuda_error) and is not kept: the next call retries.
  *   - All calls share the one array and it keeps the previous call's
  *     contents (no call reads what an earlier one left). Calls that overlap
  *     on the GPU (several streams or threads) race on it and must not be made.
@@ -384,6 +388,12 @@ int spec_verify_chain_noalloc(const void* tgt, int64_t ld_tgt, const void* drf,
                               uint64_t seed, const int32_t* seq_id, uint32_t round,
                               int32_t* accept_len, int32_t* out_tok, double* diag,
                               int32_t* dev_status, void* stream);
+
+/* Test hook of spec_verify_chain_noalloc (no counterpart in the paper):
+ * forgets every kept scratch address and makes the next n address lookups
+ * fail as a lookup inside a stream capture does (SPEC_ECUDA), so a test can
+ * check that a failed lookup does not stay cached. n >= 0; 0 ends it. */
+int spec_noalloc_test_fail_lookups(int n);
 
 /* Diagnostic: text of the last CUDA error behind a SPEC_ECUDA return on the
  * calling thread ("no error" if none). Static storage. */

@@ -5,17 +5,20 @@ bf16, Zipf prior, T=1) on B sequences, and optionally the paged commit that
 follows it, `--iters` times. B=32 keeps the logits (140 MB) above the L2 size
 while the whole case stays well under a few GB of device memory.
 
-    python -m speculative_decoding_verification_89_b200.profile_case --B 32
-    python -m speculative_decoding_verification_89_b200.profile_case --B 64 --commit
+    python profile_case.py --B 32
+    python profile_case.py --B 64 --commit
 """
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import torch
 
-from . import capi
-from . import workloads as W
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+from speculative_decoding_verification_89_b200 import capi  # noqa: E402
+from speculative_decoding_verification_89_b200 import workloads as W  # noqa: E402
 
 
 def main():

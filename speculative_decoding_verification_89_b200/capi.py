@@ -52,6 +52,7 @@ _SIGS = {
     "spec_last_cuda_error": (ctypes.c_char_p, []),
     "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
                                        _u32, _p, _p, _p, _p, _p]),
+    "spec_noalloc_test_fail_lookups": (_i, [_i]),
     "spec_draft_workspace_bytes": (_sz, [_i, _i, _i]),
     "spec_outcome_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spec_outcome_law": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p,

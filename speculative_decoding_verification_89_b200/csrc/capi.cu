@@ -140,6 +140,10 @@ DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_to
 
 }  // namespace
 
+// The recorder behind every SPEC_ECUDA return of the library (other sources
+// of the library return through it too, so spec_last_cuda_error names it).
+int specv::record_cuda_status(cudaError_t e) { return cuda_status(e); }
+
 // Host checks of a paged commit's arguments; fills *out. SPEC_OK with B == 0
 // means nothing to do.
 static int commit_args(int B, int block_size, int max_blocks, int32_t* block_tables,
@@ -219,15 +223,21 @@ const char* spec_status_string(int status) {
 // the draw that follows finds them in L2: as many (at most 2) as fit in 60%
 // of the L2 with rows_per_pos rows per position and sequence.
 static int late_positions(int B, int V, int dtype, int rows_per_pos) {
-  static int l2 = -1;  // bytes; the same on every device of a B200 node
-  if (l2 < 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
+  static int l2s[kMaxDevs];  // bytes per device, looked up once per device (0: unknown)
+  static bool known[kMaxDevs];
+  const int dev = current_device();
+  int l2 = 0;
+  if (dev >= 0 && dev < kMaxDevs && known[dev]) {
+    l2 = l2s[dev];
+  } else {
+    if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
       cudaGetLastError();
-      v = 0;
+      l2 = 0;
     }
-    l2 = v;
+    if (dev >= 0 && dev < kMaxDevs) {
+      l2s[dev] = l2;
+      known[dev] = true;
+    }
   }
   const double per_pos = (double)B * rows_per_pos * V * elem_size(dtype);
   const int n = per_pos > 0.0 ? (int)(0.6 * l2 / per_pos) : 0;

@@ -71,10 +71,17 @@ static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
   int* s_kept = s_seq + 2 * a.B;
   __shared__ int s_push[kPushCache];
   __shared__ int s_stack[kStackCache];
-  __shared__ int s_bad, s_sbad, s_code, s_ft;
-  // The status word is read with the per-sequence inputs, not before them.
-  const int32_t st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
-  if (threadIdx.x == 0) { s_bad = 0; s_sbad = 0; s_code = 0; s_ft = *a.free_top; }
+  __shared__ int s_bad, s_sbad, s_code, s_ft, s_st0;
+  // One thread reads the status word (with the per-sequence inputs, not
+  // before them) and the block acts on that one value, so the early return
+  // below is taken by every thread or by none.
+  if (threadIdx.x == 0) {
+    s_st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
+    s_bad = 0;
+    s_sbad = 0;
+    s_code = 0;
+    s_ft = *a.free_top;
+  }
   const int bs = a.block_size;
   // Each thread owns a contiguous run of sequences (sequence order matters
   // for the allocation order).
@@ -104,7 +111,8 @@ static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
     cnt.z += kept;
     cnt.w += held;
   }
-  if (st0 != SPEC_OK) return;  // sticky error: the same in every thread
+  __syncthreads();  // publishes s_st0
+  if (s_st0 != SPEC_OK) return;  // sticky error: one value for every thread
   if (bad) atomicOr(&s_bad, 1);
   int4 tot;
   const int4 pre = block_excl_scan4(cnt, &tot);  // its barriers also publish s_ft, s_bad
@@ -217,8 +225,10 @@ static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
 static __device__ void copy_body(const CommitArgs& a, int cta, int ncta, int* s_off) {
   // [B + 1] exclusive scan of kept rows, then [B] new lengths
   int* s_len = s_off + a.B + 1;
-  // The status word is read with the counts, and checked once they are in.
-  const int32_t st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
+  // The status word is read (by one thread) with the counts, and checked by
+  // every thread on that one value once they are in.
+  __shared__ int s_st0;
+  if (threadIdx.x == 0) s_st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int b = (int)threadIdx.x - 32; b >= 0 && b < a.B; b += blockDim.x - 32)
     s_len[b] = a.seq_lens[b];  // the other warps, while warp 0 scans
@@ -239,7 +249,7 @@ static __device__ void copy_body(const CommitArgs& a, int cta, int ncta, int* s_
     if (lane == 0) s_off[a.B] = carry;
   }
   __syncthreads();
-  if (st0 != SPEC_OK) return;  // sticky error: the same in every thread
+  if (s_st0 != SPEC_OK) return;  // sticky error: one value for every thread
   const int KT = s_off[a.B];
   const int nseg = a.kv_stage ? a.layers * 2 : 0;
   const int piece = a.kv_stage ? a.seg_bytes : 2048;

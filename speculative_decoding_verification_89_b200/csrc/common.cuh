@@ -234,35 +234,51 @@ __device__ __forceinline__ void pdl_begin() {
   grid_dependents_launch();
 }
 
-// Streaming multiprocessors of the current device (148 on a B200), looked up
-// once per process.
-static inline int sm_count() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-      cudaGetLastError();
-      v = 0;
-    }
-    sms = v > 0 ? v : 148;
+// Device index of the calling thread (0 if the runtime cannot say).
+static inline int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
   }
-  return sms;
+  return dev;
+}
+constexpr int kMaxDevs = 64;  // per-device host caches
+
+// Streaming multiprocessors of the current device (148 on a B200), looked up
+// once per device.
+static inline int sm_count() {
+  static int sms[kMaxDevs];
+  const int dev = current_device();
+  int* slot = (dev >= 0 && dev < kMaxDevs) ? &sms[dev] : nullptr;
+  if (slot && *slot > 0) return *slot;
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    v = 0;
+  }
+  v = v > 0 ? v : 148;
+  if (slot) *slot = v;
+  return v;
 }
 
-// Lets kernel `fn` launch with `bytes` of dynamic shared memory: a kernel
-// whose static plus dynamic shared memory passes 48 KB needs the opt-in. The
-// largest size granted so far is kept per kernel, so the attribute is set
-// only when a launch needs more than before (and never lowered under a
-// concurrent caller).
+// Lets kernel `fn` launch with `bytes` of dynamic shared memory on the
+// current device: a kernel whose static plus dynamic shared memory passes
+// 48 KB needs the opt-in, which is a setting of the function on one device.
+// The largest size granted so far is kept per (device, kernel), so the
+// attribute is set only when a launch needs more than before (and never
+// lowered under a concurrent caller).
 static cudaError_t reserve_dyn_smem(const void* fn, size_t bytes) {
   static std::mutex mu;
-  static const void* fns[64];
-  static size_t granted[64];
+  constexpr int kSlots = 256;
+  static const void* fns[kSlots];
+  static int devs[kSlots];
+  static size_t granted[kSlots];
   static int n = 0;
+  const int dev = current_device();
   std::lock_guard<std::mutex> lock(mu);
   int i = 0;
-  while (i < n && fns[i] != fn) ++i;
+  while (i < n && !(fns[i] == fn && devs[i] == dev)) ++i;
   if (i < n && granted[i] >= bytes) return cudaSuccess;
   const cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -272,8 +288,9 @@ static cudaError_t reserve_dyn_smem(const void* fn, size_t bytes) {
   }
   if (i < n) {
     granted[i] = bytes;
-  } else if (n < 64) {
+  } else if (n < kSlots) {
     fns[n] = fn;
+    devs[n] = dev;
     granted[n++] = bytes;
   }
   return cudaSuccess;

@@ -264,6 +264,10 @@ struct FusedArgs {
 // row statistics precede.
 cudaError_t launch_chain_fused(const FusedArgs& a, cudaStream_t st);
 
+// SPEC_OK for cudaSuccess; otherwise records e as the calling thread's last
+// CUDA error (spec_last_cuda_error) and returns SPEC_ECUDA.
+int record_cuda_status(cudaError_t e);
+
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
 
 // Outcome law of a chain check (drafts fixed): see outcome.cu.

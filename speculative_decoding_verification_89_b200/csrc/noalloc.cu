@@ -11,12 +11,16 @@
 //
 // The array is a file-scope __device__ variable of SPEC_NOALLOC_SCRATCH_BYTES,
 // so every GPU that loads the library keeps that much of its memory until the
-// process exits. Host code cannot use the array's name as a device address;
-// the first call on each device, with that device current, asks the runtime
-// for the address (cudaGetSymbolAddress) and keeps it, so make that first call
-// outside any stream capture. The array is shared by every call and keeps the
-// previous call's contents, none of which a later call reads before writing.
-// Calls that overlap on the GPU (other streams, other threads) race on it.
+// process exits. Host code cannot use the array's name as a device address:
+// a call asks the runtime for the address (cudaGetSymbolAddress) with the
+// device current, and keeps it per device and per CUDA context, so the
+// lookup runs once per device (again only if the device's context was
+// destroyed and re-created). A lookup that fails is not kept: the next call
+// tries again. Make the first call on a device outside any stream capture.
+// The array is shared by every call and keeps the previous call's contents;
+// the per-call counters in it are cleared by the call's own first launch, and
+// nothing else is read before it is written. Calls that overlap on the GPU
+// (other streams, other threads) race on it.
 #include <mutex>
 
 #include "common.cuh"
@@ -29,22 +33,62 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::once_flag g_once[kMaxDevices];
-void* g_addr[kMaxDevices];
-cudaError_t g_err[kMaxDevices];
+// Successful lookups only: the context they were made in and the address.
+struct Slot {
+  void* ctx;
+  void* addr;
+};
+std::mutex g_mu;
+Slot g_slot[kMaxDevices];
+int g_fail_lookups = 0;  // test hook: lookups still to be refused
 
-// Device address of the scratch array on the current device, looked up once
-// per device.
+// cuCtxGetCurrent through the runtime's driver entry point (no link against
+// the driver library); null if the driver does not provide it.
+typedef int (*CtxGetCurrentFn)(void**);
+CtxGetCurrentFn ctx_get_current() {
+  static const CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      p = nullptr;
+    }
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+void* current_ctx() {
+  const CtxGetCurrentFn fn = ctx_get_current();
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the scratch array on the current device.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev]() {
-    g_err[dev] = cudaGetSymbolAddress(&g_addr[dev], g_noalloc_scratch);
-  });
-  *out = g_addr[dev];
-  return g_err[dev];
+  void* ctx = current_ctx();
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_fail_lookups > 0) {
+    --g_fail_lookups;
+    return cudaErrorStreamCaptureUnsupported;  // what a lookup inside a capture returns
+  }
+  if (ctx && g_slot[dev].addr && g_slot[dev].ctx == ctx) {
+    *out = g_slot[dev].addr;
+    return cudaSuccess;
+  }
+  void* addr = nullptr;
+  e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;  // nothing kept: the next call looks it up again
+  ctx = current_ctx();             // the lookup made the device's context current
+  if (ctx) g_slot[dev] = Slot{ctx, addr};
+  *out = addr;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -62,13 +106,21 @@ int spec_verify_chain_noalloc(const void* tgt, int64_t ld_tgt, const void* drf, 
   if (B == 0) return SPEC_OK;
   if (need > kScratchBytes) return SPEC_EWORKSPACE;
   void* ws = nullptr;
-  cudaError_t e = scratch_address(&ws);
+  const cudaError_t e = scratch_address(&ws);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return SPEC_ECUDA;
+    return specv::record_cuda_status(e);
   }
   return spec_verify_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok, temperature, seed,
                            seq_id, round, accept_len, out_tok, diag, dev_status, ws, need, stream);
+}
+
+int spec_noalloc_test_fail_lookups(int n) {
+  if (n < 0) return SPEC_EINVAL;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_fail_lookups = n;
+  for (int d = 0; d < kMaxDevices; ++d) g_slot[d] = Slot{nullptr, nullptr};
+  return SPEC_OK;
 }
 
 }  // extern "C"

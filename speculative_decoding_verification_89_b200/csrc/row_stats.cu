@@ -534,15 +534,9 @@ template <typename T, typename Rows>
 static cudaError_t launch_rs(const Rows& rows, int nrows, int V, Partial* part, double* mom,
                              int32_t* zero_word, int32_t* status, cudaStream_t st) {
   auto kern = row_stats_kernel<T, Rows>;
-  static bool smem_set = false;  // once per instantiation (same on every B200)
-  if (!smem_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmemTotal);
-    if (e != cudaSuccess) {
-      cudaGetLastError();  // do not leave the error pending for later calls
-      return e;
-    }
-    smem_set = true;
+  {
+    const cudaError_t e = reserve_dyn_smem(kern, (size_t)kRsSmemTotal);
+    if (e != cudaSuccess) return e;
   }
   constexpr int kEpt = kTileBytes / (int)sizeof(T);
   const long long ntiles = (V + kEpt - 1) / kEpt;

@@ -23,6 +23,7 @@ class Tally:
         self.details = []
 
     def check_share(self):
+        print(f"decisions compared: {self.decisions}, excused near-margin: {self.excused}")
         assert self.excused <= 1e-4 * max(self.decisions, 1) or self.excused == 0, \
             f"{self.excused} near-margin decisions of {self.decisions}: {self.details[:5]}"
 

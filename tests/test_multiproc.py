@@ -70,3 +70,23 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_gpus_flag_launches_one_rank_per_gpu():
+    """`bench.py --gpus 2` outside a launcher starts two ranks itself (gloo
+    here, --plan-only: no GPU work); each rank takes its own device index,
+    its own sequences and its own seeds."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--plan-only"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout          # rank 0 alone prints
+    plans = json.loads(lines[0])["plans"]
+    assert [p["rank"] for p in plans] == [0, 1] and all(p["world"] == 2 for p in plans)
+    assert [p["device"] for p in plans] == [0, 1]
+    assert plans[0]["seq_id_base"] != plans[1]["seq_id_base"]
+    assert plans[1]["seq_id_base"] - plans[0]["seq_id_base"] >= 64   # disjoint B=64 ranges
+    assert plans[0]["logit_seed"] != plans[1]["logit_seed"]
+    assert plans[0]["pool_seed"] != plans[1]["pool_seed"]

@@ -169,3 +169,29 @@ def test_log_partition_is_logsumexp():
             l[rng.integers(0, 257, size=5)] = -np.inf
             want = scipy.special.logsumexp(l / T)
             assert abs(log_partition(l, T) - want) <= 1e-13 * max(1.0, abs(want))
+
+
+def test_inverse_cdf_boundary_and_rounding_fallback():
+    """The draw's boundary rule (smallest v with C(v) > u * Z) at the
+    interval ends, and the fallback for a target that reaches Z itself:
+    u * Z == Z happens for u = 1 (valid Philox uniforms stop at 1 - 2^-24,
+    so only rounding could get there); the draw then takes the last token
+    with mass, never a zero-mass token past it."""
+    from oracle.verify import inverse_cdf
+    w = np.array([0.0, 0.25, 0.0, 0.5, 0.25, 0.0, 0.0])
+    z = w.sum()
+    # Interval ends: C = [0, .25, .25, .75, 1, 1, 1].
+    assert inverse_cdf(w, 0.0)[0] == 1              # C(1) = .25 > 0
+    assert inverse_cdf(w, 0.25)[0] == 3             # C(1) = .25 is not > .25
+    assert inverse_cdf(w, np.nextafter(0.25, 0))[0] == 1
+    assert inverse_cdf(w, 0.75)[0] == 4
+    # u * Z == Z: the last token with positive mass (index 4), margin 0.
+    assert 1.0 * z == z
+    tok, margin = inverse_cdf(w, 1.0)
+    assert tok == 4 and margin == 0.0
+    # The largest valid uniform lands on the same token without the fallback.
+    assert inverse_cdf(w, 1.0 - 2.0 ** -24)[0] == 4
+    # A single token with mass is drawn for every u, the fallback included.
+    one = np.array([0.0, 0.0, 3.0, 0.0])
+    for u in (2.0 ** -24, 0.5, 1.0 - 2.0 ** -24, 1.0):
+        assert inverse_cdf(one, u)[0] == 2
