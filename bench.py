@@ -6,13 +6,12 @@ drafts over a V=128256 bf16 vocabulary (targets N(0, 2^2) plus a Zipf(1.1)
 log-prior over ids, drafts = target + N(0, 1), T = 1), followed by the
 paged-KV commit of a+1 rows per sequence (block 16, contexts U[512, 4096],
 128 KiB of K/V per token, hidden rows of 4096 bf16). One step = the fused
-verify-and-commit path through the C ABI: row statistics; the check and draw
-per sequence, whose last sequence to pass its accept test plans the commit,
-copying the kept K/V rows that land in held blocks; then the remaining copy --
-three launches. Each step
-verifies a fresh Philox round and commits against the same committed prefix,
-so it rolls the previous round back and grows again: the pool stays bounded
-and every step does the same kind of work.
+verify-and-commit path through the C ABI (spec_verify_chain_commit's
+launches: row statistics; the check and draw per sequence, whose last
+sequence to pass its accept test plans the commit; the copy of the kept
+rows). Each step verifies a fresh Philox round and commits against the same
+committed prefix, so it rolls the previous round back and grows again: the
+pool stays bounded and every step does the same kind of work.
 
 Prints one JSON line (rank 0). ``--impl reference`` times the fp64 oracle on
 the host cores instead: a plain single-threaded program as the reference arm.
@@ -47,7 +46,7 @@ WORKLOAD = ("batched chain verification + paged commit: B=64, K=8, V=128256 bf16
             "(N(0,4) + Zipf(1.1) log-prior targets, drafts +N(0,1), T=1), block 16, "
             "contexts U[512,4096], 128 KiB K/V + 8 KiB hidden per token")
 NCU_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
-ROW_STATS_SOURCES = ["row_stats.cu", "common.cuh", "kernels.cuh"]
+ROW_STATS_SOURCES = ["row_stats.cu", "rowmath.cuh", "common.cuh", "kernels.cuh"]
 
 
 def parse():
@@ -252,19 +251,28 @@ def cpu_baseline(prob, state, budget_s=12.0):
                       f"fp64 numpy, single thread), {sec:.1f} s"}
 
 
-def spot_check(prob, acc_round0):
-    """Oracle vs GPU on two sequences of round 0 (both as run in the bench)."""
+def spot_check(prob, acc, out, rnd):
+    """Oracle vs GPU on every sequence of one step run after the timed region
+    (accepted count and emitted tokens), with the verification rule: a
+    difference is allowed only at a decision whose fp64 oracle margin is
+    below 1e-6, and such decisions must stay under 1e-4 of all."""
     from oracle.verify import verify_chain
     to64 = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
-    ok = True
-    for b in (0, B - 1):
-        r = verify_chain(to64(prob.tgt[b:b + 1]), to64(prob.drf[b:b + 1]),
-                         prob.draft_tok[b:b + 1].cpu().numpy(),
-                         prob.temperature[b:b + 1].cpu().numpy(), prob.seed,
-                         prob.seq_id[b:b + 1].cpu().numpy(), 0)[0]
-        if r.accepted != int(acc_round0[b]):
-            ok = ok and min(d.margin for d in r.decisions) < 1e-6
-    return "ok" if ok else "MISMATCH"
+    ref = verify_chain(to64(prob.tgt), to64(prob.drf), prob.draft_tok.cpu().numpy(),
+                       prob.temperature.cpu().numpy(), prob.seed, prob.seq_id.cpu().numpy(), rnd)
+    decisions = excused = 0
+    for b, r in enumerate(ref):
+        decisions += len(r.decisions)
+        a = int(acc[b])
+        if a == r.accepted and [int(x) for x in out[b, :a + 1]] == list(r.tokens):
+            continue
+        if min(d.margin for d in r.decisions) < 1e-6:
+            excused += 1
+        else:
+            return {"result": "MISMATCH", "sequence": b}
+    ok = excused == 0 or excused <= 1e-4 * decisions
+    return {"result": "ok" if ok else "too many near-margin differences",
+            "sequences": len(ref), "decisions": decisions, "excused": excused}
 
 
 # ----------------------------------------------------------------------------
@@ -299,7 +307,7 @@ def run_ours(args, dist):
                                       hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
                                       hid_off=bufs.hid_off, stream=stream)
 
-    clocks = Clocks(dist.local)
+    clocks = Clocks(plan["device"])
     clocks.start()
     for i in range(args.warmup):
         row_stats()
@@ -371,6 +379,7 @@ def run_ours(args, dist):
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
+    result["persistent_step"] = run_persistent_step(args, prob, state, bufs, base, dev, dist)
     result["two_call_step"] = run_two_call_step(args, prob, state, bufs, base, dev, dist)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, prob, state, bufs, base, dev, dist)
@@ -378,10 +387,56 @@ def run_ours(args, dist):
     result["outcome_law"] = run_outcome_law(args, prob, dev, dist, peak)
     result["hier_step"] = run_hier_step(args, dev, dist, peak)
     if dist.world == 1 and dist.rank == 0:
-        result["parity_spot_check"] = spot_check(prob, hist[0].cpu().numpy())
+        rnd = args.warmup + args.steps
+        acc1 = torch.empty(B, dtype=torch.int32, device=dev)
+        capi.spec_verify_chain_commit(tgt, drf, dt, T, prob.seed, sid, rnd, acc1, out_tok,
+                                      state.tables, state.seq_lens, base, state.free_stack,
+                                      state.free_top, status, ws, block_size=16,
+                                      kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
+                                      hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
+                                      hid_off=bufs.hid_off, stream=stream)
+        torch.cuda.synchronize()
+        result["parity_spot_check"] = spot_check(prob, acc1.cpu().numpy(),
+                                                 out_tok.cpu().numpy(), rnd)
         if not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(prob, state)
     return result
+
+
+def run_persistent_step(args, prob, state, bufs, base, dev, dist):
+    """The same step through spec_verify_chain_commit_persistent: a prologue
+    launch, then one persistent kernel for the row statistics, the checks,
+    the draws, the plan and the copy -- two launches."""
+    from speculative_decoding_verification_89_b200 import capi
+    n = max(10, min(args.steps, 2000))
+    acc = torch.empty((n, B), dtype=torch.int32, device=dev)
+    out = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = capi.workspace(B, K, V, torch.bfloat16, device=dev)
+
+    def step(i):
+        capi.spec_verify_chain_commit_persistent(
+            prob.tgt, prob.drf, prob.draft_tok, prob.temperature, prob.seed, prob.seq_id, i,
+            acc[i], out, state.tables, state.seq_lens, base, state.free_stack, state.free_top,
+            status, ws, block_size=16, kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
+            hid_stage=bufs.hid_stage, hid_out=bufs.hid_out, hid_off=bufs.hid_off)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.reduce(e0.elapsed_time(e1), "max")
+    if int(status.item()) != 0:
+        raise RuntimeError("device status during the persistent run")
+    tokens = float((acc.cpu().numpy() + 1).sum())
+    return {"steps": n, "ms_per_step": ms / n, "tokens_per_s": tokens / (ms * 1e-3),
+            "gpu_launches_per_step": 2}
 
 
 def run_two_call_step(args, prob, state, bufs, base, dev, dist):
@@ -530,9 +585,9 @@ def run_hier_step(args, dev, dist, peak):
     ctok, cn = torch.empty((Bh, WC + 1), **i32), torch.empty(Bh, **i32)
     status = torch.zeros(1, **i32)
     ws = capi.workspace(Bh, Kh, Vh, hp.lg_f.dtype, Ni=Ni, device=dev)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(11)
-    drafts = torch.randint(0, Vh, (Bh, Kh), generator=gen, device=dev, dtype=torch.int32)
+    # Drafts drawn from the drafting exit L_d at the window's first slots, as
+    # an engine would produce them.
+    drafts = W.window_drafts(hp.lg_d, win_len, Kh, hp.temperature, W.generator(11, dev))
 
     def call(i):
         capi.spec_verify_hier(hp.lg_d, hp.lg_i, hp.lg_f, Ni, drafts, hp.temperature, hp.seed,

@@ -290,6 +290,39 @@ int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf,
                              void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The same two calls on one persistent kernel ([HS] "Verlustfreie Garantie",
+ * "Wiederverwendung von KV-Cache", "Unterstuetzung fuer Batch-Inferenz", as
+ * above). A prologue launch clears the call's counters in the workspace, then
+ * one CTA of 16 warps per SM takes (row, chunk) items of the logit rows from
+ * a counter in global memory (dynamic balance over the SMs); the warp that
+ * completes a row combines it, the one that completes a sequence runs its
+ * accept test, residual draws run as 4 KiB parts of the row pair taken by
+ * any warp, and (the commit form) the warp that checks the last sequence
+ * plans the commit before every warp copies 8 KiB units of the kept rows.
+ * Arguments, layouts, results and errors: those of spec_verify_chain and
+ * spec_verify_chain_commit (same workspace size); a bounded wait that runs
+ * out records SPEC_ETIMEOUT and stops every other wait of the call. The
+ * outputs agree with the other entry points' to the verification tolerance
+ * (the row sums are taken in chunks of other sizes, so bits may differ).
+ * ------------------------------------------------------------------------- */
+int spec_verify_chain_persistent(const void* tgt, int64_t ld_tgt, const void* drf,
+                                 int64_t ld_drf, int dtype, int B, int K, int V,
+                                 const int32_t* draft_tok, const float* temperature,
+                                 uint64_t seed, const int32_t* seq_id, uint32_t round,
+                                 int32_t* accept_len, int32_t* out_tok, double* diag,
+                                 int32_t* dev_status, void* ws, size_t ws_bytes,
+                                 void* stream);
+int spec_verify_chain_commit_persistent(
+    const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype, int B, int K,
+    int V, const int32_t* draft_tok, const float* temperature, uint64_t seed,
+    const int32_t* seq_id, uint32_t round, int32_t* accept_len, int32_t* out_tok, double* diag,
+    int block_size, int max_blocks, int32_t* block_tables, int32_t* seq_lens,
+    const int32_t* base_len, int32_t* free_stack, int32_t* free_top, int num_blocks,
+    const void* kv_stage, void* kv_pool, int layers, int kv_heads, int head_dim,
+    const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden, int32_t* dev_status,
+    void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Draft step ([HS] Kernmechanismus: the shallow exit L_d drafts the tokens the
  * deeper exits check; [SV] the entropy of the drafting distribution). The
  * pages print no interface; this is the step that produces the draft_tok of

@@ -13,9 +13,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libspecverify.so")
-SOURCES = ["row_stats.cu", "decide.cu", "draft.cu", "outcome.cu", "commit.cu", "capi.cu",
-           "noalloc.cu"]
-HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh", "commit.cuh"]
+SOURCES = ["row_stats.cu", "step.cu", "decide.cu", "draft.cu", "outcome.cu", "commit.cu",
+           "capi.cu", "noalloc.cu"]
+HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh", "commit.cuh", "rowmath.cuh"]
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",

@@ -48,6 +48,12 @@ _SIGS = {
     "spec_chain_decide_commit": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
                                       _u32, _p, _p, _p, _i, _i, _p, _p, _p, _p, _p, _i, _p,
                                       _p, _i, _i, _i, _p, _p, _p, _i, _p, _p, _sz, _p]),
+    "spec_verify_chain_persistent": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64,
+                                          _p, _u32, _p, _p, _p, _p, _p, _sz, _p]),
+    "spec_verify_chain_commit_persistent": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p,
+                                                 _u64, _p, _u32, _p, _p, _p, _i, _i, _p, _p, _p,
+                                                 _p, _p, _i, _p, _p, _i, _i, _i, _p, _p, _p, _i,
+                                                 _p, _p, _sz, _p]),
     "spec_philox_uniforms": (_i, [_u64, _p, _i, _p, _p]),
     "spec_last_cuda_error": (ctypes.c_char_p, []),
     "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
@@ -131,15 +137,21 @@ def workspace(B, K, V, dtype, Ni=0, device="cuda"):
 
 
 def spec_verify_chain(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
-                      out_tok, dev_status, ws, diag=None, stream=None):
+                      out_tok, dev_status, ws, diag=None, stream=None,
+                      _entry="spec_verify_chain"):
     B, Kp1, V = tgt.shape
     K = Kp1 - 1
-    rc = _lib.spec_verify_chain(
+    rc = getattr(_lib, _entry)(
         _ptr(tgt), _rows(tgt, Kp1), _ptr(drf) if K > 0 else None,
         _rows(drf, K) if K > 0 else 0, _dtype_code(tgt), B, K, V, _ptr(draft_tok),
         _ptr(temperature), seed, _ptr(seq_id), rnd, _ptr(accept_len), _ptr(out_tok),
         _ptr(diag), _ptr(dev_status), _ptr(ws), ws.numel(), _stream(stream))
-    _check("spec_verify_chain", rc)
+    _check(_entry, rc)
+
+
+def spec_verify_chain_persistent(*args, **kw):
+    """spec_verify_chain on the persistent kernel (same arguments)."""
+    spec_verify_chain(*args, _entry="spec_verify_chain_persistent", **kw)
 
 
 def spec_verify_chain_noalloc(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
@@ -258,6 +270,11 @@ def spec_chain_decide_commit(tgt, drf, draft_tok, temperature, seed, seq_id, rnd
     spec_verify_chain_commit(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accept_len,
                              out_tok, block_tables, seq_lens, base_len, free_stack, free_top,
                              dev_status, ws, _entry="spec_chain_decide_commit", **kw)
+
+
+def spec_verify_chain_commit_persistent(*args, **kw):
+    """spec_verify_chain_commit on the persistent kernel (same arguments)."""
+    spec_verify_chain_commit(*args, _entry="spec_verify_chain_commit_persistent", **kw)
 
 
 def spec_philox_uniforms(seed, ctr, out, stream=None):

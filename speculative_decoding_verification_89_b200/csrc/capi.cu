@@ -1,6 +1,7 @@
 // C ABI of libspecverify: argument checks on the host, workspace carving and
 // the launch sequence of each call. Declarations and the contract of every
 // entry point are in include/spec_verify.h.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 
@@ -21,13 +22,15 @@ int stat_tiles(int V, int dtype) {
 }
 
 struct Layout {
-  size_t part, fin, ticket, total;
+  size_t part, fin, ticket, seq, tsum, ctr, ints, total;
   long long rows;
 };
 
-// Workspace: final row statistics and tile partials for the largest row set,
-// then the ticket word of the fused verify-and-commit path, each region
-// 256-byte aligned.
+// Workspace, each region 256-byte aligned: final row statistics and tile
+// partials for the largest row set (the step kernel keeps its chunk
+// statistics in the partials' place), the ticket word of the staged
+// verify-and-commit path, then the step kernel's per-sequence states,
+// residual tile sums, counters and per-sequence integer arrays.
 bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   if (B < 0 || K < 0 || K > SPEC_MAX_K || V < 1 || V > SPEC_MAX_V) return false;
   if (dtype != SPEC_F32 && dtype != SPEC_BF16) return false;
@@ -39,7 +42,15 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   L->fin = 0;
   L->part = align_up((size_t)rows * sizeof(RowFinal));
   L->ticket = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
-  L->total = L->ticket + kAlign;
+  L->seq = L->ticket + kAlign;
+  L->tsum = L->seq + align_up((size_t)B * sizeof(SeqState));
+  // residual tile sums [B][nrt], then the draw-part totals [B][D]
+  const size_t pt = part_tiles(elem_size(dtype));
+  const size_t nrt = residual_tiles(V), D = (nrt + pt - 1) / pt;
+  L->ctr = L->tsum + align_up((size_t)B * (nrt + D) * sizeof(double));
+  L->ints = L->ctr + align_up(sizeof(StepCounters));
+  // seq_cnt, seq_done, draw_cnt, tok_off [B] each; tok_seq [B * (K+1)]; row_cnt [rows]
+  L->total = L->ints + align_up(((size_t)B * (4 + K + 1) + (size_t)rows) * sizeof(int));
   return true;
 }
 
@@ -136,6 +147,61 @@ DecideCommon common_args(int dtype, int B, int K, int V, const int32_t* draft_to
   c.diag = diag;
   c.status = dev_status;
   return c;
+}
+
+// Arguments of the verification step kernel for a chain call (workspace
+// already checked).
+StepArgs step_args(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                   int B, int K, int V, const int32_t* draft_tok, const float* temperature,
+                   uint64_t seed, const int32_t* seq_id, uint32_t round, int32_t* accept_len,
+                   int32_t* out_tok, double* diag, int32_t* dev_status, void* ws,
+                   const Layout& L, int late_pos) {
+  StepArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const int es = elem_size(dtype);
+  a.dtype = dtype;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.tgt = (const unsigned char*)tgt;
+  a.drf = (const unsigned char*)drf;
+  a.ld_tgt = ld_tgt * es;
+  a.ld_drf = ld_drf * es;
+  a.draft_tok = draft_tok;
+  a.temperature = temperature;
+  a.seed = seed;
+  a.seq_id = seq_id;
+  a.round = round;
+  a.accept_len = accept_len;
+  a.out_tok = out_tok;
+  a.diag = diag;
+  a.status = dev_status;
+  a.nt = stat_tiles(V, dtype);
+  a.NCe = (a.nt + kChunkTiles - 1) / kChunkTiles;
+  a.NCl = (a.nt + kLateChunkTiles - 1) / kLateChunkTiles;
+  a.NC = std::max(a.NCe, a.NCl);
+  a.lp = std::min(late_pos, K);
+  a.re = 2 * K + 1 - 2 * a.lp;
+  a.rl = 2 * a.lp;
+  a.n_early = (unsigned)((long long)B * a.re * a.NCe);
+  a.n_total = a.n_early + (unsigned)((long long)B * a.rl * a.NCl);
+  a.nrt = residual_tiles(V);
+  a.D = (a.nrt + part_tiles(es) - 1) / part_tiles(es);
+  char* w = (char*)ws;
+  a.part = reinterpret_cast<ChunkStat*>(w + L.part);
+  a.fin = reinterpret_cast<RowFinal*>(w + L.fin);
+  a.seq = reinterpret_cast<SeqState*>(w + L.seq);
+  a.tsum = reinterpret_cast<double*>(w + L.tsum);
+  a.ptot = a.tsum + (size_t)B * a.nrt;
+  a.ctr = reinterpret_cast<StepCounters*>(w + L.ctr);
+  int* ints = reinterpret_cast<int*>(w + L.ints);
+  a.seq_cnt = ints;
+  a.seq_done = ints + B;
+  a.draw_cnt = ints + 2 * B;
+  a.tok_off = ints + 3 * B;
+  a.tok_seq = ints + 4 * B;
+  a.row_cnt = ints + (size_t)B * (4 + K + 1);
+  return a;
 }
 
 }  // namespace
@@ -305,6 +371,26 @@ int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t 
                            stream);
 }
 
+int spec_verify_chain_persistent(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                                 int dtype, int B, int K, int V, const int32_t* draft_tok,
+                                 const float* temperature, uint64_t seed, const int32_t* seq_id,
+                                 uint32_t round, int32_t* accept_len, int32_t* out_tok,
+                                 double* diag, int32_t* dev_status, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!seq_id || !accept_len || !out_tok || (K > 0 && !draft_tok)) {
+    Layout L;
+    if (layout(B, K, V, dtype, 0, &L) && B == 0) return SPEC_OK;
+    return SPEC_EINVAL;
+  }
+  const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
+                                    ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  const StepArgs a = step_args(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok, temperature,
+                               seed, seq_id, round, accept_len, out_tok, diag, dev_status, ws,
+                               ck.L, late_positions(B, V, dtype, 2));
+  return cuda_status(launch_chain_step(a, (cudaStream_t)stream));
+}
+
 int spec_verify_hier(const void* lg_d, const void* lg_i, const void* lg_f, int64_t ld, int dtype,
                      int B, int K, int V, int Ni, const int32_t* draft_tok,
                      const float* temperature, uint64_t seed, const int32_t* seq_id,
@@ -447,6 +533,41 @@ int spec_verify_chain_commit(const void* tgt, int64_t ld_tgt, const void* drf, i
                                   free_stack, free_top, num_blocks, kv_stage, kv_pool, layers,
                                   kv_heads, head_dim, hid_stage, hid_out, hid_off, hidden,
                                   dev_status, ws, ws_bytes, stream);
+}
+
+int spec_verify_chain_commit_persistent(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                             int dtype, int B, int K, int V, const int32_t* draft_tok,
+                             const float* temperature, uint64_t seed, const int32_t* seq_id,
+                             uint32_t round, int32_t* accept_len, int32_t* out_tok, double* diag,
+                             int block_size, int max_blocks, int32_t* block_tables,
+                             int32_t* seq_lens, const int32_t* base_len, int32_t* free_stack,
+                             int32_t* free_top, int num_blocks, const void* kv_stage,
+                             void* kv_pool, int layers, int kv_heads, int head_dim,
+                             const void* hid_stage, void* hid_out, int32_t* hid_off, int hidden,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  // Every host check of the second half first, so a refused call launches nothing.
+  if (B < 0 || B > SPEC_MAX_FUSED_B || K < 0 || K > SPEC_MAX_K) return SPEC_EINVAL;
+  CommitArgs cm;
+  int rc = commit_args(B, block_size, max_blocks, block_tables, seq_lens, base_len, accept_len,
+                       1, free_stack, free_top, num_blocks, K + 1, kv_stage, kv_pool, layers,
+                       kv_heads, head_dim, hid_stage, hid_out, hid_off, hidden, dev_status, &cm);
+  if (rc != SPEC_OK) return rc;
+  const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
+                                    ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!seq_id || !out_tok || (K > 0 && !draft_tok)) return SPEC_EINVAL;
+  StepArgs a = step_args(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok, temperature, seed,
+                         seq_id, round, accept_len, out_tok, diag, dev_status, ws, ck.L,
+                         late_positions(B, V, dtype, 2));
+  a.commit = 1;
+  a.cm = cm;
+  if (cm.kv_stage) {
+    const int nseg = cm.layers * 2;
+    a.unit_segs = std::max(1, kCopyUnit / cm.seg_bytes);
+    a.units_kv = (nseg + a.unit_segs - 1) / a.unit_segs;
+  }
+  a.units_tok = a.units_kv + (cm.hid_stage ? 1 : 0);
+  return cuda_status(launch_chain_step(a, (cudaStream_t)stream));
 }
 
 size_t spec_draft_workspace_bytes(int B, int V, int dtype) {

@@ -234,8 +234,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
   if (!o.bad && !greedy) {
     prow = tp(o.a);
     qrow = o.a < K ? dp(o.a) : nullptr;
-    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], sc);
-    kq = make_coef(o.a < K ? dl(o.a) : 0.0, sc);
+    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], lsh->m[o.a], sc);
+    kq = o.a < K ? make_coef(dl(o.a), lsh->m[K + 1 + o.a], sc) : make_coef(0.0, 0.0f, sc);
     const int chunk = (nrt + kCluster - 1) / kCluster;
     residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
                           min(nrt, ((int)rank + 1) * chunk), ltsum);
@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier1_decide_kernel(HierDecide
   if (!o.bad && !greedy) {
     prow = tp(o.a);
     qrow = o.a < K ? dp(o.a) : nullptr;
-    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], sc);
-    kq = make_coef(o.a < K ? dl(o.a) : 0.0, sc);
+    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], lsh->m[o.a], sc);
+    kq = o.a < K ? make_coef(dl(o.a), lsh->m[K + 1 + o.a], sc) : make_coef(0.0, 0.0f, sc);
     const int chunk = (nrt + kCluster - 1) / kCluster;
     residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
                           min(nrt, ((int)rank + 1) * chunk), ltsum);
@@ -440,8 +440,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
   if (!o.bad && !greedy) {
     prow = tp(o.a);
     qrow = o.a < W ? dp(o.a) : nullptr;
-    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], sc);
-    kq = make_coef(o.a < W ? dl(o.a) : 0.0, sc);
+    kp = make_coef(lsh->M[o.a] + lsh->L[o.a], lsh->m[o.a], sc);
+    kq = o.a < W ? make_coef(dl(o.a), (float)wst[2 * o.a], sc) : make_coef(0.0, 0.0f, sc);
     const int chunk = (nrt + kCluster - 1) / kCluster;
     residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
                           min(nrt, ((int)rank + 1) * chunk), ltsum);
@@ -588,8 +588,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
   if (draw) {
     prow = tp(a);
     qrow = a < K ? dp(a) : nullptr;
-    kp = make_coef(lsh->M[a] + lsh->L[a], sc);
-    kq = make_coef(a < K ? dl(a) : 0.0, sc);
+    kp = make_coef(lsh->M[a] + lsh->L[a], lsh->m[a], sc);
+    kq = a < K ? make_coef(dl(a), lsh->m[K + 1 + a], sc) : make_coef(0.0, 0.0f, sc);
     const int chunk = (nrt + kWorkers - 1) / kWorkers, wr = (int)rank - 1;
     if (wr >= 0)
       residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, wr * chunk),

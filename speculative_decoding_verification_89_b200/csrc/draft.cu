@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
     if (rank == 0 && threadIdx.x == 0) finish(st.amax, 0.0, 0.0, !st.ok);
     return;
   }
-  const ProbCoef kp = make_coef(st.Lt, sc);
+  const ProbCoef kp = make_coef(st.Lt, st.m, sc);
   const int nrt = residual_tiles(V);
   const int chunk = (nrt + kCluster - 1) / kCluster;
   asm volatile("barrier.cluster.wait;" ::: "memory");  // every CTA runs: remote writes allowed
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
   const bool fin = m_r > -INFINITY && m_r < INFINITY;
   if (!greedy && fin) {
     const float Mr = __fmul_rn(m_r, sc.hi);
-    const ProbCoef kr = make_coef((double)Mr, sc);
+    const ProbCoef kr = make_coef((double)Mr, m_r, sc);
     double ws = 0.0, wt = 0.0;
     for (int t = warp; t < nt; t += kDecWarps) {
       float x[8], w[8];
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     const unsigned holder = __ballot_sync(0xffffffffu, cand == best && best >= 0);
     const double pre = holder ? __shfl_sync(0xffffffffu, c_cand, __ffs(holder) - 1) : 0.0;
     const float Mr = __fmul_rn(s_part[owner].m, sc.hi);
-    const ProbCoef kr = make_coef((double)Mr, sc);
+    const ProbCoef kr = make_coef((double)Mr, s_part[owner].m, sc);
     float x[8], w[8];
     smem8(xs, tile * kResTile + lane * 8, n, x);
 #pragma unroll

@@ -35,7 +35,9 @@ constexpr int kResGroup = sizeof(T) == 2 ? 4 : 2;
 // Residual weights of 8 consecutive elements
 // ---------------------------------------------------------------------------
 // 8 consecutive logits as raw 16-byte vectors (one for bf16, two for fp32);
-// zeros when `on` is false (nothing is read then).
+// zeros when `on` is false (nothing is read then). The loads go to L2 and
+// allocate nothing in L1: a warp keeps several tiles of them in flight, more
+// than the L1 left beside a large shared-memory carve-out can hold.
 template <typename T>
 struct Raw8 {
   uint4 v[sizeof(T) / 2];
@@ -46,7 +48,7 @@ __device__ __forceinline__ Raw8<T> raw8(const T* row, int e0, bool on) {
   const uint4* p = reinterpret_cast<const uint4*>(row + e0);
 #pragma unroll
   for (int i = 0; i < (int)(sizeof(T) / 2); ++i)
-    r.v[i] = on ? __ldg(p + i) : make_uint4(0u, 0u, 0u, 0u);
+    r.v[i] = on ? __ldcg(p + i) : make_uint4(0u, 0u, 0u, 0u);
   return r;
 }
 __device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16>& r, float x[8]) {
@@ -71,26 +73,31 @@ __device__ __forceinline__ void load8(const T* row, int e0, int V, float x[8]) {
   }
 }
 
-// Probability of a logit x of a row with log2-partition Lt = M + L:
-// 2^(x*c - Lt), c = chi + clo, Lt = Lhi + Llo; the product x*chi - Lhi is
-// rounded once relative to the (small) result.
+// Probability of a logit x of a row with log2-partition Lt and largest logit
+// m: p = 2^(x*c - Lt) (c = chi + clo), formed as 2^(x*c - M) * k with the
+// integral shift M = ceil(m * chi) and k = 2^(M - Lt) carried as two floats.
+// The most likely tokens get exponents in (-1, 0], where the fp32 rounding of
+// x*chi - M (once, by the FMA) is smallest; k is exact to about 2^-48.
 struct ProbCoef {
-  float chi, clo, nLhi, nLlo;
+  float chi, clo, nM, khi, klo;
 };
-__device__ __forceinline__ ProbCoef make_coef(double Lt, const Scale& s) {
+__device__ __forceinline__ ProbCoef make_coef(double Lt, float m, const Scale& s) {
   ProbCoef k;
   k.chi = s.hi;
   k.clo = s.lo;
-  const float hi = (float)Lt;
-  k.nLhi = -hi;
-  k.nLlo = -(float)(Lt - (double)hi);
+  float M = ceilf(m * s.hi);
+  if (!(M > -INFINITY && M < INFINITY)) M = 0.0f;  // no finite maximum: any shift
+  k.nM = -M;
+  const double f = exp2((double)M - Lt);
+  k.khi = (float)f;
+  k.klo = (float)(f - (double)k.khi);
   return k;
 }
 __device__ __forceinline__ float2 prob2(float2 x, const ProbCoef& k) {
-  float2 t = __ffma2_rn(x, make_float2(k.chi, k.chi), make_float2(k.nLhi, k.nLhi));
+  float2 t = __ffma2_rn(x, make_float2(k.chi, k.chi), make_float2(k.nM, k.nM));
   t = __ffma2_rn(x, make_float2(k.clo, k.clo), t);
-  t = __fadd2_rn(t, make_float2(k.nLlo, k.nLlo));
-  return make_float2(ex2(t.x), ex2(t.y));
+  const float2 e = make_float2(ex2(t.x), ex2(t.y));
+  return __ffma2_rn(e, make_float2(k.khi, k.khi), __fmul2_rn(e, make_float2(k.klo, k.klo)));
 }
 
 // Weights w = max(0, p - q) (or p when there is no draft row) of 8 elements

@@ -268,6 +268,94 @@ cudaError_t launch_chain_fused(const FusedArgs& a, cudaStream_t st);
 // CUDA error (spec_last_cuda_error) and returns SPEC_ECUDA.
 int record_cuda_status(cudaError_t e);
 
+// ----------------------------------------------------------------------------
+// Chain verification step: one persistent launch for the row statistics, the
+// checks, the draws and (optionally) the paged commit, after a prologue launch
+// that clears its counters.
+// ----------------------------------------------------------------------------
+constexpr int kChunkTiles = 4;   // tiles per stream chunk of an early row (about)
+constexpr int kLateChunkTiles = 2;  // tiles per stream chunk of a late row (about)
+constexpr int kCopyUnit = 8192;  // bytes of K/V rows per copy unit
+constexpr int kPartBytes = 4096;  // bytes of each row per draw part
+__host__ __device__ constexpr int part_tiles(int esz) { return kPartBytes / (256 * esz); }
+
+// Statistics of one chunk of consecutive tiles of one row. Sampled rows:
+// largest raw logit m, the exact fp32 shift M (as bits in aux) the chunk's
+// sum s = sum 2^(l*c - M) is taken against. Greedy rows: m and its first
+// index (aux); s = 0.
+struct ChunkStat {
+  float m;
+  int aux;
+  double s;
+};
+
+// Per-call counters, cleared by the prologue launch.
+struct StepCounters {
+  unsigned stream;  // next stream item
+  unsigned draw;    // next draw part
+  unsigned copy;    // next copy unit
+  int ticket;       // sequences whose check is done
+  int plan;         // 0 pending, 1 commit planned, 2 nothing to copy
+  int abort;        // a bounded wait gave up: the other waits stop too
+  int kt;           // kept tokens of the planned commit
+  int pad;
+};
+
+// What a sequence's check leaves for its draw and its commit.
+constexpr int kSeqDraw = 1;  // a token is to be drawn (sampled, valid)
+constexpr int kSeqHasQ = 2;  // the draw is a residual (a < K): draft row a exists
+struct SeqState {
+  double lt, lq;  // log2-partitions of target row a and draft row a
+  float mt, mq;   // their largest logits
+  float u;        // draw uniform of position a
+  int a;          // accepted drafts (-1: invalid sequence)
+  int flags;
+  int old_len, base, kept, bad;  // commit: lengths before, kept rows, checks failed
+  int pad;
+};
+
+struct StepArgs {
+  int dtype, B, K, V;
+  const unsigned char* tgt;
+  const unsigned char* drf;
+  long long ld_tgt, ld_drf;  // bytes
+  const int32_t* draft_tok;
+  const float* temperature;
+  uint64_t seed;
+  const int32_t* seq_id;
+  uint32_t round;
+  int32_t* accept_len;
+  int32_t* out_tok;
+  double* diag;
+  int32_t* status;
+  // schedule: nt tiles per row; rows of positions < lp ("late") are streamed
+  // after all others, in NCl chunks each, the others in NCe chunks (re early
+  // and rl late row slots per sequence); chunk statistics have a row stride
+  // of NC = max(NCe, NCl)
+  int nt, NC, NCe, NCl, lp, re, rl;
+  unsigned n_early, n_total;  // stream items
+  int nrt, D;                 // residual tiles per row, draw parts (part_tiles tiles) per sequence
+  // workspace
+  ChunkStat* part;  // [B * (2K+1)][NC]
+  RowFinal* fin;    // [B * (2K+1)] row statistics
+  SeqState* seq;    // [B]
+  double* tsum;     // [B][nrt] residual tile sums
+  double* ptot;     // [B][D] draw-part totals
+  StepCounters* ctr;
+  int* row_cnt;     // [B * (2K+1)] chunks done
+  int* seq_cnt;     // [B] rows done
+  int* seq_done;    // [B] check done
+  int* draw_cnt;    // [B] draw parts done
+  int* tok_seq;     // [B * (K+1)] sequence of each kept token
+  int* tok_off;     // [B] first kept token of each sequence
+  // commit (commit != 0)
+  int commit;
+  int unit_segs, units_kv, units_tok;  // K/V segments per copy unit; units per token
+  CommitArgs cm;
+};
+
+cudaError_t launch_chain_step(const StepArgs& a, cudaStream_t st);
+
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
 
 // Outcome law of a chain check (drafts fixed): see outcome.cu.

@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kPairWarps * 32, 6) outcome_pair_kernel(Outcom
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y, k = blockIdx.x, K = A.K, V = A.V, n = A.n_top;
   __shared__ double s_Lt[2];
+  __shared__ float s_m[2];
   __shared__ int s_ok[2];
   __shared__ double s_z[kPairWarps];
   __shared__ float s_lw[kPairWarps][32];
@@ -115,6 +116,7 @@ __global__ void __launch_bounds__(kPairWarps * 32, 6) outcome_pair_kernel(Outcom
     const RowFinal f = combine_row(A.part + (size_t)r * A.ntiles, A.ntiles, false, sc.hi, lane);
     if (lane == 0) {
       s_Lt[warp] = f.M + f.L;
+      s_m[warp] = f.m;
       s_ok[warp] = f.ok;
     }
   }
@@ -122,8 +124,8 @@ __global__ void __launch_bounds__(kPairWarps * 32, 6) outcome_pair_kernel(Outcom
   if (!s_ok[0] || (k < K && !s_ok[1])) return;  // reported by the final kernel
   const T* prow = row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + k);
   const T* qrow = k < K ? row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + k) : nullptr;
-  const ProbCoef kp = make_coef(s_Lt[0], sc);
-  const ProbCoef kq = make_coef(k < K ? s_Lt[1] : 0.0, sc);
+  const ProbCoef kp = make_coef(s_Lt[0], s_m[0], sc);
+  const ProbCoef kq = k < K ? make_coef(s_Lt[1], s_m[1], sc) : make_coef(0.0, 0.0f, sc);
   const int nrt = residual_tiles(V);
   double z = 0.0;
   TopList e = top_empty();

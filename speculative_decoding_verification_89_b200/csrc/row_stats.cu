@@ -15,167 +15,20 @@
 // tile buffers filled by 1-D bulk copies (TMA engine, no tensor map, no
 // multicast) that complete on per-stage mbarriers. Per lane, the largest
 // logit and the sum of 2^(l*c - M) are carried across the tiles of a row with
-// a shift M that moves only when the exponents would exceed 2^64, so a tile
-// costs no warp shuffle and no division; the lanes are combined once per row
-// run into one Partial at the run's first tile (its other tiles get empty
-// partials).
-#include <cfloat>
-
+// an integral shift M that follows the lane's largest element (moved by exact
+// powers of two), so a tile costs no warp shuffle and no division; the lanes
+// are combined once per row run into one Partial at the run's first tile (its
+// other tiles get empty partials).
 #include "common.cuh"
 #include "kernels.cuh"
+#include "rowmath.cuh"
 
 namespace specv {
-
-template <typename T> struct VecOf;
-template <> struct VecOf<__nv_bfloat16> { static constexpr int n = 8; };
-template <> struct VecOf<float> { static constexpr int n = 4; };
-
-// Largest element of a 16-byte vector.
-__device__ __forceinline__ float vec_max(uint4 w, __nv_bfloat16*) {
-  __nv_bfloat162 a = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.x),
-                             *reinterpret_cast<__nv_bfloat162*>(&w.y));
-  __nv_bfloat162 c = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.z),
-                             *reinterpret_cast<__nv_bfloat162*>(&w.w));
-  a = __hmax2(a, c);
-  return fmaxf(__low2float(a), __high2float(a));
-}
-__device__ __forceinline__ float vec_max(uint4 w, float*) {
-  return fmaxf(fmaxf(__uint_as_float(w.x), __uint_as_float(w.y)),
-               fmaxf(__uint_as_float(w.z), __uint_as_float(w.w)));
-}
-__device__ __forceinline__ float vec_elem(uint4 w, int e, __nv_bfloat16*) {
-  const uint32_t word = e < 2 ? w.x : e < 4 ? w.y : e < 6 ? w.z : w.w;
-  return (e & 1) ? bf_hi(word) : bf_lo(word);
-}
-__device__ __forceinline__ float vec_elem(uint4 w, int e, float*) {
-  const uint32_t word = e == 0 ? w.x : e == 1 ? w.y : e == 2 ? w.z : w.w;
-  return __uint_as_float(word);
-}
-
-// Largest element of a lane's register-resident vectors.
-template <int kVpl>
-__device__ __forceinline__ float regs_max(const uint4* x, __nv_bfloat16*) {
-  __nv_bfloat162 m2 = __float2bfloat162_rn(-INFINITY);
-#pragma unroll
-  for (int i = 0; i < kVpl; ++i) {
-    uint4 w = x[i];
-    const __nv_bfloat162 a = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.x),
-                                     *reinterpret_cast<__nv_bfloat162*>(&w.y));
-    const __nv_bfloat162 b = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.z),
-                                     *reinterpret_cast<__nv_bfloat162*>(&w.w));
-    m2 = __hmax2(m2, __hmax2(a, b));
-  }
-  return fmaxf(__low2float(m2), __high2float(m2));
-}
-template <int kVpl>
-__device__ __forceinline__ float regs_max(const uint4* x, float*) {
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < kVpl; ++i) m = fmaxf(m, vec_max(x[i], (float*)nullptr));
-  return m;
-}
-
-// Sum over one 16-byte vector of 2^(x*c - M) with c = chi + clo and M an
-// exact fp32 shift: two packed FP32x2 FMAs per element pair form the
-// exponent (the product x*chi - M is rounded once, relative to the small
-// result), one MUFU ex2 per element, packed adds pairwise inside the vector.
-__device__ __forceinline__ float2 expo2(float2 x, float2 chi, float2 clo, float2 nM) {
-  return __ffma2_rn(x, clo, __ffma2_rn(x, chi, nM));
-}
-__device__ __forceinline__ float2 ex2x2(float2 a) { return make_float2(ex2(a.x), ex2(a.y)); }
-
-__device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, float2 nM,
-                                             __nv_bfloat16*) {
-  const float2 e0 = ex2x2(expo2(make_float2(bf_lo(w.x), bf_hi(w.x)), chi, clo, nM));
-  const float2 e1 = ex2x2(expo2(make_float2(bf_lo(w.y), bf_hi(w.y)), chi, clo, nM));
-  const float2 e2 = ex2x2(expo2(make_float2(bf_lo(w.z), bf_hi(w.z)), chi, clo, nM));
-  const float2 e3 = ex2x2(expo2(make_float2(bf_lo(w.w), bf_hi(w.w)), chi, clo, nM));
-  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
-}
-__device__ __forceinline__ float2 vec_expsum(uint4 w, float2 chi, float2 clo, float2 nM, float*) {
-  const float2 e0 =
-      ex2x2(expo2(make_float2(__uint_as_float(w.x), __uint_as_float(w.y)), chi, clo, nM));
-  const float2 e1 =
-      ex2x2(expo2(make_float2(__uint_as_float(w.z), __uint_as_float(w.w)), chi, clo, nM));
-  return __fadd2_rn(e0, e1);
-}
-// x - a, held at -FLT_MAX for x = -inf (a masked or padded entry), whose term
-// 2^(x*c - M) = 0 must then contribute 0, not 0 * -inf.
-__device__ __forceinline__ float dev1(float x, float a) { return fmaxf(x - a, -FLT_MAX); }
-__device__ __forceinline__ float2 dev2(float2 x, float2 nA) {
-  const float2 d = __fadd2_rn(x, nA);
-  return make_float2(fmaxf(d.x, -FLT_MAX), fmaxf(d.y, -FLT_MAX));
-}
-
-// Same, also returning the pairwise sums of 2^(x*c - M) * (x - a) (nA = -a),
-// the first moment the entropy of the row's distribution needs.
-__device__ __forceinline__ float2 vec_expsum_ent(uint4 w, float2 chi, float2 clo, float2 nM,
-                                                 float2 nA, float2* mom, __nv_bfloat16*) {
-  const float2 x0 = make_float2(bf_lo(w.x), bf_hi(w.x)), x1 = make_float2(bf_lo(w.y), bf_hi(w.y));
-  const float2 x2 = make_float2(bf_lo(w.z), bf_hi(w.z)), x3 = make_float2(bf_lo(w.w), bf_hi(w.w));
-  const float2 e0 = ex2x2(expo2(x0, chi, clo, nM)), e1 = ex2x2(expo2(x1, chi, clo, nM));
-  const float2 e2 = ex2x2(expo2(x2, chi, clo, nM)), e3 = ex2x2(expo2(x3, chi, clo, nM));
-  float2 t = __fmul2_rn(e0, dev2(x0, nA));
-  t = __ffma2_rn(e1, dev2(x1, nA), t);
-  t = __ffma2_rn(e2, dev2(x2, nA), t);
-  *mom = __ffma2_rn(e3, dev2(x3, nA), t);
-  return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
-}
-__device__ __forceinline__ float2 vec_expsum_ent(uint4 w, float2 chi, float2 clo, float2 nM,
-                                                 float2 nA, float2* mom, float*) {
-  const float2 x0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
-  const float2 x1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
-  const float2 e0 = ex2x2(expo2(x0, chi, clo, nM)), e1 = ex2x2(expo2(x1, chi, clo, nM));
-  *mom = __ffma2_rn(e1, dev2(x1, nA), __fmul2_rn(e0, dev2(x0, nA)));
-  return __fadd2_rn(e0, e1);
-}
-
-// Scalar form of one term (tail elements).
-__device__ __forceinline__ float term(float x, float chi, float clo, float nM) {
-  return ex2(fmaf(x, clo, fmaf(x, chi, nM)));
-}
-
-// Slow form for |M| >= 2^26, where 2^(m*c - M) itself could overflow:
-// x*c - M = (x - m)*c + (m*chi - M) + m*clo with the product residual exact.
-__device__ __forceinline__ float term_far(float x, float m, float chi, float clo, float rr) {
-  const float d = x - m;
-  return ex2(fmaf(d, chi, fmaf(d, clo, rr)));
-}
-template <typename T>
-__device__ __forceinline__ float vec_expsum_far(uint4 w, float m, float chi, float clo, float rr);
-template <>
-__device__ __forceinline__ float vec_expsum_far<__nv_bfloat16>(uint4 w, float m, float chi,
-                                                              float clo, float rr) {
-  float s = 0.0f;
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    s += term_far(bf_lo(ws[q]), m, chi, clo, rr) + term_far(bf_hi(ws[q]), m, chi, clo, rr);
-  return s;
-}
-template <>
-__device__ __forceinline__ float vec_expsum_far<float>(uint4 w, float m, float chi, float clo,
-                                                      float rr) {
-  return (term_far(__uint_as_float(w.x), m, chi, clo, rr) +
-          term_far(__uint_as_float(w.y), m, chi, clo, rr)) +
-         (term_far(__uint_as_float(w.z), m, chi, clo, rr) +
-          term_far(__uint_as_float(w.w), m, chi, clo, rr));
-}
 
 // A launch lists at most kMaxListRows rows (the host splits larger calls).
 constexpr int kMaxListRows = 8192;
 constexpr int kRsSmemTotal = kRsSmem + kMaxListRows * (int)sizeof(int);
 static_assert(kRsSmemTotal <= 227 * 1024, "row list and ring exceed shared memory");
-constexpr float kShiftSlack = 64.0f;  // exponents above the shift stay below 2^64
-constexpr float kFarShift = 67108864.0f;  // 2^26: beyond, 2^(m*c - M) itself may overflow
-
-template <typename T> __device__ __forceinline__ uint4 neg_inf_vec();
-template <> __device__ __forceinline__ uint4 neg_inf_vec<__nv_bfloat16>() {
-  return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
-}
-template <> __device__ __forceinline__ uint4 neg_inf_vec<float>() {
-  return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);
-}
 
 template <typename T, typename Rows>
 __global__ void __launch_bounds__(kRsWarps * 32, 1)
@@ -401,20 +254,20 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
       }
     } else {
       const float tm = fmaxf(regs_max<kVpl>(x, (T*)nullptr), tailx);
-      if (tm > mrun) {
-        mrun = tm;
-        // Move the shift on the lane's first finite maximum, or when the
-        // exponents could exceed 2^kShiftSlack.
-        if (!(anchor > -INFINITY) || fmaf(tm, chi, -Msh) > kShiftSlack) {
-          const float Mn = __fmul_rn(tm, chi);
-          if (acc != 0.0) {
-            const double f = exp2((double)Msh - (double)Mn);
-            if constexpr (Rows::kEntropy) acc1 = (acc1 + ((double)anchor - (double)tm) * acc) * f;
-            acc *= f;
-          }
-          anchor = tm;
-          Msh = Mn;
+      if (tm > mrun) mrun = tm;
+      // The lane's shift is an integer at or just above its largest scaled
+      // element, moved (by an exact power of two) as soon as an element
+      // passes it: the largest terms have exponents in (-1, 0], where fp32
+      // rounds them least.
+      const float Mn = ceilf(tm * chi);
+      if (tm > -INFINITY && (!(anchor > -INFINITY) || Mn > Msh)) {
+        if (acc != 0.0) {
+          const double f = pow2i(Msh - Mn);
+          if constexpr (Rows::kEntropy) acc1 = (acc1 + ((double)anchor - (double)tm) * acc) * f;
+          acc *= f;
         }
+        anchor = tm;
+        Msh = Mn;
       }
       const bool has = anchor > -INFINITY;
       float a = 0.0f, a1s = 0.0f;

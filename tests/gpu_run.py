@@ -25,7 +25,7 @@ def to_np(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run_chain_gpu(prob, diag=True, split=False):
+def run_chain_gpu(prob, diag=True, split=False, persistent=False):
     from speculative_decoding_verification_89_b200 import capi
     dev = torch.device("cuda")
     tgt = padded(prob.tgt.to(dev))
@@ -45,8 +45,8 @@ def run_chain_gpu(prob, diag=True, split=False):
         capi.spec_chain_decide(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, st, ws,
                                diag=dg)
     else:
-        capi.spec_verify_chain(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, st, ws,
-                               diag=dg)
+        fn = capi.spec_verify_chain_persistent if persistent else capi.spec_verify_chain
+        fn(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, st, ws, diag=dg)
     torch.cuda.synchronize()
     return (acc.cpu().numpy(), out.cpu().numpy(),
             dg.cpu().numpy() if diag else None, int(st.item()))

@@ -19,7 +19,7 @@ FIELDS = ("acc", "out", "diag", "status", "tables", "seq_lens", "free_stack", "f
           "kv_pool", "hid_out", "hid_off")
 
 
-def _run(prob, state, bufs, fused, base=None, status0=0):
+def _run(prob, state, bufs, fused, base=None, status0=0, persistent=False):
     from speculative_decoding_verification_89_b200 import capi
     dev = "cuda"
     tgt = padded(prob.tgt.to(dev))
@@ -43,9 +43,10 @@ def _run(prob, state, bufs, fused, base=None, status0=0):
     dg = torch.full((B, 4 * K + 2), -7.0, dtype=torch.float64, device=dev)
     s = torch.full((1,), status0, dtype=torch.int32, device=dev)
     if fused:
-        capi.spec_verify_chain_commit(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, t, l,
-                                      b_len, f, top, s, ws, block_size=state.block_size,
-                                      diag=dg, **kw)
+        fn = capi.spec_verify_chain_commit_persistent if persistent else \
+            capi.spec_verify_chain_commit
+        fn(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, t, l, b_len, f, top, s, ws,
+           block_size=state.block_size, diag=dg, **kw)
     else:
         capi.spec_verify_chain(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, s, ws,
                                diag=dg)
