@@ -385,7 +385,7 @@ def run_ours(args, dist):
         result["e2e"] = run_e2e(args, prob, state, bufs, base, dev, dist)
     result["draft_step"] = run_draft_step(args, dev, dist, peak)
     result["outcome_law"] = run_outcome_law(args, prob, dev, dist, peak)
-    result["hier_step"] = run_hier_step(args, dev, dist, peak)
+    result["configs"] = run_configs(args, dev, dist, peak, result)
     if dist.world == 1 and dist.rank == 0:
         rnd = args.warmup + args.steps
         acc1 = torch.empty(B, dtype=torch.int32, device=dev)
@@ -399,7 +399,15 @@ def run_ours(args, dist):
         result["parity_spot_check"] = spot_check(prob, acc1.cpu().numpy(),
                                                  out_tok.cpu().numpy(), rnd)
         if not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(prob, state)
+            cb = cpu_baseline(prob, state)
+            r = oracle_rates("chain_commit")
+            if "all_cores" in r:
+                cb["single_thread_value"] = cb["value"]
+                cb["value"] = r["all_cores"]
+                cb["cores"] = r["cores"]
+                cb["sample"] += (f"; all cores: {r['tasks']} tasks of {r['task']}, one process "
+                                 f"per core, tokens over the busiest process's oracle time")
+            result["cpu_baseline"] = cb
     return result
 
 
@@ -564,72 +572,352 @@ def run_outcome_law(args, prob, dev, dist, peak):
             "gpu_launches_per_call": 3}
 
 
-def run_hier_step(args, dev, dist, peak):
-    """Two-stage verification at the large mixed-temperature shape (B=256,
-    K=N_i=4, V=151936 fp32, 51 greedy sequences), each call from an empty
-    window: stage one always, stage two for the sequences whose window then
-    holds N_i tokens. A call's algorithmic bytes are the logit rows it must
-    read once: stage one K+1 L_i rows, plus K L_d rows for a sampled
-    sequence; stage two W+1 L_f rows per firing sequence, W = a1 + 1. Each
-    call is timed alone (CUDA events around it, the window reset outside)."""
+# ----------------------------------------------------------------------------
+# The other configurations (chain small, two-stage peaked, two-stage mixed,
+# engine loop): per-config throughput at one GPU, each against the oracle's on
+# the host cores (one core, and one process per core)
+# ----------------------------------------------------------------------------
+class HierLoop:
+    """Rolling two-stage verification of B sequences on the device: before
+    every round the rows of slots >= win_len are redrawn (earlier slots keep
+    the rows the window was checked against), drafts come from L_d at the
+    window's next slots, and spec_verify_hier runs on the stream."""
+
+    def __init__(self, B, K, Ni, V, dtype, dev):
+        from speculative_decoding_verification_89_b200 import capi
+        self.capi, self.B, self.K, self.Ni, self.S, self.dev = capi, B, K, Ni, Ni + K + 1, dev
+        i32 = dict(dtype=torch.int32, device=dev)
+        WC = Ni + K
+        self.win_len = torch.zeros(B, **i32)
+        self.win_tok = torch.full((B, WC), -1, **i32)
+        self.win_stat = torch.zeros((B, WC, 2), dtype=torch.float64, device=dev)
+        self.acc1, self.acc2 = torch.empty(B, **i32), torch.empty(B, **i32)
+        self.ctok, self.cn = torch.empty((B, WC + 1), **i32), torch.empty(B, **i32)
+        self.status = torch.zeros(1, **i32)
+        self.ws = capi.workspace(B, K, V, dtype, Ni=Ni, device=dev)
+        self.lg = None
+
+    def logits(self, fresh):
+        """This round's rows: fresh ones for slots >= win_len."""
+        if self.lg is None:
+            self.lg = [x.clone() for x in fresh]
+        else:
+            keep = torch.arange(self.S, device=self.dev).view(1, -1, 1) < \
+                self.win_len.view(-1, 1, 1)
+            self.lg = [torch.where(keep, o, n) for o, n in zip(self.lg, fresh)]
+        return self.lg
+
+    def call(self, drafts, T, seed, seq_id, rnd):
+        lg_d, lg_i, lg_f = self.lg
+        self.capi.spec_verify_hier(lg_d, lg_i, lg_f, self.Ni, drafts, T, seed, seq_id, rnd,
+                                   self.win_len, self.win_tok, self.win_stat, self.acc1,
+                                   self.acc2, self.ctok, self.cn, self.status, self.ws)
+
+    def rows_read(self, w_before, greedy):
+        """Logit rows the call had to read once: stage one K+1 L_i rows and K
+        L_d rows (sampled sequences); stage two W+1 L_f rows where it ran."""
+        a1, a2 = self.acc1.cpu().numpy(), self.acc2.cpu().numpy()
+        st1 = (self.K + 1) + np.where(greedy, 0, self.K)
+        W = w_before + a1 + 1
+        st2 = np.where(a2 >= 0, W + 1, 0)
+        return int(st1.sum() + st2.sum())
+
+
+def _timed(fn):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fn()
+    e1.record()
+    return e0, e1
+
+
+def run_cfg_chain_small(dev):
+    """Chain verification, B=1, K=4, V=1024 fp32, T=1, fresh logits every
+    round for 100 rounds: latency of one spec_verify_chain call."""
     from speculative_decoding_verification_89_b200 import capi
     from speculative_decoding_verification_89_b200 import workloads as W
-    hp = W.hier_mixed(device=dev)
-    Bh, Kh, Ni, Vh = hp.lg_f.shape[0], hp.K, hp.Ni, hp.lg_f.shape[2]
-    WC = Ni + Kh
-    i32 = dict(dtype=torch.int32, device=dev)
-    win_len = torch.zeros(Bh, **i32)
-    win_tok = torch.full((Bh, WC), -1, **i32)
-    win_stat = torch.zeros((Bh, WC, 2), dtype=torch.float64, device=dev)
-    acc1, acc2 = torch.empty(Bh, **i32), torch.empty(Bh, **i32)
-    ctok, cn = torch.empty((Bh, WC + 1), **i32), torch.empty(Bh, **i32)
-    status = torch.zeros(1, **i32)
-    ws = capi.workspace(Bh, Kh, Vh, hp.lg_f.dtype, Ni=Ni, device=dev)
-    # Drafts drawn from the drafting exit L_d at the window's first slots, as
-    # an engine would produce them.
-    drafts = W.window_drafts(hp.lg_d, win_len, Kh, hp.temperature, W.generator(11, dev))
+    probs = [W.chain_small(rnd=r, device=dev) for r in range(100)]
+    ws = capi.workspace(1, 4, 1024, torch.float32, device=dev)
+    acc = torch.empty((100, 1), dtype=torch.int32, device=dev)
+    out = torch.empty((1, 5), dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def call(i):
-        capi.spec_verify_hier(hp.lg_d, hp.lg_i, hp.lg_f, Ni, drafts, hp.temperature, hp.seed,
-                              hp.seq_id, i, win_len, win_tok, win_stat, acc1, acc2, ctok, cn,
-                              status, ws)
+    def call(p, i):
+        capi.spec_verify_chain(p.tgt, p.drf, p.draft_tok, p.temperature, p.seed, p.seq_id, p.rnd,
+                               acc[i], out, st, ws)
 
-    for i in range(max(3, args.warmup)):
-        win_len.zero_()
-        call(i)
-    n = 20
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(n)]
-    a1s, a2s, cns = (torch.empty((n, Bh), **i32) for _ in range(3))
+    for i in range(5):
+        call(probs[i], i)
     torch.cuda.synchronize()
-    dist.barrier()
-    for i in range(n):
-        win_len.zero_()
-        ev[i][0].record()
-        call(1000 + i)
-        ev[i][1].record()
-        a1s[i].copy_(acc1)
-        a2s[i].copy_(acc2)
-        cns[i].copy_(cn)
+    ev = [_timed(lambda i=i: call(probs[i], i)) for i in range(100)]
     torch.cuda.synchronize()
-    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev)
-    ms = dist.reduce(ms, "max")
-    if int(status.item()) != 0:
-        raise RuntimeError(f"two-stage verification: device status {int(status.item())}")
-    greedy = (hp.temperature == 0).cpu().numpy()
-    a1, a2 = a1s.cpu().numpy(), a2s.cpu().numpy()
-    stage1 = ((Kh + 1) + np.where(greedy, 0, Kh)).sum() * n
-    stage2 = np.where(a2 >= 0, a1 + 2, 0).sum()
-    nbytes = int(stage1 + stage2) * Vh * hp.lg_f.element_size()
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    return {"workload": "two-stage verification, B=256, K=N_i=4, V=151936 fp32, 51 greedy "
-                        "sequences, each call from an empty window",
-            "us_per_call": ms * 1e3 / n, "calls": n,
-            "stage_two_sequences_per_call": float((a2 >= 0).sum()) / n,
-            "algorithmic_bytes_per_call": nbytes / n,
-            "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / peak,
-            "committed_tokens_per_s": float(cns.sum().item()) / (ms * 1e-3),
+    us = [a.elapsed_time(b) * 1e3 for a, b in ev]
+    tokens = float((acc.cpu().numpy() + 1).sum())
+    if int(st.item()) != 0:
+        raise RuntimeError("chain small: device status")
+    return {"workload": "chain verification B=1, K=4, V=1024 fp32 (N(0,4) targets, drafts "
+                        "+N(0,1), T=1), fresh logits each of 100 rounds",
+            "us_per_round_median": statistics.median(us), "us_per_round_mean": statistics.mean(us),
+            "tokens_per_s": tokens / (sum(us) * 1e-6), "rounds": 100,
+            "bound": "latency (9 rows of 4 KB; two launches)", "gpu_launches_per_round": 2}
+
+
+def run_cfg_hier(dev, peak, kind, rounds):
+    """Two-stage verification as a rolling loop (the window carries from call
+    to call): kind 'peaked' = B=8, V=32000 bf16, T=0.7 with one greedy
+    sequence; kind 'mixed' = B=256, V=151936 fp32, T ~ U(0, 1.2] with 51
+    greedy sequences. Each call is timed alone (events around it); the row
+    redraw and the drafts are outside."""
+    from speculative_decoding_verification_89_b200 import workloads as W
+    if kind == "peaked":
+        base = W.hier_peaked(device=dev)
+        kw = dict(final_std=2.5, inter_noise=0.7, draft_noise=1.5, boost_p=0.05, boost=6.0)
+        dtype, desc = torch.bfloat16, ("two-stage verification B=8, K=N_i=4, V=32000 bf16, peaked "
+                                       "rows (+6 on 5%), T=0.7 with one greedy sequence")
+    else:
+        base = W.hier_mixed(device=dev)
+        kw = dict(final_std=2.0, inter_noise=0.5, draft_noise=2.0)
+        dtype, desc = torch.float32, ("two-stage verification B=256, K=N_i=4, V=151936 fp32, "
+                                      "T ~ U(0,1.2] with 51 greedy sequences")
+    B, K, Ni, V = base.lg_f.shape[0], base.K, base.Ni, base.lg_f.shape[2]
+    loop = HierLoop(B, K, Ni, V, dtype, dev)
+    T = base.temperature.to(dev)
+    greedy = (base.temperature == 0).cpu().numpy()
+    esz = torch.tensor([], dtype=dtype).element_size()
+    ms = 0.0
+    rows = committed = calls = 0
+    for r in range(rounds + 3):
+        fresh = [base.lg_d, base.lg_i, base.lg_f] if r == 0 else list(
+            W.hier_logits(B, loop.S, V, dtype, W.generator(9000 + r, dev), dev, **kw))
+        loop.logits(fresh)
+        w_before = loop.win_len.cpu().numpy()
+        drafts = W.window_drafts(loop.lg[0], loop.win_len, K, T, W.generator(40 + r, dev))
+        e0, e1 = _timed(lambda: loop.call(drafts, T, base.seed, base.seq_id, r))
+        torch.cuda.synchronize()
+        if r >= 3:  # the first rounds fill the windows
+            ms += e0.elapsed_time(e1)
+            rows += loop.rows_read(w_before, greedy)
+            committed += int(loop.cn.sum().item())
+            calls += 1
+    if int(loop.status.item()) != 0:
+        raise RuntimeError(f"two-stage {kind}: device status")
+    nbytes = rows * V * esz
+    return {"workload": desc + ", rolling windows", "calls": calls,
+            "us_per_call": ms * 1e3 / calls,
+            "committed_tokens_per_s": committed / (ms * 1e-3),
+            "algorithmic_bytes_per_call": nbytes / calls,
+            "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac_of_peak_hbm": nbytes / (ms * 1e-3) / 1e9 / peak,
             "gpu_launches_per_call": 4}
+
+
+def run_cfg_engine(dev, rounds=256):
+    """Engine loop: 64 sequences x 256 rounds, K = N_i = 4, V=32000 bf16,
+    logits regenerated each round from a generator seeded by (4, round); each
+    round reserves the cycle's slots in the block tables, verifies, commits
+    the committed tokens and rolls the reservation back (block 16, pool of
+    65536 blocks, starts U[128, 2048]). Committed tokens per second of the
+    device work, with and without the round's logit generation."""
+    from speculative_decoding_verification_89_b200 import capi
+    from speculative_decoding_verification_89_b200 import workloads as W
+    B, K, Ni, V = 64, 4, 4, 32000
+    S = Ni + K + 1
+    ctx = W.context_lengths(B, 128, 2048, seed=4)
+    max_blocks = (max(ctx) + rounds * S + S) // 16 + 2
+    state = W.paged_state(ctx, 16, max_blocks, 65536, device=dev)
+    committed = state.seq_lens.clone()
+    T = torch.ones(B, device=dev)
+    seq_id = torch.arange(B, dtype=torch.int32, device=dev)
+    full = torch.full((B,), S, dtype=torch.int32, device=dev)
+    loop = HierLoop(B, K, Ni, V, torch.bfloat16, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    ms_work = ms_all = 0.0
+    total = 0
+    for r in range(rounds):
+        a0 = torch.cuda.Event(enable_timing=True)
+        a0.record()
+        fresh, _ = W.engine_round_logits(B, S, V, r, dev)
+        loop.logits(fresh)
+        w0 = torch.cuda.Event(enable_timing=True)
+        w0.record()
+        capi.spec_commit_paged(state.tables, state.seq_lens, committed, full, 0,
+                               state.free_stack, state.free_top, S, st, block_size=16)
+        drafts = W.window_drafts(loop.lg[0], loop.win_len, K, T, W.generator(40 + r, dev))
+        loop.call(drafts, T, 4, seq_id, r)
+        capi.spec_commit_paged(state.tables, state.seq_lens, committed, loop.cn, 0,
+                               state.free_stack, state.free_top, S, st, block_size=16)
+        committed.copy_(state.seq_lens)
+        w1 = torch.cuda.Event(enable_timing=True)
+        w1.record()
+        torch.cuda.synchronize()
+        ms_work += w0.elapsed_time(w1)
+        ms_all += a0.elapsed_time(w1)
+        total += int(loop.cn.sum().item())
+    if int(st.item()) != 0 or int(loop.status.item()) != 0:
+        raise RuntimeError("engine loop: device status")
+    return {"workload": "engine loop 64 sequences x 256 rounds, K=N_i=4, V=32000 bf16, paged "
+                        "commit/rollback every round (block 16, pool 65536)",
+            "rounds": rounds, "committed_tokens": total,
+            "committed_tokens_per_s": total / (ms_work * 1e-3),
+            "committed_tokens_per_s_with_logit_generation": total / (ms_all * 1e-3),
+            "ms_per_round": ms_work / rounds, "ms_per_round_with_logit_generation": ms_all / rounds}
+
+
+# ----------------------------------------------------------------------------
+# Oracle throughput per configuration on the host cores
+# ----------------------------------------------------------------------------
+ORACLE_CFG = {
+    # kind: (description of one task, tasks per process)
+    "chain_small": ("20 rounds of B=1, K=4, V=1024 chain verification", 2),
+    "hier_peaked": ("one sequence, 6 rolling two-stage rounds, K=N_i=4, V=32000, peaked rows", 2),
+    "chain_commit": ("one sequence-round of B=64-shape chain verification (K=8, V=128256) "
+                     "plus its paged commit", 2),
+    "hier_mixed": ("one sequence, 8 rolling two-stage rounds, K=N_i=4, V=151936", 1),
+    "engine": ("one sequence, 8 rolling two-stage rounds with paged commit, K=N_i=4, V=32000", 2),
+}
+
+
+def _softmax_draw(rows, T, rng):
+    """Drafts by the Gumbel-max construction from rows [n, V] at temperature T."""
+    if T == 0.0:
+        return rows.argmax(axis=1)
+    g = -np.log(-np.log(rng.random(rows.shape)))
+    return (rows / T + g).argmax(axis=1)
+
+
+def _oracle_task(job):
+    """One task of oracle work on inputs drawn (numpy) with the recipe of the
+    configuration; returns (pid, tokens, seconds spent in the oracle)."""
+    kind, i = job
+    from oracle.commit import commit_paged
+    from oracle.philox import STAGE_ONE, STAGE_TWO, PhiloxUniforms
+    from oracle.verify import verify_chain, verify_hier_seq
+    rng = np.random.default_rng(7000 + 13 * i + len(kind))
+    tok, sec = 0, 0.0
+
+    def hier_rounds(V, rounds, fstd, inoise, dnoise, T, boost=0.0, commit=False):
+        nonlocal tok, sec
+        K, Ni = 4, 4
+        S = Ni + K + 1
+        lf = rng.normal(0, fstd, (S, V))
+        if boost:
+            lf += boost * (rng.random((S, V)) < 0.05)
+        rows = [lf + rng.normal(0, dnoise, (S, V)), lf + rng.normal(0, inoise, (S, V)), lf]
+        window = []
+        length = int(rng.integers(128, 2048))
+        table = np.arange((length + S * rounds) // 16 + 4, dtype=np.int64)
+        for r in range(rounds):
+            w = len(window)
+            fresh_f = rng.normal(0, fstd, (S, V))
+            fresh = [fresh_f + rng.normal(0, dnoise, (S, V)), fresh_f + rng.normal(0, inoise, (S, V)),
+                     fresh_f]
+            for e in range(3):
+                rows[e][w:] = fresh[e][w:]
+            drafts = _softmax_draw(rows[0][w:w + K], T, rng)
+            t0 = time.perf_counter()
+            res = verify_hier_seq(rows[0], rows[1], rows[2], drafts, T, window, Ni,
+                                  PhiloxUniforms(5, i, r, STAGE_ONE),
+                                  PhiloxUniforms(5, i, r, STAGE_TWO))
+            n = len(res.committed)
+            if commit:
+                stack = np.zeros(1064, dtype=np.int64)
+                stack[:64] = np.arange(1000, 1064)
+                commit_paged(table[None, :], np.array([length + S]), np.array([length]),
+                             np.array([n]), stack, 64, 16, 1064, S)
+            sec += time.perf_counter() - t0
+            tok += n
+            length += n
+            window = list(res.window) if res.stage2 is None else []
+
+    if kind == "chain_small":
+        for r in range(20):
+            tgt = rng.normal(0, 2, (1, 5, 1024))
+            drf = tgt[:, :4] + rng.normal(0, 1, (1, 4, 1024))
+            drafts = _softmax_draw(drf[0], 1.0, rng)[None, :]
+            t0 = time.perf_counter()
+            res = verify_chain(tgt, drf, drafts, np.array([1.0]), 0, np.array([i]), r)
+            sec += time.perf_counter() - t0
+            tok += res[0].accepted + 1
+    elif kind == "chain_commit":
+        V = 128256
+        prior = -1.1 * np.log(np.arange(V) + 1.0)
+        tgt = (rng.normal(0, 2, (1, 9, V)) + prior).astype(np.float32).astype(np.float64)
+        drf = (tgt[:, :8] + rng.normal(0, 1, (1, 8, V))).astype(np.float32).astype(np.float64)
+        drafts = _softmax_draw(drf[0], 1.0, rng)[None, :]
+        length = int(rng.integers(512, 4096))
+        tabs = np.arange((length + 9) // 16 + 2, dtype=np.int64)[None, :]
+        t0 = time.perf_counter()
+        res = verify_chain(tgt, drf, drafts, np.array([1.0]), 2, np.array([i]), 0)[0]
+        stack = np.zeros(1032, dtype=np.int64)
+        stack[:32] = np.arange(1000, 1032)
+        commit_paged(tabs, np.array([length]), np.array([length]), np.array([res.accepted + 1]),
+                     stack, 32, 16, 1032, 9)
+        sec += time.perf_counter() - t0
+        tok += res.accepted + 1
+    elif kind == "hier_peaked":
+        hier_rounds(32000, 6, 2.5, 0.7, 1.5, 0.7, boost=6.0)
+    elif kind == "hier_mixed":
+        hier_rounds(151936, 8, 2.0, 0.5, 2.0, float(rng.uniform(0.05, 1.2)))
+    elif kind == "engine":
+        hier_rounds(32000, 8, 2.0, 0.5, 1.0, 1.0, commit=True)
+    return os.getpid(), tok, sec
+
+
+_POOL = None
+
+
+def start_oracle_pool():
+    """A process pool for the oracle, forked before any GPU call (a process
+    forked after CUDA starts would hang); one process per host core, at most
+    64."""
+    global _POOL
+    import multiprocessing as mp
+    n = max(1, min(os.cpu_count() or 1, 64))
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    _POOL = mp.get_context("fork").Pool(n)
+    return n
+
+
+def oracle_rates(kind):
+    """Oracle tokens per second for one configuration: single-threaded (tasks
+    run in turn in this process), and with one process per core (tokens over
+    the busiest process's oracle time)."""
+    desc, per = ORACLE_CFG[kind]
+    one = [_oracle_task((kind, 10_000 + k)) for k in range(per)]
+    r1 = sum(t for _, t, _ in one) / max(sum(s for _, _, s in one), 1e-9)
+    out = {"unit": "tokens/s", "kind": "oracle", "task": desc, "single_thread": r1}
+    if _POOL is not None:
+        procs = _POOL._processes
+        res = _POOL.map(_oracle_task, [(kind, k) for k in range(procs * per)])
+        busy = {}
+        for pid, _, sec in res:
+            busy[pid] = busy.get(pid, 0.0) + sec
+        out["all_cores"] = sum(t for _, t, _ in res) / max(max(busy.values()), 1e-9)
+        out["cores"] = procs
+        out["tasks"] = len(res)
+    return out
+
+
+def run_configs(args, dev, dist, peak, head):
+    """Every configuration at one GPU: config 1 (latency), 2 and 4 (rolling
+    two-stage loops), 3 (the headline step above), 5 (engine loop), each with
+    the oracle's throughput on one host core and on all of them."""
+    with_oracle = dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline
+    out = {
+        "cfg1_chain_small": run_cfg_chain_small(dev),
+        "cfg2_hier_peaked": run_cfg_hier(dev, peak, "peaked", rounds=24),
+        "cfg3_chain_commit": {"workload": "the headline step", "tokens_per_s": head["value"],
+                              "ms_per_step": head["ms_per_step"], "hbm_gbs": head["hbm_gbs"],
+                              "frac_of_peak_hbm": head["hbm_frac_of_measured"]},
+        "cfg4_hier_mixed": run_cfg_hier(dev, peak, "mixed", rounds=10),
+        "cfg5_engine_loop": run_cfg_engine(dev),
+    }
+    if with_oracle:
+        for key, kind in (("cfg1_chain_small", "chain_small"), ("cfg2_hier_peaked", "hier_peaked"),
+                          ("cfg3_chain_commit", "chain_commit"), ("cfg4_hier_mixed", "hier_mixed"),
+                          ("cfg5_engine_loop", "engine")):
+            out[key]["oracle"] = oracle_rates(kind)
+    return out
 
 
 def run_e2e(args, prob, state, bufs, base, dev, dist):
@@ -733,12 +1021,17 @@ def main():
         if dist.rank == 0:
             print(json.dumps(run_reference(args, dist)), flush=True)
         return 0
+    if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
+        start_oracle_pool()  # before the first GPU call
     dist.init("nccl")
     try:
         res = run_ours(args, dist)
         if dist.rank == 0:
             print(json.dumps(res), flush=True)
     finally:
+        if _POOL is not None:
+            _POOL.terminate()
+            _POOL.join()
         dist.close()
     return 0
 
