@@ -86,6 +86,10 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 #define SPEC_MAX_V (1 << 21)     /* vocabulary size                   */
 #define SPEC_MAX_COMMIT_B 16384  /* sequences per paged commit        */
 #define SPEC_MAX_FUSED_B 4096    /* sequences per fused verify+commit */
+#define SPEC_MAX_CACHED 1024     /* cached tokens per sequence (Saguaro) */
+#define SPEC_VP_MAX_RANKS 64     /* vocabulary shards (ranks)         */
+#define SPEC_VP_ROW_BYTES 32     /* one row record of a shard         */
+#define SPEC_VP_MASS_BYTES 16    /* one sequence's draw masses of a shard */
 
 /* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
  * chain call, Ni > 0 a two-stage call. Returns 0 for invalid sizes. */
@@ -421,6 +425,109 @@ int spec_verify_chain_noalloc(const void* tgt, int64_t ld_tgt, const void* drf,
                               uint64_t seed, const int32_t* seq_id, uint32_t round,
                               int32_t* accept_len, int32_t* out_tok, double* diag,
                               int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Saguaro sampling ([SSD] Technische Zusammenfassung 3.B): lower the draft
+ * probability of the tokens held in the speculation cache, so a rejection's
+ * residual (proportional to the target-minus-draft difference) lands on them
+ * more often. The lowered draft law is q'(v) proportional to
+ * q(v) (1 - eps [v cached]); at temperature T > 0 that is the softmax of the
+ * draft logits with T ln(1 - eps) added to the cached tokens, which this call
+ * adds IN PLACE to every draft row of each sequence. Run it on the drafting
+ * exit's rows before spec_draft_sample and the verification: both then use
+ * q' as the draft law and the check stays lossless.
+ *
+ * logits      : draft rows [B, rows_per_seq, V] (in/out); row (b, r) starts
+ *               at element (b * rows_per_seq + r) * ld. The rows of a chain
+ *               check are [B, K, V] (rows_per_seq = K); those of the draft
+ *               step [B, V] (rows_per_seq = 1).
+ * dtype       : SPEC_F32 or SPEC_BF16. The shift float32(T * ln(1 - eps))
+ *               is added in float32 and the sum rounded to the rows' type.
+ * cached      : int32 token ids, [B, n_cached] (per_row = 0: one list per
+ *               sequence, lowered in each of its rows) or
+ *               [B, rows_per_seq, n_cached] (per_row = 1: one list per row,
+ *               e.g. the bonus tokens prepared for that position). Ids
+ *               outside [0, V) are padding; an id repeated within a list is
+ *               lowered once.
+ * n_cached    : 0 .. SPEC_MAX_CACHED ids per list.
+ * per_row     : 0 or 1, as above.
+ * eps         : the lowering, 0 <= eps < 1 (0: nothing to do).
+ * temperature : float [B]; sequences at 0 (greedy) or with an invalid
+ *               temperature are left unchanged.
+ * Returns SPEC_EINVAL for bad sizes, dtype, per_row or eps (nothing
+ * launched); SPEC_ECUDA if the launch fails.
+ * ------------------------------------------------------------------------- */
+int spec_saguaro_adjust(void* logits, int64_t ld, int dtype, int B, int rows_per_seq, int V,
+                        const int32_t* cached, int n_cached, int per_row, double eps,
+                        const float* temperature, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Vocabulary-parallel chain verification. The check of spec_verify_chain
+ * (speculative sampling as HiSpec, gist.science summary of arXiv 2510.01336,
+ * section 2 "Verlustfreie Garantie", appeals to it; residual per Speculative
+ * Speculative Decoding, Technische Zusammenfassung 3.B) for rows split over
+ * the vocabulary: rank r of R holds the columns [v0, v0 + Vs) of every target
+ * and draft row (e.g. the output of a vocabulary-parallel LM head) and no
+ * rank ever holds a whole row. The partition functions, greedy argmaxes and
+ * residual masses are sums or maxima over the vocabulary, so the ranks
+ * exchange small records instead of rows. Per call, on every rank in the same
+ * order (the exchanges are the caller's collectives, e.g. NCCL):
+ *
+ *   spec_vp_shard_stats -> rows_out [B, 2K+1] records
+ *   all-gather rows_out in rank order       -> rows_all [R, B, 2K+1]
+ *   spec_vp_decide      -> mass_out [B]     (every rank: same accepted counts)
+ *   all-gather mass_out in rank order       -> mass_all [R, B]
+ *   spec_vp_pick        -> accept_len [B], out_tok [B, K+1] (-1 at the drawn
+ *                          position unless this rank drew it), diag
+ *   max-reduce out_tok over the ranks       -> the tokens of spec_verify_chain
+ *
+ * The outputs follow spec_verify_chain's rule on the same Philox counters;
+ * they differ from a one-GPU call only where the order of the sums moves a
+ * decision (fp64 margin below 1e-6). The records are opaque bytes
+ * (SPEC_VP_ROW_BYTES, SPEC_VP_MASS_BYTES each, 8-byte aligned).
+ *
+ * Common arguments:
+ * tgt, ld_tgt : this rank's target columns [B, K+1, Vs], row stride ld_tgt
+ *               >= Vs elements; rows 16-byte aligned.
+ * drf, ld_drf : its draft columns [B, K, Vs] (may be NULL when K == 0).
+ * Vs, v0, V   : the shard [v0, v0 + Vs) of the vocabulary [0, V); the R
+ *               shards must cover [0, V) without overlap (a drafted id that
+ *               no shard holds flags the sequence).
+ * R, rank     : 1 <= R <= SPEC_VP_MAX_RANKS, 0 <= rank < R.
+ * draft_tok, temperature, seed, seq_id, round, diag: as spec_verify_chain;
+ *               diag is written identically by every rank.
+ * ws          : spec_vp_workspace_bytes(B, K, Vs, dtype) bytes, 256-byte
+ *               aligned, kept by the caller from spec_vp_shard_stats through
+ *               spec_vp_pick of the same call.
+ * Errors: SPEC_EINVAL / SPEC_EWORKSPACE on the host before any launch;
+ * sequences with invalid values get accept_len = -1, out_tok = -1 and
+ * SPEC_EDEVICE in dev_status on every rank alike.
+ * ------------------------------------------------------------------------- */
+size_t spec_vp_workspace_bytes(int B, int K, int Vs, int dtype);
+int spec_vp_shard_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                        int dtype, int B, int K, int Vs, int v0, int V,
+                        const int32_t* draft_tok, const float* temperature, void* rows_out,
+                        int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);
+int spec_vp_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                   int B, int K, int Vs, int v0, int V, int R, int rank, const void* rows_all,
+                   const int32_t* draft_tok, const float* temperature, uint64_t seed,
+                   const int32_t* seq_id, uint32_t round, void* mass_out, double* diag,
+                   int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);
+int spec_vp_pick(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                 int B, int K, int Vs, int v0, int V, int R, int rank, const void* mass_all,
+                 const int32_t* draft_tok, const float* temperature, int32_t* accept_len,
+                 int32_t* out_tok, double* diag, int32_t* dev_status, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/* Test hook (no counterpart in the paper): the limit of the row-statistics
+ * kernel's waits for its tile copies on the current device, in nanoseconds
+ * (2e9 by default). 0 makes every such wait one non-blocking test, so a copy
+ * still in flight makes it run out: the kernel then records SPEC_ETIMEOUT in
+ * dev_status, waits (2 s at most) for its copies in flight and returns; a
+ * commit in the same call changes nothing. Lets a test exercise the timeout
+ * path without any hang; set it back to 2000000000 afterwards. It is a
+ * device-wide setting: calls on other streams see it too. */
+int spec_test_set_wait_limit_ns(uint64_t ns);
 
 /* Test hook of spec_verify_chain_noalloc (no counterpart in the paper):
  * forgets every kept scratch address and makes the next n address lookups

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libspecverify.so")
 SOURCES = ["row_stats.cu", "step.cu", "decide.cu", "draft.cu", "outcome.cu", "commit.cu",
-           "capi.cu", "noalloc.cu"]
+           "saguaro.cu", "vocab.cu", "capi.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.cuh", "draw.cuh", "commit.cuh", "rowmath.cuh"]
 
 NVCC_FLAGS = [

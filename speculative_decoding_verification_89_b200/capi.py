@@ -58,7 +58,16 @@ _SIGS = {
     "spec_last_cuda_error": (ctypes.c_char_p, []),
     "spec_verify_chain_noalloc": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _u64, _p,
                                        _u32, _p, _p, _p, _p, _p]),
+    "spec_saguaro_adjust": (_i, [_p, _i64, _i, _i, _i, _i, _p, _i, _i, ctypes.c_double, _p, _p]),
+    "spec_vp_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "spec_vp_shard_stats": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p,
+                                 _sz, _p]),
+    "spec_vp_decide": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p,
+                            _u64, _p, _u32, _p, _p, _p, _p, _sz, _p]),
+    "spec_vp_pick": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p,
+                          _p, _p, _p, _p, _sz, _p]),
     "spec_noalloc_test_fail_lookups": (_i, [_i]),
+    "spec_test_set_wait_limit_ns": (_i, [_u64]),
     "spec_draft_workspace_bytes": (_sz, [_i, _i, _i]),
     "spec_outcome_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spec_outcome_law": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p,
@@ -191,6 +200,53 @@ def spec_chain_decide(tgt, drf, draft_tok, temperature, seed, seq_id, rnd, accep
     _check("spec_chain_decide", rc)
 
 
+VP_ROW_BYTES, VP_MASS_BYTES, VP_MAX_RANKS = 32, 16, 64
+
+
+def spec_vp_workspace_bytes(B, K, Vs, dtype):
+    code = dtype if isinstance(dtype, int) else (SPEC_BF16 if dtype == torch.bfloat16 else SPEC_F32)
+    return int(_lib.spec_vp_workspace_bytes(B, K, Vs, code))
+
+
+def _vp_common(tgt, drf):
+    B, Kp1, Vs = tgt.shape
+    K = Kp1 - 1
+    return (_ptr(tgt), _rows(tgt, Kp1), _ptr(drf) if K > 0 else None,
+            _rows(drf, K) if K > 0 else 0, _dtype_code(tgt), B, K, Vs)
+
+
+def spec_vp_shard_stats(tgt, drf, v0, V, draft_tok, temperature, rows_out, dev_status, ws,
+                        stream=None):
+    """Shard records of the vocabulary-parallel check. tgt [B, K+1, Vs] and
+    drf [B, K, Vs]: this rank's columns [v0, v0+Vs) of the rows; rows_out:
+    uint8 [B, 2K+1, VP_ROW_BYTES]."""
+    rc = _lib.spec_vp_shard_stats(*_vp_common(tgt, drf), v0, V, _ptr(draft_tok),
+                                  _ptr(temperature), _ptr(rows_out), _ptr(dev_status), _ptr(ws),
+                                  ws.numel(), _stream(stream))
+    _check("spec_vp_shard_stats", rc)
+
+
+def spec_vp_decide(tgt, drf, v0, V, R, rank, rows_all, draft_tok, temperature, seed, seq_id, rnd,
+                   mass_out, dev_status, ws, diag=None, stream=None):
+    """rows_all: uint8 [R, B, 2K+1, VP_ROW_BYTES] (every rank's records in rank
+    order); mass_out: uint8 [B, VP_MASS_BYTES]."""
+    rc = _lib.spec_vp_decide(*_vp_common(tgt, drf), v0, V, R, rank, _ptr(rows_all),
+                             _ptr(draft_tok), _ptr(temperature), seed, _ptr(seq_id), rnd,
+                             _ptr(mass_out), _ptr(diag), _ptr(dev_status), _ptr(ws), ws.numel(),
+                             _stream(stream))
+    _check("spec_vp_decide", rc)
+
+
+def spec_vp_pick(tgt, drf, v0, V, R, rank, mass_all, draft_tok, temperature, accept_len, out_tok,
+                 dev_status, ws, diag=None, stream=None):
+    """mass_all: uint8 [R, B, VP_MASS_BYTES]; out_tok int32 [B, K+1] holds -1 at
+    the drawn position unless this rank drew it (max-reduce over ranks)."""
+    rc = _lib.spec_vp_pick(*_vp_common(tgt, drf), v0, V, R, rank, _ptr(mass_all),
+                           _ptr(draft_tok), _ptr(temperature), _ptr(accept_len), _ptr(out_tok),
+                           _ptr(diag), _ptr(dev_status), _ptr(ws), ws.numel(), _stream(stream))
+    _check("spec_vp_pick", rc)
+
+
 def spec_verify_hier(lg_d, lg_i, lg_f, Ni, draft_tok, temperature, seed, seq_id, rnd,
                      win_len, win_tok, win_stat, acc1, acc2, commit_tok, commit_n,
                      dev_status, ws, diag=None, stream=None):
@@ -275,6 +331,27 @@ def spec_chain_decide_commit(tgt, drf, draft_tok, temperature, seed, seq_id, rnd
 def spec_verify_chain_commit_persistent(*args, **kw):
     """spec_verify_chain_commit on the persistent kernel (same arguments)."""
     spec_verify_chain_commit(*args, _entry="spec_verify_chain_commit_persistent", **kw)
+
+
+def spec_saguaro_adjust(logits, cached, eps, temperature, stream=None):
+    """Saguaro sampling: lower the cached tokens of the draft rows in place.
+    logits: [B, n, V] (or [B, V]) float32/bfloat16 with contiguous, evenly
+    spaced rows; cached: int32 on the device, [B, n_cached] (one list per
+    sequence) or [B, n, n_cached] (one list per row); ids outside [0, V) pad;
+    temperature: float [B]."""
+    lg = logits if logits.dim() == 3 else logits.unsqueeze(1)
+    B, n, V = lg.shape
+    ld = lg.stride(1) if n > 1 else lg.stride(0)
+    if lg.stride(2) != 1 or (B > 1 and lg.stride(0) != n * ld):
+        raise ValueError("logits must be [B, n, V] with evenly spaced contiguous rows")
+    per_row = 1 if cached.dim() == 3 else 0
+    if cached.dtype != torch.int32 or not cached.is_contiguous() or cached.shape[0] != B or \
+            (per_row and cached.shape[1] != n):
+        raise ValueError("cached must be contiguous int32 [B, n_cached] or [B, n, n_cached]")
+    rc = _lib.spec_saguaro_adjust(_ptr(lg), ld, _dtype_code(lg), B, n, V, _ptr(cached),
+                                  cached.shape[-1], per_row, float(eps), _ptr(temperature),
+                                  _stream(stream))
+    _check("spec_saguaro_adjust", rc)
 
 
 def spec_philox_uniforms(seed, ctr, out, stream=None):

@@ -2,6 +2,7 @@
 // the launch sequence of each call. Declarations and the contract of every
 // entry point are in include/spec_verify.h.
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 
@@ -83,6 +84,21 @@ bool outcome_layout(int B, int K, int V, int dtype, int n_top, OutcomeLayout* O)
   O->cw = O->zk + align_up(slots * sizeof(double));
   O->cv = O->cw + align_up(slots * (size_t)n_top * sizeof(float));
   O->total = O->cv + align_up(slots * (size_t)n_top * sizeof(int));
+  return true;
+}
+
+// Vocabulary-parallel workspace (one rank): the chain layout of the shard
+// rows (partials, residual tile sums), then the per-sequence states and the
+// prefixes of the tile sums.
+struct VpLayout {
+  Layout L;
+  size_t seq, pre, total;
+};
+bool vp_layout(int B, int K, int Vs, int dtype, VpLayout* P) {
+  if (!layout(B, K, Vs, dtype, 0, &P->L)) return false;
+  P->seq = P->L.total;
+  P->pre = P->seq + align_up((size_t)B * sizeof(VpSeq));
+  P->total = P->pre + align_up((size_t)B * residual_tiles(Vs) * sizeof(double));
   return true;
 }
 
@@ -264,6 +280,59 @@ static int commit_args(int B, int block_size, int max_blocks, int32_t* block_tab
 }
 
 #pragma GCC visibility push(default)
+namespace {
+
+struct VpCheck {
+  VpLayout P;
+  int rc;
+};
+
+VpCheck check_vp(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                 int B, int K, int Vs, int v0, int V, int R, int rank,
+                 const int32_t* draft_tok, const float* temperature, void* ws,
+                 size_t ws_bytes) {
+  VpCheck c{};
+  c.rc = SPEC_EINVAL;
+  if (!vp_layout(B, K, Vs, dtype, &c.P)) return c;
+  if (V < 1 || V > SPEC_MAX_V || v0 < 0 || v0 > V - Vs) return c;
+  if (R < 1 || R > SPEC_VP_MAX_RANKS || rank < 0 || rank >= R) return c;
+  if (B == 0) { c.rc = SPEC_OK; return c; }
+  if (!rows_ok(tgt, ld_tgt, Vs, dtype) || !temperature) return c;
+  if (K > 0 && (!rows_ok(drf, ld_drf, Vs, dtype) || !draft_tok)) return c;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < c.P.total) { c.rc = SPEC_EWORKSPACE; return c; }
+  c.rc = SPEC_OK;
+  return c;
+}
+
+VpArgs vp_args(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype, int B,
+               int K, int Vs, int v0, int V, int R, int rank, const int32_t* draft_tok,
+               const float* temperature, int32_t* dev_status, void* ws, const VpLayout& P) {
+  VpArgs a{};
+  const int es = elem_size(dtype);
+  a.B = B;
+  a.K = K;
+  a.Vs = Vs;
+  a.v0 = v0;
+  a.V = V;
+  a.R = R;
+  a.rank = rank;
+  a.tgt = (const unsigned char*)tgt;
+  a.drf = (const unsigned char*)drf;
+  a.ld_tgt = ld_tgt * es;
+  a.ld_drf = ld_drf * es;
+  a.draft_tok = draft_tok;
+  a.temperature = temperature;
+  a.part = reinterpret_cast<const Partial*>((char*)ws + P.L.part);
+  a.ntiles = stat_tiles(Vs, dtype);
+  a.seq = reinterpret_cast<VpSeq*>((char*)ws + P.seq);
+  a.tsum = reinterpret_cast<double*>((char*)ws + P.L.tsum);
+  a.pre = reinterpret_cast<double*>((char*)ws + P.pre);
+  a.status = dev_status;
+  return a;
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t spec_workspace_bytes(int B, int K, int V, int dtype, int Ni) {
@@ -649,6 +718,95 @@ int spec_outcome_law(const void* tgt, int64_t ld_tgt, const void* drf, int64_t l
   a.top_prob = top_prob;
   a.status = dev_status;
   return cuda_status(launch_outcome(dtype, a, st));
+}
+
+int spec_saguaro_adjust(void* logits, int64_t ld, int dtype, int B, int rows_per_seq, int V,
+                        const int32_t* cached, int n_cached, int per_row, double eps,
+                        const float* temperature, void* stream) {
+  if (B < 0 || rows_per_seq < 0 || V < 1 || V > SPEC_MAX_V || n_cached < 0 ||
+      n_cached > SPEC_MAX_CACHED || (per_row != 0 && per_row != 1))
+    return SPEC_EINVAL;
+  if (dtype != SPEC_F32 && dtype != SPEC_BF16) return SPEC_EINVAL;
+  if (!(eps >= 0.0 && eps < 1.0)) return SPEC_EINVAL;
+  if (B == 0 || n_cached == 0 || rows_per_seq == 0 || eps == 0.0) return SPEC_OK;
+  if (!logits || ld < V || !cached || !temperature) return SPEC_EINVAL;
+  return cuda_status(launch_saguaro_adjust(
+      dtype, (unsigned char*)logits, ld * elem_size(dtype), B, rows_per_seq, V, cached, n_cached,
+      per_row, std::log1p(-eps), temperature, (cudaStream_t)stream));
+}
+
+// ---------------------------------------------------------------------------
+// Vocabulary-parallel chain verification
+// ---------------------------------------------------------------------------
+size_t spec_vp_workspace_bytes(int B, int K, int Vs, int dtype) {
+  VpLayout P;
+  if (!vp_layout(B, K, Vs, dtype, &P)) return 0;
+  return P.total;
+}
+
+int spec_vp_shard_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                        int dtype, int B, int K, int Vs, int v0, int V,
+                        const int32_t* draft_tok, const float* temperature, void* rows_out,
+                        int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  const VpCheck ck = check_vp(tgt, ld_tgt, drf, ld_drf, dtype, B, K, Vs, v0, V, 1, 0, draft_tok,
+                              temperature, ws, ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!rows_out || !aligned(rows_out, 8)) return SPEC_EINVAL;
+  const cudaStream_t st = (cudaStream_t)stream;
+  ChainRows rows;
+  rows.tgt = (const unsigned char*)tgt;
+  rows.drf = (const unsigned char*)drf;
+  rows.ld_tgt = ld_tgt * elem_size(dtype);
+  rows.ld_drf = ld_drf * elem_size(dtype);
+  rows.temperature = temperature;
+  rows.K = K;
+  rows.late_pos = 0;
+  const RsBuffers rb = rs_buffers(ws, ck.P.L);
+  cudaError_t e = launch_row_stats(dtype, rows, B * (2 * K + 1), Vs, rb, dev_status, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  VpArgs a = vp_args(tgt, ld_tgt, drf, ld_drf, dtype, B, K, Vs, v0, V, 1, 0, draft_tok,
+                     temperature, dev_status, ws, ck.P);
+  a.rows = reinterpret_cast<VpRow*>(rows_out);
+  return cuda_status(launch_vp_records(dtype, a, st));
+}
+
+int spec_vp_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                   int B, int K, int Vs, int v0, int V, int R, int rank, const void* rows_all,
+                   const int32_t* draft_tok, const float* temperature, uint64_t seed,
+                   const int32_t* seq_id, uint32_t round, void* mass_out, double* diag,
+                   int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  const VpCheck ck = check_vp(tgt, ld_tgt, drf, ld_drf, dtype, B, K, Vs, v0, V, R, rank,
+                              draft_tok, temperature, ws, ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!rows_all || !aligned(rows_all, 8) || !mass_out || !aligned(mass_out, 8) || !seq_id)
+    return SPEC_EINVAL;
+  VpArgs a = vp_args(tgt, ld_tgt, drf, ld_drf, dtype, B, K, Vs, v0, V, R, rank, draft_tok,
+                     temperature, dev_status, ws, ck.P);
+  a.rows_all = reinterpret_cast<const VpRow*>(rows_all);
+  a.mass = reinterpret_cast<VpMass*>(mass_out);
+  a.seed = seed;
+  a.seq_id = seq_id;
+  a.round = round;
+  a.diag = diag;
+  return cuda_status(launch_vp_decide(dtype, a, (cudaStream_t)stream));
+}
+
+int spec_vp_pick(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                 int B, int K, int Vs, int v0, int V, int R, int rank, const void* mass_all,
+                 const int32_t* draft_tok, const float* temperature, int32_t* accept_len,
+                 int32_t* out_tok, double* diag, int32_t* dev_status, void* ws, size_t ws_bytes,
+                 void* stream) {
+  const VpCheck ck = check_vp(tgt, ld_tgt, drf, ld_drf, dtype, B, K, Vs, v0, V, R, rank,
+                              draft_tok, temperature, ws, ws_bytes);
+  if (ck.rc != SPEC_OK || B == 0) return ck.rc;
+  if (!mass_all || !aligned(mass_all, 8) || !accept_len || !out_tok) return SPEC_EINVAL;
+  VpArgs a = vp_args(tgt, ld_tgt, drf, ld_drf, dtype, B, K, Vs, v0, V, R, rank, draft_tok,
+                     temperature, dev_status, ws, ck.P);
+  a.mass_all = reinterpret_cast<const VpMass*>(mass_all);
+  a.accept_len = accept_len;
+  a.out_tok = out_tok;
+  a.diag = diag;
+  return cuda_status(launch_vp_pick(dtype, a, (cudaStream_t)stream));
 }
 
 const char* spec_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }

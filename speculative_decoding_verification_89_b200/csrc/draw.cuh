@@ -193,11 +193,12 @@ __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const Pr
 
 // Leader: given all tile sums in shared memory (tsum), prefix them in a fixed
 // order, locate u * Z, rescan that tile and return the drawn token in every
-// thread (-1 if the weights have no mass). *Z_out gets Z.
+// thread (-1 if the weights have no mass). *Z_out gets Z. A caller that owns
+// one piece of a longer row passes its own target (>= 0) instead of u * Z.
 template <typename T>
 __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef& kp,
                              const ProbCoef& kq, const double* tsum, double* pre, int nrt,
-                             float u, double* Z_out) {
+                             float u, double* Z_out, double target_in = -1.0) {
   __shared__ double s_wtot[kDecWarps];
   __shared__ int s_tile, s_tok;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -226,7 +227,7 @@ __device__ int residual_pick(const T* prow, const T* qrow, int V, const ProbCoef
   }
   *Z_out = Z;
   if (!(Z > 0.0)) return -1;
-  const double target = (double)u * Z;
+  const double target = target_in >= 0.0 ? target_in : (double)u * Z;
   // The last tile with mass whose prefix does not exceed the target.
   c += excl;
   int cand = -1;

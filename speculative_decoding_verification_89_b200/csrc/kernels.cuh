@@ -115,9 +115,10 @@ struct RsBuffers {
 };
 
 // Combine a row's tile partials (warp-cooperative; result valid in lane 0).
-// Up to 4*32 tiles are read once into registers; longer rows loop.
+// Up to 4*32 tiles are read once into registers; longer rows loop. s_out, if
+// given, gets the sum 2^L itself (0 where it is not formed).
 __device__ __forceinline__ RowFinal combine_row(const Partial* p, int ntiles, bool greedy,
-                                                float chi, int lane) {
+                                                float chi, int lane, double* s_out = nullptr) {
   constexpr int kReg = 4;
   float pm[kReg];
   double ps[kReg];
@@ -167,6 +168,7 @@ __device__ __forceinline__ RowFinal combine_row(const Partial* p, int ntiles, bo
     s = warp_sum_d(s);
     ok = (s > 0.0 && s < INFINITY);
     f.L = log2(s);
+    if (s_out) *s_out = s;
   }
   f.ok = ok;
   return f;
@@ -225,6 +227,69 @@ cudaError_t launch_hier2_decide(const HierDecideArgs& a, cudaStream_t st);
 __host__ __device__ __forceinline__ int residual_tiles(int V) {  // kResTile tiles per row
   return (V + kResTile - 1) / kResTile;
 }
+
+// ----------------------------------------------------------------------------
+// Vocabulary-parallel chain verification (vocab.cu)
+// ----------------------------------------------------------------------------
+// One row's statistics over one vocabulary shard [v0, v0 + Vs): the shard's
+// largest logit m and its global id, the shift M = fl(m * c_hi) and
+// S = sum over the shard of 2^(l*c - M), and the logit x of the row's
+// drafted token when the shard holds it. 32 bytes, exchanged between ranks.
+constexpr int kVpHasX = 1;  // the shard holds the drafted token: x is its logit
+constexpr int kVpBad = 2;   // the shard saw a NaN or +inf logit
+struct VpRow {
+  double M, S;
+  float m;
+  int amax;
+  float x;
+  int flags;
+};
+static_assert(sizeof(VpRow) == SPEC_VP_ROW_BYTES, "record size is part of the C ABI");
+// One sequence's draw weights over one shard: z = the shard's sum of the
+// weights of the draw (max(0, p - q) at a rejection, p for the bonus token),
+// p = the shard's mass under the target row of the draw.
+struct VpMass {
+  double z, p;
+};
+static_assert(sizeof(VpMass) == SPEC_VP_MASS_BYTES, "record size is part of the C ABI");
+// What the decide launch leaves for the pick launch, per sequence.
+struct VpSeq {
+  double Lp, Lq;  // log2-partitions of the draw's target / draft rows
+  float mp, mq;   // their largest logits
+  float u;        // draw uniform
+  int a;          // first rejection (K: all accepted)
+  int state;      // kVpSeqBad, kVpSeqGreedy or kVpSeqDraw
+  int tok;        // greedy: the token at a
+};
+constexpr int kVpSeqBad = 0, kVpSeqGreedy = 1, kVpSeqDraw = 2;
+
+struct VpArgs {
+  int B, K, Vs, v0, V, R, rank;
+  const unsigned char* tgt;   // this rank's shard rows
+  const unsigned char* drf;
+  long long ld_tgt, ld_drf;   // bytes
+  const int32_t* draft_tok;
+  const float* temperature;
+  uint64_t seed;
+  const int32_t* seq_id;
+  uint32_t round;
+  const Partial* part;        // row-statistics partials of the shard rows
+  int ntiles;
+  VpRow* rows;                // [B, 2K+1] this rank's records
+  const VpRow* rows_all;      // [R, B, 2K+1] every rank's, in rank order
+  VpMass* mass;               // [B] this rank's
+  const VpMass* mass_all;     // [R, B]
+  VpSeq* seq;                 // [B]
+  double* tsum;               // [B, nrt] residual tile sums of the shard
+  double* pre;                // [B, nrt] their prefixes
+  int32_t* accept_len;
+  int32_t* out_tok;
+  double* diag;
+  int32_t* status;
+};
+cudaError_t launch_vp_records(int dtype, const VpArgs& a, cudaStream_t st);
+cudaError_t launch_vp_decide(int dtype, const VpArgs& a, cudaStream_t st);
+cudaError_t launch_vp_pick(int dtype, const VpArgs& a, cudaStream_t st);
 
 // ----------------------------------------------------------------------------
 // Paged commit
@@ -355,6 +420,13 @@ struct StepArgs {
 };
 
 cudaError_t launch_chain_step(const StepArgs& a, cudaStream_t st);
+
+// Saguaro sampling: T ln(1 - eps) added in place to the cached tokens' logits
+// of each sequence's draft rows (see saguaro.cu).
+cudaError_t launch_saguaro_adjust(int dtype, unsigned char* lg, long long ld_bytes, int B,
+                                  int rows_per_seq, int V, const int32_t* cached, int n_cached,
+                                  int per_row, double ln1m_eps, const float* temperature,
+                                  cudaStream_t st);
 
 cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out, cudaStream_t st);
 

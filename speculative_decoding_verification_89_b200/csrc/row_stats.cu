@@ -25,6 +25,12 @@
 
 namespace specv {
 
+// Limit of the waits for this kernel's tile copies: kWaitLimitNs unless a
+// test has set another with spec_test_set_wait_limit_ns (0: one non-blocking
+// test per wait, so a copy still in flight makes the wait run out). The
+// drain of the copies in flight after a timeout always uses kWaitLimitNs.
+__device__ unsigned long long g_rs_wait_limit_ns = kWaitLimitNs;
+
 // A launch lists at most kMaxListRows rows (the host splits larger calls).
 constexpr int kMaxListRows = 8192;
 constexpr int kRsSmemTotal = kRsSmem + kMaxListRows * (int)sizeof(int);
@@ -170,8 +176,9 @@ __global__ void __launch_bounds__(kRsWarps * 32, 1)
   double acc1 = 0.0;         // sum of 2^(l*c - Msh) * (l - anchor) (Rows::kEntropy)
   int gidx = 0x7fffffff;     // greedy rows: first index of mrun
 
+  const uint64_t wait_limit = g_rs_wait_limit_ns;
   for (; cc.left > 0; s = (s + 1 == kRsStages) ? 0 : s + 1) {
-    const bool ok = mbar_wait_bounded(&bars[s], (phase >> s) & 1u, kWaitLimitNs);
+    const bool ok = mbar_wait_bounded(&bars[s], (phase >> s) & 1u, wait_limit);
     if (__any_sync(0xffffffffu, !ok)) {
       timed_out = true;
       break;
@@ -415,6 +422,19 @@ cudaError_t launch_row_stats(int dtype, const Rows& rows, int nrows, int V, cons
     return launch_rs<__nv_bfloat16>(rows, nrows, V, b.part, b.mom, b.zero, status, st);
   return launch_rs<float>(rows, nrows, V, b.part, b.mom, b.zero, status, st);
 }
+
+}  // namespace specv
+
+#pragma GCC visibility push(default)
+extern "C" int spec_test_set_wait_limit_ns(uint64_t ns) {
+  const unsigned long long v = ns;
+  const cudaError_t e = cudaMemcpyToSymbol(specv::g_rs_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return specv::record_cuda_status(e);
+  return SPEC_OK;
+}
+#pragma GCC visibility pop
+
+namespace specv {
 
 template cudaError_t launch_row_stats<ChainRows>(int, const ChainRows&, int, int,
                                                  const RsBuffers&, int32_t*, cudaStream_t);

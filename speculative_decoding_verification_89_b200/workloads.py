@@ -201,6 +201,24 @@ def draft_batch(device="cpu", rnd=0, B=64, V=128256, seed=5):
                          temperature=1.0, philox_seed=5)
 
 
+def cached_tokens(lg, n_cached, *, seed, extra=None):
+    """Synthetic speculation-cache lists (Saguaro sampling), one per row of
+    lg [..., V]: the ids of the row's n_cached - 3 largest logits (the likely
+    bonus tokens a cache prepares), then ``extra[...]`` (e.g. the drafted
+    token) or a repeat of the top id, then the padding ids -1 and V; each list
+    shuffled. Returns int32 [..., n_cached] on lg's device."""
+    V = lg.shape[-1]
+    top = torch.topk(lg.float(), max(n_cached - 3, 1), dim=-1).indices.to(torch.int32)
+    top = top[..., :n_cached - 3]
+    third = top[..., :1] if extra is None else extra.to(torch.int32)[..., None]
+    pad = torch.tensor([-1, V], dtype=torch.int32, device=lg.device).expand(*lg.shape[:-1], 2)
+    ids = torch.cat([top, third, pad], dim=-1)
+    gen = generator(seed, "cpu")
+    flat = ids.reshape(-1, n_cached)
+    perm = torch.stack([torch.randperm(n_cached, generator=gen) for _ in range(flat.shape[0])])
+    return torch.gather(flat, 1, perm.to(flat.device)).reshape(ids.shape).contiguous()
+
+
 # ----------------------------------------------------------------------------
 # Paged KV state
 # ----------------------------------------------------------------------------

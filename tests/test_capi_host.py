@@ -194,3 +194,61 @@ def test_outcome_workspace_and_host_errors(lib):
         bad = list(base)
         bad[i] = v
         assert f(*bad) == want, (i, v)
+
+
+def test_saguaro_host_argument_errors(lib):
+    """Bad sizes, dtype, list layout or eps are refused before any launch;
+    eps = 0, empty lists and B = 0 return at once (the fake pointers are never
+    read)."""
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    f = lib.spec_saguaro_adjust
+    f.restype = I
+    f.argtypes = [P, I64, I, I, I, I, P, I, I, ctypes.c_double, P, P]
+    fake = P(0x10000)
+    base = [fake, 1024, 1, 4, 3, 1000, fake, 8, 0, 0.3, fake, None]
+    assert f(*base[:9], 0.0, *base[10:]) == 0        # eps = 0
+    assert f(*base[:7], 0, *base[8:]) == 0           # no cached ids
+    assert f(*base[:3], 0, *base[4:]) == 0           # B = 0
+    for i, v in [(1, 999), (2, 7), (3, -1), (4, -1), (5, 0), (7, 1025), (8, 2), (9, 1.0),
+                 (9, -0.5), (9, float("nan")), (0, None), (6, None), (10, None)]:
+        bad = list(base)
+        bad[i] = v
+        assert f(*bad) == -1, (i, v)
+
+
+def test_vocab_parallel_workspace_and_host_errors(lib):
+    """Shard outside the vocabulary, bad rank counts, missing buffers and a
+    short workspace are refused on the host; B = 0 returns at once. Every
+    call here must be refused before a launch: the pointers are fake."""
+    P, I, I64, U32, U64, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
+                               ctypes.c_uint64, ctypes.c_size_t)
+    g = lib.spec_vp_workspace_bytes
+    g.restype = SZ
+    g.argtypes = [I, I, I, I]
+    full = g(64, 8, 16032, 1)
+    assert full > g(64, 8, 8000, 1) > 0 and g(64, 300, 1000, 1) == 0 and g(4, 2, 100, 5) == 0
+    f = lib.spec_vp_decide
+    f.restype = I
+    f.argtypes = [P, I64, P, I64, I, I, I, I, I, I, I, I, P, P, P, U64, P, U32, P, P, P, P, SZ, P]
+    fake = P(0x10000)
+    # tgt, ld, drf, ld, dtype, B, K, Vs, v0, V, R, rank, rows_all, drafts, T, seed, seq_id,
+    # round, mass_out, diag, status, ws, ws_bytes, stream
+    base = [fake, 1024, fake, 1024, 1, 4, 3, 1000, 1000, 2000, 2, 1, fake, fake, fake, 0, fake,
+            0, fake, None, fake, fake, 1 << 30, None]
+    assert f(*base[:5], 0, *base[6:]) == 0                 # B = 0
+    for i, v, want in [(8, 1001, -1), (8, -1, -1), (9, 1999, -1), (10, 0, -1), (10, 65, -1),
+                       (11, 2, -1), (11, -1, -1), (12, None, -1), (13, None, -1),
+                       (16, None, -1), (18, None, -1), (0, None, -1), (1, 999, -1),
+                       (22, 64, -3), (21, None, -3)]:
+        bad = list(base)
+        bad[i] = v
+        assert f(*bad) == want, (i, v)
+    s = lib.spec_vp_shard_stats
+    s.restype = I
+    s.argtypes = [P, I64, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+    sb = [fake, 1024, fake, 1024, 1, 4, 3, 1000, 1000, 2000, fake, fake, fake, fake, fake,
+          1 << 30, None]
+    for i, v, want in [(10, None, -1), (12, None, -1), (12, P(0x10004), -1), (8, 1001, -1)]:
+        bad = list(sb)
+        bad[i] = v
+        assert s(*bad) == want, (i, v)
