@@ -74,15 +74,16 @@ bool draft_layout(int B, int V, int dtype, DraftLayout* L) {
 // per-(sequence, position) best weights and tokens.
 struct OutcomeLayout {
   Layout L;
-  size_t zk, cw, cv, total;
+  size_t zk, lt, cw, cv, total;
 };
 bool outcome_layout(int B, int K, int V, int dtype, int n_top, OutcomeLayout* O) {
   if (n_top < 0 || n_top > SPEC_MAX_TOP) return false;
   if (!layout(B, K, V, dtype, 0, &O->L)) return false;
   const size_t slots = (size_t)B * (K + 1);
   O->zk = O->L.total;
-  O->cw = O->zk + align_up(slots * sizeof(double));
-  O->cv = O->cw + align_up(slots * (size_t)n_top * sizeof(float));
+  O->lt = O->zk + align_up(slots * sizeof(double));
+  O->cw = O->lt + align_up((size_t)B * (2 * K + 1) * sizeof(double));
+  O->cv = O->cw + align_up(slots * (size_t)n_top * sizeof(double));
   O->total = O->cv + align_up(slots * (size_t)n_top * sizeof(int));
   return true;
 }
@@ -689,7 +690,9 @@ int spec_outcome_law(const void* tgt, int64_t ld_tgt, const void* drf, int64_t l
   rows.ld_drf = ld_drf * es;
   rows.temperature = temperature;
   rows.K = K;
-  rows.late_pos = 0;  // every target row pair is read again
+  // every row pair is read again: those of the first late_pos positions are
+  // streamed last, to be still in L2 when the pair pass reads them
+  rows.late_pos = late_positions(B, V, dtype, 2);
   const cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = launch_row_stats(dtype, rows, B * (2 * K + 1), V, rs_buffers(ws, O.L),
                                    dev_status, st);
@@ -708,7 +711,9 @@ int spec_outcome_law(const void* tgt, int64_t ld_tgt, const void* drf, int64_t l
   a.temperature = temperature;
   a.part = reinterpret_cast<const Partial*>((char*)ws + O.L.part);
   a.zk = reinterpret_cast<double*>((char*)ws + O.zk);
-  a.cw = reinterpret_cast<float*>((char*)ws + O.cw);
+  a.lt = reinterpret_cast<double*>((char*)ws + O.lt);
+  a.cw = reinterpret_cast<double*>((char*)ws + O.cw);
+  a.late_pos = rows.late_pos;
   a.cv = reinterpret_cast<int*>((char*)ws + O.cv);
   a.p_len = p_len;
   a.beta = beta;

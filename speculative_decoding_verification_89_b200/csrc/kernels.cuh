@@ -433,6 +433,7 @@ cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out,
 // Outcome law of a chain check (drafts fixed): see outcome.cu.
 struct OutcomeArgs {
   int B, K, V, n_top, ntiles;
+  int late_pos;         // row pairs k < late_pos were streamed last by the statistics
   const unsigned char* tgt;
   const unsigned char* drf;
   long long ld_tgt, ld_drf;  // bytes
@@ -440,7 +441,8 @@ struct OutcomeArgs {
   const float* temperature;
   const Partial* part;  // [B * (2K+1), ntiles]
   double* zk;           // [B, K+1] residual masses
-  float* cw;            // [B, K+1, n_top] best weights
+  double* lt;           // [B, 2K+1] row log2-partitions (NaN: no finite statistics)
+  double* cw;           // [B, K+1, n_top] best weights (fp64)
   int* cv;              // [B, K+1, n_top] their tokens
   double* p_len;        // out [B, K+1]
   double* beta;         // out [B, K] or null
