@@ -134,6 +134,11 @@ def test_bf16_rounding_is_nearest_even():
     for v in (0.0, -2.5, 3.0 * 2.0 ** 100, -np.inf, np.inf):
         assert round_bf16(np.float32(v)) == np.float32(v)
     assert np.isnan(round_bf16(np.float32(np.nan)))
+    # rounding up carries into the exponent: the float just below 2 becomes 2
+    assert round_bf16(np.nextafter(np.float32(2.0), np.float32(0))) == np.float32(2.0)
+    assert round_bf16(np.float32(-(2.0 - 2.0 ** -23))) == np.float32(-2.0)
+    # the sign of zero is kept
+    assert np.signbit(round_bf16(np.float32(-0.0)))
 
 
 def test_stored_shift_follows_the_kernel_arithmetic():
