@@ -384,7 +384,9 @@ def run_ours(args, dist):
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, prob, state, bufs, base, dev, dist)
     result["draft_step"] = run_draft_step(args, dev, dist, peak)
+    result["saguaro_draft"] = run_saguaro_draft(args, dev, dist)
     result["outcome_law"] = run_outcome_law(args, prob, dev, dist, peak)
+    result["vocab_parallel_emulated"] = run_vocab_parallel(args, prob, dev, dist)
     result["configs"] = run_configs(args, dev, dist, peak, result)
     if dist.world == 1 and dist.rank == 0:
         rnd = args.warmup + args.steps
@@ -485,6 +487,37 @@ def run_two_call_step(args, prob, state, bufs, base, dev, dist):
             "gpu_launches_per_step": 4}
 
 
+def graph_us_per_call(calls, reps, dist):
+    """Device time per call of a short launch sequence: the calls (each a
+    closure that launches on the current stream) captured once in a CUDA
+    graph and the graph replayed `reps` times between events, so that the
+    Python-side cost of each call does not set the pace."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for fn in calls:  # warm-up outside the capture (attributes, lookups)
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for fn in calls:
+            fn()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.reduce(e0.elapsed_time(e1), "max") / (reps * len(calls))
+    del g
+    return ms * 1e3
+
+
 def run_draft_step(args, dev, dist, peak):
     """The draft step (next token of each sequence from the drafting exit,
     with its entropy) on B=64 rows of V=128256 bf16: calls per second and the
@@ -515,18 +548,112 @@ def run_draft_step(args, dev, dist, peak):
                                logq=logq, entropy=ent)
     e1.record()
     torch.cuda.synchronize()
-    ms = dist.reduce(e0.elapsed_time(e1), "max") / n
+    ms_host = dist.reduce(e0.elapsed_time(e1), "max") / n
+    calls = [lambda i=i: capi.spec_draft_sample(probs[i].logits, T, prob.seed, sid, i, pos, tok,
+                                                status, ws, logq=logq, entropy=ent)
+             for i in range(10)]
+    ms = graph_us_per_call(calls, max(10, n // 10), dist) * 1e-3
     if int(status.item()) != 0:
         raise RuntimeError(f"draft step: device status {int(status.item())}")
     nbytes = B * V * 2
     return {"workload": "draft step: B=64 rows, V=128256 bf16 (N(0,4) + Zipf(1.1)), T=1, "
                         "token + ln q + entropy per row; 10 batches in turn (164 MB > L2)",
-            "us_per_call": ms * 1e3, "calls": n,
+            "us_per_call": ms * 1e3, "timing": "CUDA graph of 10 calls, replayed",
+            "us_per_call_from_python": ms_host * 1e3, "calls": n,
             "tokens_per_s": B * dist.world / (ms * 1e-3),
             "algorithmic_bytes_per_call": nbytes,
             "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": nbytes / (ms * 1e-3) / 1e9 / peak,
             "gpu_launches_per_call": 1}
+
+
+def run_saguaro_draft(args, dev, dist):
+    """Saguaro sampling before the draft step: the 32 cached tokens of each of
+    B=64 sequences lowered in place (eps = 0.5) in rows of V=128256 bf16, then
+    the draft step on the lowered rows; 10 batches in turn. The lowering
+    accumulates over the calls on the same batch; timing is not affected."""
+    from speculative_decoding_verification_89_b200 import capi
+    from speculative_decoding_verification_89_b200 import workloads as W
+    probs = [W.draft_batch(device=dev, rnd=r) for r in range(10)]
+    cached = [W.cached_tokens(p.logits, 32, seed=700 + r).to(dev) for r, p in enumerate(probs)]
+    prob = probs[0]
+    T, sid, pos = prob.temperature, prob.seq_id, prob.pos
+    ws = capi.draft_workspace(B, V, prob.logits.dtype, device=dev)
+    tok = torch.empty(B, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = max(10, min(args.steps, 2000))
+
+    def adjust(i):
+        capi.spec_saguaro_adjust(probs[i % 10].logits, cached[i % 10], 0.5, T)
+
+    def both(i):
+        adjust(i)
+        capi.spec_draft_sample(probs[i % 10].logits, T, prob.seed, sid, i, pos, tok, status, ws)
+
+    out = {}
+    for name, fn in (("us_per_call_adjust", adjust), ("us_per_call_adjust_and_draft", both)):
+        out[name] = graph_us_per_call([lambda i=i: fn(i) for i in range(10)],
+                                      max(10, n // 10), dist)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"saguaro draft: device status {int(status.item())}")
+    return {"workload": "Saguaro lowering (eps 0.5, 32 cached ids per sequence) of B=64 rows, "
+                        "V=128256 bf16, then the draft step; 10 batches in turn",
+            **out, "timing": "CUDA graph of 10 calls, replayed", "calls": n,
+            "bound": "latency (2048 logits updated per call)",
+            "gpu_launches_per_call": 2}
+
+
+def run_vocab_parallel(args, prob, dev, dist):
+    """The vocabulary-parallel check at the benchmark's verification shape
+    with its R=8 ranks emulated on this one GPU: each rank's three launches
+    (after the row statistics of its shard) run in turn and the exchanges are
+    device copies in rank order. The NVLink exchange of a multi-GPU run is
+    not measured here; the figure is the kernels' total over the ranks."""
+    from speculative_decoding_verification_89_b200.vocab_parallel import ChainShard, vocab_shards
+    R = 8
+    Bp, Kp1, Vv = prob.tgt.shape
+    K1 = Kp1 - 1
+    dt, T, sid = prob.draft_tok, prob.temperature, prob.seq_id
+    ranks = []
+    for r, (v0, Vs) in enumerate(vocab_shards(Vv, R)):
+        ranks.append(dict(
+            sh=ChainShard(Bp, K1, Vv, v0, Vs, R, r, prob.tgt.dtype, device=dev),
+            tgt=prob.tgt[:, :, v0:v0 + Vs].contiguous(),
+            drf=prob.drf[:, :, v0:v0 + Vs].contiguous(),
+            acc=torch.empty(Bp, dtype=torch.int32, device=dev),
+            out=torch.empty((Bp, Kp1), dtype=torch.int32, device=dev)))
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rows_all = ranks[0]["sh"].rows_all
+    mass_all = ranks[0]["sh"].mass_all
+    out_all = torch.empty((R, Bp, Kp1), dtype=torch.int32, device=dev)
+
+    def check(i):
+        for x in ranks:
+            x["sh"].stats(x["tgt"], x["drf"], dt, T, status)
+        for r, x in enumerate(ranks):
+            rows_all[r].copy_(x["sh"].rows)
+        for x in ranks:
+            x["sh"].rows_all = rows_all
+            x["sh"].decide(x["tgt"], x["drf"], dt, T, prob.seed, sid, i, status)
+        for r, x in enumerate(ranks):
+            mass_all[r].copy_(x["sh"].mass)
+        for r, x in enumerate(ranks):
+            x["sh"].mass_all = mass_all
+            x["sh"].pick(x["tgt"], x["drf"], dt, T, x["acc"], out_all[r], status)
+        return out_all.amax(0)
+
+    n = max(10, min(args.steps // 20, 200))
+    ms = graph_us_per_call([lambda: check(0)], n, dist) * 1e-3
+    if int(status.item()) != 0:
+        raise RuntimeError(f"vocabulary-parallel check: device status {int(status.item())}")
+    per_seq = 32 * (2 * K1 + 1) + 16 + 4 * (K1 + 1)
+    return {"workload": f"vocabulary-parallel chain check, B={Bp}, K={K1}, V={Vv} bf16 over "
+                        f"R={R} shards, ranks emulated in turn on one GPU",
+            "us_per_check_all_ranks": ms * 1e3, "checks": n,
+            "timing": "CUDA graph of one check (all ranks), replayed",
+            "exchange_bytes_per_rank_per_check": Bp * per_seq,
+            "note": "unmeasured on hardware with R GPUs: exchanges here are device copies",
+            "gpu_launches_per_check": 4 * R}
 
 
 def run_outcome_law(args, prob, dev, dist, peak):
