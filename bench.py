@@ -388,6 +388,10 @@ def run_ours(args, dist):
     result["outcome_law"] = run_outcome_law(args, prob, dev, dist, peak)
     result["vocab_parallel_emulated"] = run_vocab_parallel(args, prob, dev, dist)
     result["configs"] = run_configs(args, dev, dist, peak, result)
+    if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
+        for key, kind in (("draft_step", "draft"), ("saguaro_draft", "saguaro"),
+                          ("outcome_law", "outcome"), ("vocab_parallel_emulated", "chain")):
+            result[key]["oracle"] = oracle_rates(kind)
     if dist.world == 1 and dist.rank == 0:
         rnd = args.warmup + args.steps
         acc1 = torch.empty(B, dtype=torch.int32, device=dev)
@@ -901,7 +905,13 @@ ORACLE_CFG = {
                      "plus its paged commit", 2),
     "hier_mixed": ("one sequence, 8 rolling two-stage rounds, K=N_i=4, V=151936", 1),
     "engine": ("one sequence, 8 rolling two-stage rounds with paged commit, K=N_i=4, V=32000", 2),
+    "draft": ("16 draft rows of V=128256 (N(0,4) + Zipf(1.1)), token + ln q + entropy", 2),
+    "saguaro": ("16 draft rows of V=128256: 32 cached ids lowered (eps 0.5, bf16 form), then "
+                "the draft step", 2),
+    "outcome": ("one sequence's outcome law, K=8, V=128256, 32 outcomes", 2),
+    "chain": ("one sequence-round of B=64-shape chain verification (K=8, V=128256)", 2),
 }
+ORACLE_UNIT = {"outcome": "sequences/s"}
 
 
 def _softmax_draw(rows, T, rng):
@@ -981,6 +991,40 @@ def _oracle_task(job):
                      stack, 32, 16, 1032, 9)
         sec += time.perf_counter() - t0
         tok += res.accepted + 1
+    elif kind in ("draft", "saguaro"):
+        from oracle.draft import draft_step, saguaro_logits
+        V = 128256
+        prior = -1.1 * np.log(np.arange(V) + 1.0)
+        lg = (rng.normal(0, 2, (16, V)) + prior).astype(np.float32).astype(np.float64)
+        T = np.ones(16)
+        cached = np.argsort(-lg, axis=1)[:, :32] if kind == "saguaro" else None
+        t0 = time.perf_counter()
+        if kind == "saguaro":
+            lg = np.stack([saguaro_logits(lg[r], 1.0, cached[r], 0.5, "bf16") for r in range(16)])
+        draft_step(lg, T, 5, np.arange(16) + 100 * i, 0, np.zeros(16, dtype=np.int64))
+        sec += time.perf_counter() - t0
+        tok += 16
+    elif kind == "outcome":
+        from oracle.outcome import outcome_law, top_outcomes
+        V = 128256
+        prior = -1.1 * np.log(np.arange(V) + 1.0)
+        tgt = (rng.normal(0, 2, (9, V)) + prior).astype(np.float32).astype(np.float64)
+        drf = (tgt[:8] + rng.normal(0, 1, (8, V))).astype(np.float32).astype(np.float64)
+        drafts = _softmax_draw(drf, 1.0, rng)
+        t0 = time.perf_counter()
+        top_outcomes(outcome_law(tgt, drf, drafts, 1.0), 32)
+        sec += time.perf_counter() - t0
+        tok += 1
+    elif kind == "chain":
+        V = 128256
+        prior = -1.1 * np.log(np.arange(V) + 1.0)
+        tgt = (rng.normal(0, 2, (1, 9, V)) + prior).astype(np.float32).astype(np.float64)
+        drf = (tgt[:, :8] + rng.normal(0, 1, (1, 8, V))).astype(np.float32).astype(np.float64)
+        drafts = _softmax_draw(drf[0], 1.0, rng)[None, :]
+        t0 = time.perf_counter()
+        res = verify_chain(tgt, drf, drafts, np.array([1.0]), 2, np.array([i]), 0)[0]
+        sec += time.perf_counter() - t0
+        tok += res.accepted + 1
     elif kind == "hier_peaked":
         hier_rounds(32000, 6, 2.5, 0.7, 1.5, 0.7, boost=6.0)
     elif kind == "hier_mixed":
@@ -1012,7 +1056,8 @@ def oracle_rates(kind):
     desc, per = ORACLE_CFG[kind]
     one = [_oracle_task((kind, 10_000 + k)) for k in range(per)]
     r1 = sum(t for _, t, _ in one) / max(sum(s for _, _, s in one), 1e-9)
-    out = {"unit": "tokens/s", "kind": "oracle", "task": desc, "single_thread": r1}
+    out = {"unit": ORACLE_UNIT.get(kind, "tokens/s"), "kind": "oracle", "task": desc,
+           "single_thread": r1}
     if _POOL is not None:
         procs = _POOL._processes
         res = _POOL.map(_oracle_task, [(kind, k) for k in range(procs * per)])
