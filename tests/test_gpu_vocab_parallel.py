@@ -8,10 +8,10 @@ check's (accepted counts and tokens bit-exact except at decisions within the
 relative). Every rank must also end with identical outputs.
 
 Most tests run the R ranks in one process: each launch for every shard, and
-the exchanges as plain stacking of their outputs in rank order. The last test
-runs two gloo processes that share the GPU and exchange through
-torch.distributed. Their kernels never wait on one another; only the host
-collectives do."""
+the exchanges as plain stacking of their outputs in rank order. Two tests go
+through torch.distributed: two gloo processes sharing the GPU (their kernels
+never wait on one another; only the host collectives do), and a world of one
+NCCL rank, which takes the device-tensor collectives."""
 import os
 import socket
 import sys
@@ -261,4 +261,60 @@ def test_vp_two_gloo_processes_on_one_gpu():
         a = int(a0[b])
         if compare_check(f"gloo/seq{b}", r, a, [int(x) for x in o0[b, :a + 1]], tally):
             compare_probs(f"gloo/seq{b}", r, d0[b], K, float(prob.temperature[b]))
+    tally.check_share()
+
+
+# ---------------------------------------------------------------------------
+# One rank over NCCL: the device-tensor exchange calls
+# ---------------------------------------------------------------------------
+def _nccl_worker(port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+    from speculative_decoding_verification_89_b200.vocab_parallel import (
+        ChainShard, verify_chain_vocab_parallel)
+    from speculative_decoding_verification_89_b200 import workloads as W2
+    try:
+        torch.cuda.set_device(0)
+        dist.init_process_group("nccl", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+        prob = W2.chain_problem(16, 4, 5000, torch.bfloat16, seed=77, temperature=0.9)
+        B, Kp1, V = prob.tgt.shape
+        K = Kp1 - 1
+        sh = ChainShard(B, K, V, 0, V, 1, 0, prob.tgt.dtype)
+        acc = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+        out = torch.full((B, K + 1), -7, dtype=torch.int32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        verify_chain_vocab_parallel(sh, prob.tgt.cuda(), prob.drf.cuda(), prob.draft_tok.cuda(),
+                                    prob.temperature.cuda(), prob.seed, prob.seq_id.cuda(),
+                                    prob.rnd, acc, out, st)
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+        q.put((acc.cpu().numpy(), out.cpu().numpy(), int(st.item())))
+    except Exception as exc:  # report instead of leaving the parent waiting
+        q.put((repr(exc), None, None))
+        raise
+
+
+def test_vp_one_rank_over_nccl():
+    """A world of one NCCL rank holding the whole vocabulary: the exchanges
+    take the device-tensor collectives (all_gather_into_tensor, all_reduce
+    MAX) and the result is the oracle's check."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_nccl_worker, args=(port, q))
+    p.start()
+    acc, out, st = q.get(timeout=300)
+    p.join(timeout=120)
+    assert out is not None, acc
+    assert p.exitcode == 0 and st == 0
+    prob = W.chain_problem(16, 4, 5000, torch.bfloat16, seed=77, temperature=0.9)
+    ref = run_chain_oracle(prob)
+    tally = Tally()
+    for b, r in ref.items():
+        a = int(acc[b])
+        compare_check(f"nccl/seq{b}", r, a, [int(x) for x in out[b, :a + 1]], tally)
     tally.check_share()
