@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
     if (diag)
       for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
   };
-  if (!tvalid) {  // same verdict in every CTA of the cluster: all leave here
+  if (!tvalid) {  // the same decision in every CTA of the cluster: all leave here
     if (rank == 0) fail();
     return;
   }

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
     if (A.out_logq) A.out_logq[b] = bad ? dnan() : logq;
     if (A.out_entropy) A.out_entropy[b] = bad ? dnan() : H;
   };
-  if (!temp_valid(Tb)) {  // the same verdict in every CTA of the cluster
+  if (!temp_valid(Tb)) {  // the same decision in every CTA of the cluster
     if (rank == 0 && threadIdx.x == 0) finish(-1, 0.0, 0.0, true);
     return;
   }
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     if (A.out_logq) A.out_logq[b] = bad ? dnan() : logq;
     if (A.out_entropy) A.out_entropy[b] = bad ? dnan() : H;
   };
-  if (!temp_valid(Tb)) {  // the same verdict in every CTA of the cluster
+  if (!temp_valid(Tb)) {  // the same decision in every CTA of the cluster
     if (rank == 0 && threadIdx.x == 0) finish(-1, 0.0, 0.0, true);
     return;
   }
