@@ -7,6 +7,7 @@ while the whole case stays well under a few GB of device memory.
 
     python profile_case.py --B 32
     python profile_case.py --B 64 --commit
+    python profile_case.py --B 64 --vp 8
 """
 from __future__ import annotations
 
@@ -30,6 +31,9 @@ def main():
     ap.add_argument("--outcome", type=int, default=-1,
                     help="run the outcome law with this many outcomes instead of verifying")
     ap.add_argument("--draft", action="store_true", help="run the draft step instead of verifying")
+    ap.add_argument("--vp", type=int, default=0,
+                    help="run the vocabulary-parallel check over this many shards, the ranks "
+                         "in turn on this GPU, instead of verifying")
     args = ap.parse_args()
     B, K, V = args.B, 8, W.LLAMA3_V
     dev = torch.device("cuda")
@@ -44,7 +48,7 @@ def main():
         base = state.seq_lens.clone()
         gen = torch.Generator(device=dev)
         gen.manual_seed(0)
-    if args.outcome >= 0 or args.draft:
+    if args.outcome >= 0 or args.draft or args.vp > 0:
         return other(args, B, K, V, dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     times = []
@@ -70,9 +74,37 @@ def main():
 
 
 def other(args, B, K, V, dev):
-    """The outcome law (on the verification inputs) or the draft step."""
+    """The outcome law (on the verification inputs), the draft step, or the
+    vocabulary-parallel check with its ranks in turn (exchanges as copies)."""
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    if args.draft:
+    if args.vp > 0:
+        from speculative_decoding_verification_89_b200.vocab_parallel import (ChainShard,
+                                                                              vocab_shards)
+        prob = W.chain_batch(device=dev, B=B)
+        R = args.vp
+        ranks = []
+        for r, (v0, Vs) in enumerate(vocab_shards(V, R)):
+            ranks.append((ChainShard(B, K, V, v0, Vs, R, r, torch.bfloat16, device=dev),
+                          prob.tgt[:, :, v0:v0 + Vs].contiguous(),
+                          prob.drf[:, :, v0:v0 + Vs].contiguous(),
+                          torch.empty(B, dtype=torch.int32, device=dev),
+                          torch.empty((B, K + 1), dtype=torch.int32, device=dev)))
+
+        def call(i):
+            for sh, tgt, drf, _, _ in ranks:
+                sh.stats(tgt, drf, prob.draft_tok, prob.temperature, st)
+            for r, (sh, _, _, _, _) in enumerate(ranks):
+                ranks[0][0].rows_all[r].copy_(sh.rows)
+            for sh, tgt, drf, _, _ in ranks:
+                sh.rows_all = ranks[0][0].rows_all
+                sh.decide(tgt, drf, prob.draft_tok, prob.temperature, prob.seed, prob.seq_id, i,
+                          st)
+            for r, (sh, _, _, _, _) in enumerate(ranks):
+                ranks[0][0].mass_all[r].copy_(sh.mass)
+            for sh, tgt, drf, a, o in ranks:
+                sh.mass_all = ranks[0][0].mass_all
+                sh.pick(tgt, drf, prob.draft_tok, prob.temperature, a, o, st)
+    elif args.draft:
         prob = W.draft_batch(device=dev, B=B)
         ws = capi.draft_workspace(B, V, torch.bfloat16, device=dev)
         tok = torch.empty(B, dtype=torch.int32, device=dev)
