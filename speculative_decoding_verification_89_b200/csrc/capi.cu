@@ -23,14 +23,15 @@ int stat_tiles(int V, int dtype) {
 }
 
 struct Layout {
-  size_t part, fin, ticket, seq, tsum, ctr, ints, total;
+  size_t part, fin, ticket, rec, seq, tsum, ctr, ints, total;
   long long rows;
 };
 
 // Workspace, each region 256-byte aligned: final row statistics and tile
 // partials for the largest row set (the step kernel keeps its chunk
-// statistics in the partials' place), the ticket word of the staged
-// verify-and-commit path, then the step kernel's per-sequence states,
+// statistics in the partials' place), the ticket and plan words and the
+// per-sequence commit records of the staged verify-and-commit path, then the
+// step kernel's per-sequence states,
 // residual tile sums, counters and per-sequence integer arrays.
 bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   if (B < 0 || K < 0 || K > SPEC_MAX_K || V < 1 || V > SPEC_MAX_V) return false;
@@ -43,7 +44,8 @@ bool layout(int B, int K, int V, int dtype, int Ni, Layout* L) {
   L->fin = 0;
   L->part = align_up((size_t)rows * sizeof(RowFinal));
   L->ticket = L->part + align_up((size_t)rows * stat_tiles(V, dtype) * sizeof(Partial));
-  L->seq = L->ticket + kAlign;
+  L->rec = L->ticket + kAlign;
+  L->seq = L->rec + align_up((size_t)B * sizeof(CommitRec));
   L->tsum = L->seq + align_up((size_t)B * sizeof(SeqState));
   // residual tile sums [B][nrt], then the draw-part totals [B][D]
   const size_t pt = part_tiles(elem_size(dtype));
@@ -570,6 +572,8 @@ int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf, i
   f.d.accept_len = accept_len;
   f.d.out_tok = out_tok;
   f.ticket = reinterpret_cast<int32_t*>((char*)ws + ck.L.ticket);
+  f.plan_flag = f.ticket + 1;
+  f.rec = reinterpret_cast<CommitRec*>((char*)ws + ck.L.rec);
   return cuda_status(launch_chain_fused(f, (cudaStream_t)stream));
 }
 

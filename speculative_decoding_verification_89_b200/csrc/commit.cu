@@ -30,6 +30,52 @@ __global__ void __launch_bounds__(kCopyThreads) commit_copy_kernel(CommitArgs a)
   copy_body(a, blockIdx.x, gridDim.x, s_off);
 }
 
+// The copy launch that follows a verify-and-commit decide launch: it does not
+// wait for that launch to complete, only for its planner. It lets its own
+// successors launch at once (they wait for its completion), waits -- one
+// thread, bounded -- until the planner has published plan_flag, copies, and
+// only then waits for the decide launch to complete, so nothing after it in
+// the stream runs before the draws are written. Its CTAs run beside the
+// decide launch's: this launch starts only once every CTA of that launch has
+// started (programmatic launch), so the planner's CTA is resident while they
+// wait.
+__global__ void __launch_bounds__(kCopyThreads) commit_copy_planned_kernel(CommitArgs a,
+                                                                           const int32_t* plan_flag) {
+  grid_dependents_launch();
+  __shared__ int s_go;
+  if (threadIdx.x == 0) {
+    int v = ld_relaxed(plan_flag);
+    if (!v) {
+      const uint64_t t0 = globaltimer_ns();
+      unsigned ns = 64;
+      for (;;) {
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+        v = ld_relaxed(plan_flag);
+        if (v || globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+    if (v) fence_acq_rel();  // the planner's writes are visible from here on
+    else set_status(a.status, SPEC_ETIMEOUT);
+    s_go = v;
+  }
+  __syncthreads();
+  if (s_go) {
+    extern __shared__ int s_off[];
+    copy_body(a, blockIdx.x, gridDim.x, s_off);
+  }
+  grid_dependency_wait();
+}
+
+cudaError_t launch_commit_copy_planned(const CommitArgs& a, const int32_t* plan_flag,
+                                       cudaStream_t st) {
+  const size_t smem = (2 * (size_t)a.B + 1) * sizeof(int);
+  cudaError_t e = reserve_dyn_smem(commit_copy_planned_kernel, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(commit_copy_planned_kernel, dim3(sm_count() * kCopyCtasPerSm),
+                    dim3(kCopyThreads), smem, st, a, plan_flag);
+}
+
 cudaError_t launch_commit_copy(const CommitArgs& a, cudaStream_t st) {
   if (a.B <= 0 || a.Kp1 <= 0 || !(a.kv_stage || a.hid_stage)) return cudaSuccess;
   const size_t smem = (2 * (size_t)a.B + 1) * sizeof(int);

@@ -61,10 +61,53 @@ static __device__ int4 block_excl_scan4(int4 v, int4* tot) {
 constexpr int kPushCache = 2048;   // freed entries cached in push order
 constexpr int kStackCache = 2048;  // stack entries popped from below the old top
 
+// One sequence's part of the plan, formed by a CTA of its own before the
+// planner runs (the verify-and-commit decide launch's leader of the sequence,
+// once its accept test is done): the table entries it holds, checked, its new
+// length and the first entries to be freed. The planner then reads one record
+// per sequence instead of the lengths and the whole table row.
+// (CommitRec, kernels.cuh)
+
+// Whole CTA; old_len = seq_lens[b]. The checks are plan_body's, per sequence.
+static __device__ void commit_record(const CommitArgs& a, int b, int old_len, int kept,
+                                     CommitRec* out) {
+  __shared__ int s_tail[kRecTail];
+  const int base = a.base_len ? a.base_len[b] : old_len;
+  const int bs = a.block_size;
+  const int nbo = ceil_div(max(old_len, 0), bs);
+  int nbn = nbo;
+  bool ok = !(kept < 0 || kept > a.Kp1 || base < 0 || base > old_len || old_len < 0);
+  if (ok) {
+    nbn = ceil_div(base + kept, bs);
+    if (nbo > a.max_blocks || nbn > a.max_blocks) ok = false;
+  }
+  const int held = min(nbo, a.max_blocks);
+  const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
+  int bad = 0;
+  for (int i = threadIdx.x; i < held; i += blockDim.x) {
+    const int v = tab[i];
+    if (v < 0 || v >= a.num_blocks) bad = 1;
+    if (i >= nbn && i < nbn + kRecTail) s_tail[i - nbn] = v;
+  }
+  bad = __syncthreads_or(bad);
+  if (threadIdx.x == 0) {
+    const bool good = ok && !bad;
+    const int4 h = make_int4(held, good ? base + kept : -1, kept, 0);
+    int t[kRecTail];
+#pragma unroll
+    for (int j = 0; j < kRecTail; ++j) t[j] = (good && nbn + j < held) ? s_tail[j] : -1;
+    reinterpret_cast<int4*>(out)[0] = h;
+    reinterpret_cast<int4*>(out)[1] = make_int4(t[0], t[1], t[2], t[3]);
+  }
+}
+
 // s_seq: dynamic shared memory of 3 * B ints. Runs in any block of up to 1024
 // threads. The kept counts are read from L2: in the fused verify-and-commit
-// path they were written by other CTAs of the same grid.
-static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
+// path they were written by other CTAs of the same grid. With recs (one
+// CommitRec per sequence, written by other CTAs of the same grid) the lengths,
+// counts, table checks and the first freed entries come from the records.
+static __device__ void plan_body(const CommitArgs& a, int* s_seq,
+                                 const CommitRec* recs = nullptr) {
   // [3][B]: table-entry prefix, new length, kept
   int* s_nbp = s_seq;             // blocks held before, then their exclusive prefix
   int* s_len = s_seq + a.B;
@@ -89,7 +132,22 @@ static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
   const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
   int4 cnt = make_int4(0, 0, 0, 0);  // frees, allocations, kept rows, table entries
   int bad = 0;
-  for (int b = b0; b < b1; ++b) {
+  int4 tail0 = make_int4(-1, -1, -1, -1);  // record tail of the run's first sequence
+  for (int b = b0; recs && b < b1; ++b) {
+    const int4 h = __ldcg(reinterpret_cast<const int4*>(recs + b));
+    if (b == b0) tail0 = __ldcg(reinterpret_cast<const int4*>(recs + b) + 1);
+    const int held = h.x, len = h.y, kept = h.z;
+    if (len < 0) bad = 1;
+    const int nbn = len < 0 ? held : ceil_div(len, bs);
+    s_nbp[b] = held;
+    s_len[b] = len < 0 ? 0 : len;
+    s_kept[b] = kept;
+    cnt.x += max(0, held - nbn);
+    cnt.y += max(0, nbn - held);
+    cnt.z += kept;
+    cnt.w += held;
+  }
+  for (int b = b0; !recs && b < b1; ++b) {
     const int old_len = a.seq_lens[b];
     const int base = a.base_len ? a.base_len[b] : old_len;
     const int kept = __ldcg(a.keep + b) + a.keep_add;
@@ -133,9 +191,10 @@ static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
   const int lo = max(0, ft + F - A);
   const bool cached = F <= kPushCache && ft - lo <= kStackCache;
   if (sizes_ok) {
-    // Every covered table entry must be a valid block id: 1, 2 or 4
-    // sequences per warp (32, 16 or 8 lanes each), 16 loads in flight per lane.
-    {
+    // Every covered table entry must be a valid block id (the records' CTAs
+    // checked them already): 1, 2 or 4 sequences per warp (32, 16 or 8 lanes
+    // each), 16 loads in flight per lane.
+    if (!recs) {
       const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
       const int need = ceil_div(a.B, nwarps);
       const int spw = need <= 1 ? 1 : (need <= 2 ? 2 : 4);
@@ -160,7 +219,15 @@ static __device__ void plan_body(const CommitArgs& a, int* s_seq) {
       int fpos = pre.x;
       for (int b = b0; b < b1; ++b) {
         const int32_t* tab = a.tables + (size_t)b * a.max_blocks;
-        for (int i = ceil_div(s_len[b], bs); i < held(b); ++i) s_push[fpos++] = tab[i];
+        const int nbn = ceil_div(s_len[b], bs);
+        for (int i = nbn; i < held(b); ++i) {
+          const int j = i - nbn;
+          int v;
+          if (!recs || j >= kRecTail) v = tab[i];
+          else if (b == b0) v = j == 0 ? tail0.x : j == 1 ? tail0.y : j == 2 ? tail0.z : tail0.w;
+          else v = __ldcg(&recs[b].tail[j]);
+          s_push[fpos++] = v;
+        }
       }
     }
     if (bad) atomicOr(&s_bad, 1);
@@ -231,12 +298,12 @@ static __device__ void copy_body(const CommitArgs& a, int cta, int ncta, int* s_
   if (threadIdx.x == 0) s_st0 = a.status ? *(volatile int32_t*)a.status : SPEC_OK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int b = (int)threadIdx.x - 32; b >= 0 && b < a.B; b += blockDim.x - 32)
-    s_len[b] = a.seq_lens[b];  // the other warps, while warp 0 scans
+    s_len[b] = __ldcg(a.seq_lens + b);  // the other warps, while warp 0 scans
   if (warp == 0) {
     int carry = 0;
     for (int b0 = 0; b0 < a.B; b0 += 32) {
       const int b = b0 + lane;
-      const int v = b < a.B ? a.keep[b] + a.keep_add : 0;
+      const int v = b < a.B ? __ldcg(a.keep + b) + a.keep_add : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -271,7 +338,7 @@ static __device__ void copy_body(const CommitArgs& a, int cta, int ncta, int* s_
     int nvec;
     if (sidx < nseg) {
       const int pos = s_len[b] - kept + i;  // base_len + i
-      const int blk = a.tables[(size_t)b * a.max_blocks + pos / a.block_size];
+      const int blk = __ldcg(a.tables + (size_t)b * a.max_blocks + pos / a.block_size);
       const int slot = pos % a.block_size;
       src = reinterpret_cast<const uint4*>(a.kv_stage +
                                            (((size_t)b * a.Kp1 + i) * nseg + sidx) * a.seg_bytes);

@@ -488,10 +488,20 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
 // stack, lengths, hidden offsets). The leader takes no residual tiles -- the
 // other kCluster - 1 CTAs sum them -- so the planner, which overlaps the
 // other sequences' draws, delays nothing but its own sequence's draw. The
-// copy launch after this one moves the kept K/V and hidden rows.
+// copy launch after this one moves the kept K/V and hidden rows: it starts
+// while this launch runs and waits for plan_flag, which the first CTA clears
+// before it lets that launch start and the planner sets when it is done.
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(FusedArgs F) {
-  pdl_begin();
+  grid_dependency_wait();
+  if (F.plan_flag && blockIdx.x == 0 && blockIdx.y == 0) {
+    if (threadIdx.x == 0) {
+      *F.plan_flag = 0;
+      __threadfence();
+    }
+    __syncthreads();  // cleared before any thread of this CTA lets the copy launch start
+  }
+  grid_dependents_launch();
   cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
@@ -506,9 +516,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
   const CommitArgs& cm = F.cm;
   const int b = blockIdx.y, K = c.K, V = c.V, per = 2 * K + 1;
   const int nrt = residual_tiles(V);
-  if (rank == 0) {  // the planner reads every held table entry: bring this row's into L2
-    const int old_len = max(cm.seq_lens[b], 0);
-    const int held = min((old_len + cm.block_size - 1) / cm.block_size, cm.max_blocks);
+  int old_len = 0;
+  if (rank == 0) {  // the record reads every held table entry: bring this row's into L2
+    old_len = cm.seq_lens[b];
+    const int held =
+        min((max(old_len, 0) + cm.block_size - 1) / cm.block_size, cm.max_blocks);
     const int32_t* row = cm.tables + (size_t)b * cm.max_blocks;
     for (int i = threadIdx.x * 32; i < held; i += blockDim.x * 32)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(row + i));
@@ -544,8 +556,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
   __syncthreads();
   const Outcome o = s_out;
   const int a = o.a;
-  // Leader: every output but a sampled sequence's drawn token, then the ticket.
+  // Leader: every output but a sampled sequence's drawn token, the sequence's
+  // commit record, then the ticket.
   if (rank == 0) {
+    commit_record(cm, b, old_len, (o.bad ? -1 : a) + cm.keep_add, F.rec + b);
     if (o.bad) {
       if (threadIdx.x == 0) {
         set_status(c.status, SPEC_EDEVICE);
@@ -576,7 +590,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
     __syncthreads();
     if (s_last) {
       __threadfence();  // every other sequence's kept count and status are visible
-      plan_body(cm, reinterpret_cast<int*>(dyn + 2 * nrt));
+      plan_body(cm, reinterpret_cast<int*>(dyn + 2 * nrt), F.rec);
+      if (F.plan_flag) {
+        __syncthreads();  // every write of the plan is made
+        if (threadIdx.x == 0) {
+          __threadfence();
+          st_release(F.plan_flag, 1);
+        }
+      }
     }
   }
   // Residual tile sums of a sampled sequence, split over the CTAs but the leader.
@@ -632,9 +653,13 @@ static cudaError_t launch_fused(const FusedArgs& a, cudaStream_t st) {
                       3 * (size_t)a.d.c.B * sizeof(int);
   cudaError_t e = reserve_dyn_smem(k, smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl_cluster(k, dim3(kCluster, a.d.c.B), dim3(kDecThreads), smem, st, kCluster, a);
-  if (e != cudaSuccess) return e;
-  return launch_commit_copy(a.cm, st);
+  const bool copy = a.cm.B > 0 && a.cm.Kp1 > 0 && (a.cm.kv_stage || a.cm.hid_stage);
+  FusedArgs f = a;
+  if (!copy) f.plan_flag = nullptr;
+  e = launch_pdl_cluster(k, dim3(kCluster, a.d.c.B), dim3(kDecThreads), smem, st, kCluster, f);
+  if (e != cudaSuccess || !copy) return e;
+  return f.plan_flag ? launch_commit_copy_planned(f.cm, f.plan_flag, st)
+                     : launch_commit_copy(f.cm, st);
 }
 
 cudaError_t launch_chain_fused(const FusedArgs& a, cudaStream_t st) {

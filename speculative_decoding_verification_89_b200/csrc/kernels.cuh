@@ -312,9 +312,24 @@ struct CommitArgs {
   int32_t* status;
 };
 
+// One sequence's part of a commit plan, formed before the planner runs.
+constexpr int kRecTail = 4;
+struct CommitRec {
+  int held;  // table entries held: min(blocks of the old length, max_blocks)
+  int len;   // new length base + kept; -1 if an input of the sequence or a held entry is invalid
+  int kept;
+  int pad;
+  int tail[kRecTail];  // the first table entries to be freed (-1 past the last)
+};
+static_assert(sizeof(CommitRec) == 32, "two 16-byte stores");
+
 // The planner launch, then the copy launch; the copy launch alone.
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 cudaError_t launch_commit_copy(const CommitArgs& a, cudaStream_t st);
+// The copy launch of the verify-and-commit path: it starts its copies once
+// *plan_flag is nonzero (set by the planner of the decide launch before it).
+cudaError_t launch_commit_copy_planned(const CommitArgs& a, const int32_t* plan_flag,
+                                       cudaStream_t st);
 
 // ----------------------------------------------------------------------------
 // Chain verification fused with the paged commit of its kept rows
@@ -323,6 +338,8 @@ struct FusedArgs {
   ChainDecideArgs d;
   CommitArgs cm;       // keep = d.accept_len, keep_add = 1, Kp1 = K + 1
   int32_t* ticket;     // zeroed by the row-statistics launch that precedes this call
+  int32_t* plan_flag;  // 0 at the decide launch's start, 1 once its planner has run
+  CommitRec* rec;      // [B] per-sequence records for the planner
 };
 
 // The decide launch that also plans the commit, then the copy launch; the

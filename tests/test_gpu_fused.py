@@ -305,3 +305,37 @@ def test_split_entry_points_repeat_after_one_row_pass():
             assert torch.equal(x, y)
     assert torch.equal(res[0][1].view(torch.int16), res[1][1].view(torch.int16))
     assert torch.equal(res[0][2].view(torch.int16), res[1][2].view(torch.int16))
+
+
+def test_fused_deep_rollback_and_invalid_entries():
+    """The per-sequence commit records of the fused path: rollbacks that free
+    more table entries than a record carries (the rest read from the table),
+    batches where a planner thread owns several sequences, and a held table
+    entry or a base length that is invalid (nothing changes). Each against the
+    two-call path and the oracle."""
+    tally = Tally()
+    for B, seed in ((7, 71), (1100, 73)):
+        prob, state, bufs = _small_case(B, 3, 300, torch.float32, 0.9, seed=seed, ctx_hi=60)
+        rng = np.random.default_rng(seed)
+        drop = torch.from_numpy(rng.integers(0, 41, size=B)).int()
+        base = torch.clamp(state.seq_lens - drop, min=0).int()
+        fused = _run(prob, state, bufs, True, base=base)
+        two = _run(prob, state, bufs, False, base=base)
+        assert fused["status"] == 0
+        _same(fused, two, f"rollback{B}")
+        _check_oracle(prob, state, bufs, fused, f"rollback{B}", tally, base=base)
+    prob, state, bufs = _small_case(6, 3, 500, torch.float32, 1.0, seed=75, ctx_hi=60)
+    held = (state.seq_lens + state.block_size - 1) // state.block_size
+    b = int(torch.argmax(held))
+    bad_tab = state.clone()
+    bad_tab.tables[b, int(held[b]) - 1] = state.free_stack.numel() + 5
+    bad_base = state.seq_lens.clone()
+    bad_base[4] += 1
+    for tag, st, base in (("entry", bad_tab, None), ("base", state, bad_base)):
+        fused = _run(prob, st, bufs, True, base=base)
+        two = _run(prob, st, bufs, False, base=base)
+        assert fused["status"] == -1, tag
+        _same(fused, two, tag)
+        _check_oracle(prob, st, bufs, fused, tag, tally, base=base)
+        assert torch.equal(fused["kv_pool"].cpu(), bufs.kv_pool)
+    tally.check_share()
