@@ -572,7 +572,7 @@ int spec_chain_decide_commit(const void* tgt, int64_t ld_tgt, const void* drf, i
   f.d.accept_len = accept_len;
   f.d.out_tok = out_tok;
   f.ticket = reinterpret_cast<int32_t*>((char*)ws + ck.L.ticket);
-  f.plan_flag = f.ticket + 1;
+  f.plan_flag = f.ticket + 32;  // its own 128-byte line: the leaders' ticket atomics stay apart
   f.rec = reinterpret_cast<CommitRec*>((char*)ws + ck.L.rec);
   return cuda_status(launch_chain_fused(f, (cudaStream_t)stream));
 }

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kCopyThreads) commit_copy_planned_kernel(Commi
       unsigned ns = 64;
       for (;;) {
         __nanosleep(ns);
-        if (ns < 1024) ns <<= 1;
+        if (ns < 256) ns <<= 1;
         v = ld_relaxed(plan_flag);
         if (v || globaltimer_ns() - t0 > kWaitLimitNs) break;
       }
