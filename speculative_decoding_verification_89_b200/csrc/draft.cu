@@ -22,6 +22,7 @@
 #include <climits>
 
 #include "draw.cuh"
+#include "rowmath.cuh"
 
 namespace specv {
 
@@ -139,22 +140,28 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
 // One launch for rows that fit the cluster's shared memory
 // ---------------------------------------------------------------------------
 // A cluster of cs CTAs per row. CTA r stages its slice of the row -- whole
-// 256-element tiles [r*tc, (r+1)*tc) -- in shared memory with bulk copies, so
-// the row is read from HBM once, and finds its largest logit m_r with its
-// first index, then per tile the sum of 2^(x*c - M_r) with its own exact
-// shift M_r = fl(m_r * c_hi), and the first moment sum 2^(x*c - M_r) (x - m_r).
-// Every CTA sends (m_r, argmax, S_r, T_r) to every other CTA of the cluster
+// 256-element tiles [r*tc, (r+1)*tc) -- in shared memory by bulk copies of
+// kDfChunk bytes, each completing on its own mbarrier, so the row is read from
+// HBM once and a warp starts on its tiles as soon as their chunk has landed.
+// Per tile, in one pass: its largest logit m_t (and for a greedy row its
+// first index), the sum S_t of 2^(x*c - M_t) with the tile's integral shift
+// M_t = ceil(m_t * c_hi), and the first moment T_t = sum 2^(x*c - M_t) (x - m_t).
+// The CTA rescales its tiles to its largest shift M_r by exact powers of two
+// and sends (m_r, argmax, M_r, S_r, T_r) to every CTA of the cluster
 // (distributed shared memory); after a cluster barrier each combines them in
-// the same order -- the row's max and shift M, partition, entropy and the draw
+// the same order -- the row's max, shift, partition, entropy and the draw
 // target u * S -- and the CTA whose slice holds the target prefixes its tile
-// sums and rescans one tile in shared memory for the token. Results equal the
-// two-launch path's up to the summation order of the partition.
+// sums and rescans one tile in shared memory, with that tile's own shift, for
+// the token.
 constexpr int kDfMaxCluster = 8;
 constexpr int kDfSliceBytes = 100 * 1024;  // staged slice per CTA, at most
-constexpr uint32_t kDfChunk = 32768;        // bytes per bulk copy
+constexpr uint32_t kDfChunk = 32768;        // bytes per bulk copy (whole tiles)
+constexpr int kDfMaxChunks = (kDfSliceBytes + (int)kDfChunk - 1) / (int)kDfChunk;
+// Per tile of the slice: the scaled sum (double), then m_t, M_t, S_t, T_t.
+constexpr size_t kDfTileBytes = sizeof(double) + 4 * sizeof(float);
 
 struct DfPart {
-  float m;
+  float m, M;
   int amax;
   double S, T;
 };
@@ -177,6 +184,43 @@ __device__ __forceinline__ void smem8(const T* xs, int i0, int n, float x[8]) {
     for (int e = 0; e < 8; ++e) x[e] = i0 + e < n ? smem_elem(xs + i0 + e) : -INFINITY;
   }
 }
+// A lane's 8 staged elements as four pairs, and their largest (-inf for
+// masked entries, as staged).
+__device__ __forceinline__ float lane_pairs(const __nv_bfloat16* xs, int i0, int n,
+                                            float2 xp[4]) {
+  if (i0 + 8 <= n) {
+    const uint4 w = *reinterpret_cast<const uint4*>(xs + i0);
+    xp[0] = make_float2(bf_lo(w.x), bf_hi(w.x));
+    xp[1] = make_float2(bf_lo(w.y), bf_hi(w.y));
+    xp[2] = make_float2(bf_lo(w.z), bf_hi(w.z));
+    xp[3] = make_float2(bf_lo(w.w), bf_hi(w.w));
+    return vec_max(w, (__nv_bfloat16*)nullptr);
+  }
+  float x[8];
+  smem8(xs, i0, n, x);
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    xp[j] = make_float2(x[2 * j], x[2 * j + 1]);
+    m = fmaxf(m, fmaxf(x[2 * j], x[2 * j + 1]));
+  }
+  return m;
+}
+__device__ __forceinline__ float lane_pairs(const float* xs, int i0, int n, float2 xp[4]) {
+  float x[8];
+  smem8(xs, i0, n, x);
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    xp[j] = make_float2(x[2 * j], x[2 * j + 1]);
+    m = fmaxf(m, fmaxf(x[2 * j], x[2 * j + 1]));
+  }
+  return m;
+}
+// 2^k for an integer-valued k (0 below the double range).
+__device__ __forceinline__ double pow2d(float k) {
+  return k < -1074.0f ? 0.0 : ldexp(1.0, (int)k);
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A, int tc) {
@@ -186,12 +230,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
   const int rank = (int)cl.block_rank(), cs = (int)cl.num_blocks();
   extern __shared__ __align__(128) unsigned char dsm[];
   T* xs = reinterpret_cast<T*>(dsm);
-  double* tsum = reinterpret_cast<double*>(dsm + (size_t)tc * kResTile * sizeof(T));
-  __shared__ __align__(8) uint64_t s_bar;
+  unsigned char* tiles = dsm + (size_t)tc * kResTile * sizeof(T);
+  double* tsum = reinterpret_cast<double*>(tiles);           // S_t 2^(M_t - M_r)
+  float* tm = reinterpret_cast<float*>(tsum + tc);           // m_t
+  float* tM = tm + tc;                                       // M_t
+  float* tS = tM + tc;                                       // S_t
+  float* tT = tS + tc;                                       // T_t
+  __shared__ __align__(8) uint64_t s_bar[kDfMaxChunks];
   __shared__ DfPart s_part[kDfMaxCluster];
   __shared__ float s_wm[kDecWarps];
   __shared__ int s_wi[kDecWarps];
-  __shared__ double s_ws[kDecWarps], s_wt[kDecWarps];
+  __shared__ DfPart s_mine;
   const int b = blockIdx.y, V = A.V, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nrt = residual_tiles(V);
   const int t0 = min(nrt, rank * tc), t1 = min(nrt, t0 + tc), nt = t1 - t0;
@@ -211,91 +260,144 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
   }
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
 
-  // Stage the slice: bulk copies of its 16-byte part, plain loads of the rest.
+  // Stage the slice: bulk copies of its 16-byte part in chunks of whole
+  // tiles, plain loads of the rest (fewer than 16 bytes, at the slice's end).
   const uint32_t bytes = ((uint32_t)n * (uint32_t)sizeof(T)) & ~15u;
   const int nbulk = (int)(bytes / sizeof(T));
+  const int nchunks = (int)((bytes + kDfChunk - 1) / kDfChunk);
   if (threadIdx.x == 0) {
-    mbar_init(&s_bar, 1);
+    for (int c = 0; c < nchunks; ++c) mbar_init(&s_bar[c], 1);
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0 && bytes) {
-    mbar_arrive_expect_tx(&s_bar, bytes);
+  if (threadIdx.x == 0) {
     const unsigned char* src = reinterpret_cast<const unsigned char*>(row + e0);
-    for (uint32_t o = 0; o < bytes; o += kDfChunk)
-      bulk_g2s(dsm + o, src + o, min(kDfChunk, bytes - o), &s_bar);
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t o = (uint32_t)c * kDfChunk, len = min(kDfChunk, bytes - o);
+      mbar_arrive_expect_tx(&s_bar[c], len);
+      bulk_g2s(dsm + o, src + o, len, &s_bar[c]);
+    }
   }
   for (int i = nbulk + (int)threadIdx.x; i < n; i += blockDim.x) xs[i] = row[e0 + i];
-  if (bytes && !mbar_wait_bounded(&s_bar, 0, kWaitLimitNs)) {
-    set_status(A.status, SPEC_ETIMEOUT);
-    mbar_wait_bounded(&s_bar, 0, kWaitLimitNs);  // let the copies land before going on
-  }
-  __syncthreads();
+  __syncthreads();  // the plain-loaded end of the slice is in
 
-  // Largest logit of the slice, and for a greedy row its first index.
-  float mv = -INFINITY;
-  int mi = 0x7fffffff;
-  if (greedy) {
-    for (int i0 = (int)threadIdx.x * 8; i0 < n; i0 += blockDim.x * 8) {
+  // One pass per tile as its chunk lands: the warp takes tiles warp, warp +
+  // kDecWarps, ... in order, waiting for each chunk the first time it needs it.
+  constexpr int kTilesPerChunk = (int)kDfChunk / (kResTile * (int)sizeof(T));
+  int have = -1;  // chunks this warp has waited for
+  bool late = false;
+  float gv = -INFINITY;  // greedy rows: the warp's largest logit and its first index
+  int gi = 0x7fffffff;
+  for (int t = warp; t < nt; t += kDecWarps) {
+    const int c = min(t / kTilesPerChunk, nchunks - 1);
+    while (have < c) {
+      ++have;
+      if (!mbar_wait_bounded(&s_bar[have], 0, kWaitLimitNs)) {
+        late = true;
+        mbar_wait_bounded(&s_bar[have], 0, kWaitLimitNs);  // let the copy land before going on
+      }
+    }
+    if (greedy) {
       float x[8];
-      smem8(xs, i0, n, x);
+      smem8(xs, t * kResTile + lane * 8, n, x);
+      float v = -INFINITY;
+      int i = 0x7fffffff;
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        if (x[e] > mv) { mv = x[e]; mi = e0 + i0 + e; }
+        if (x[e] > v) { v = x[e]; i = e0 + t * kResTile + lane * 8 + e; }
+      warp_argmax(v, i);
+      if (v > gv) { gv = v; gi = i; }  // tiles in index order: the first maximum stays
+      continue;
     }
-  } else {
-    for (int i0 = (int)threadIdx.x * 8; i0 < n; i0 += blockDim.x * 8) {
-      float x[8];
-      smem8(xs, i0, n, x);
+    float2 xp[4];
+    const float tile_max = lane_pairs(xs, t * kResTile + lane * 8, n, xp);
+    float lm = tile_max;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mv = fmaxf(mv, x[e]);
-    }
-  }
-  warp_argmax(mv, mi);
-  if (lane == 0) { s_wm[warp] = mv; s_wi[warp] = mi; }
-  __syncthreads();
-  float m_r = -INFINITY;
-  int a_r = 0x7fffffff;
-  for (int w = 0; w < kDecWarps; ++w)
-    if (s_wm[w] > m_r || (s_wm[w] == m_r && s_wi[w] < a_r)) { m_r = s_wm[w]; a_r = s_wi[w]; }
-
-  // Tile sums of 2^(x*c - M_r) and the first moment about m_r.
-  double S_r = 0.0, T_r = 0.0;
-  const bool fin = m_r > -INFINITY && m_r < INFINITY;
-  if (!greedy && fin) {
-    const float Mr = __fmul_rn(m_r, sc.hi);
-    const ProbCoef kr = make_coef((double)Mr, m_r, sc);
-    double ws = 0.0, wt = 0.0;
-    for (int t = warp; t < nt; t += kDecWarps) {
-      float x[8], w[8];
-      smem8(xs, t * kResTile + lane * 8, n, x);
+    for (int o = 16; o; o >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+    float S = 0.0f, Tm = 0.0f, Mt = 0.0f;
+    if (lm > -INFINITY && lm < INFINITY) {  // a finite element (the same in every lane)
+      Mt = ceilf(lm * sc.hi);
+      // Packed: two FMAs form each pair's exponents, one ex2 per element, the
+      // sums and the first moment about lm (x - lm held at -FLT_MAX for a
+      // masked entry, whose term 0 must contribute 0).
+      const float2 chi2 = make_float2(sc.hi, sc.hi), clo2 = make_float2(sc.lo, sc.lo);
+      const float2 nM2 = make_float2(-Mt, -Mt), nm2 = make_float2(-lm, -lm);
+      float2 s2 = make_float2(0.0f, 0.0f), t2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const float2 pr = prob2(make_float2(x[e], x[e + 1]), kr);
-        w[e] = pr.x;
-        w[e + 1] = pr.y;
+      for (int j = 0; j < 4; ++j) {
+        float2 e = __ffma2_rn(xp[j], clo2, __ffma2_rn(xp[j], chi2, nM2));
+        e = make_float2(ex2(e.x), ex2(e.y));
+        s2 = __fadd2_rn(s2, e);
+        float2 d = __fadd2_rn(xp[j], nm2);
+        d = make_float2(fmaxf(d.x, -FLT_MAX), fmaxf(d.y, -FLT_MAX));
+        t2 = __ffma2_rn(e, d, t2);
       }
-      float mom = 0.0f;
+      S = s2.x + s2.y;  // fp32 over the tile: 256 terms, each at most 1
+      float mom = t2.x + t2.y;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mom += w[e] * fmaxf(x[e] - m_r, -FLT_MAX);
-      float ls = (float)lane_sum8(w);  // fp32 over the tile: values <= 1, 256 terms
-#pragma unroll
-      for (int o = 16; o; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-      if (lane == 0) tsum[t] = (double)ls;
-      ws += (double)ls;
-      wt += (double)mom;
+      for (int o = 16; o; o >>= 1) {
+        S += __shfl_xor_sync(0xffffffffu, S, o);
+        mom += __shfl_xor_sync(0xffffffffu, mom, o);
+      }
+      Tm = mom;
     }
-    wt = warp_sum_d(wt);  // ws is the same in every lane
-    if (lane == 0) { s_ws[warp] = ws; s_wt[warp] = wt; }
-    __syncthreads();
-    for (int w = 0; w < kDecWarps; ++w) { S_r += s_ws[w]; T_r += s_wt[w]; }
+    if (lane == 0) {
+      tm[t] = lm;
+      tM[t] = Mt;
+      tS[t] = S;
+      tT[t] = Tm;
+    }
   }
+  if (late && lane == 0) set_status(A.status, SPEC_ETIMEOUT);
+  if (greedy && lane == 0) { s_wm[warp] = gv; s_wi[warp] = gi; }
+  __syncthreads();
+
+  // The slice's summary (warp 0): largest logit, largest shift, and the tile
+  // sums rescaled to it by exact powers of two.
+  if (warp == 0) {
+    DfPart me{-INFINITY, 0.0f, 0x7fffffff, 0.0, 0.0};
+    if (greedy) {
+      float v = lane < kDecWarps ? s_wm[lane] : -INFINITY;
+      int i = lane < kDecWarps ? s_wi[lane] : 0x7fffffff;
+      warp_argmax(v, i);
+      me.m = v;
+      me.amax = i;
+    } else {
+      float m = -INFINITY, M = -INFINITY;
+      for (int t = lane; t < nt; t += 32) {
+        m = fmaxf(m, tm[t]);
+        if (tS[t] > 0.0f) M = fmaxf(M, tM[t]);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      }
+      double Sr = 0.0, Tr = 0.0;
+      for (int t = lane; t < nt; t += 32) {
+        double st = 0.0;
+        if (tS[t] > 0.0f) {
+          const double f = pow2d(tM[t] - M);
+          st = (double)tS[t] * f;
+          Tr += ((double)tT[t] + ((double)tm[t] - (double)m) * (double)tS[t]) * f;
+        }
+        tsum[t] = st;
+        Sr += st;
+      }
+      me.m = m;
+      me.M = M > -INFINITY ? M : 0.0f;
+      me.S = warp_sum_d(Sr);
+      me.T = warp_sum_d(Tr);
+    }
+    if (lane == 0) s_mine = me;
+  }
+  __syncthreads();
 
   // Every CTA's summary to every CTA, then the same combine everywhere.
   asm volatile("barrier.cluster.wait;" ::: "memory");
   if (threadIdx.x < cs) {
     DfPart* dst = cl.map_shared_rank(s_part, (unsigned)threadIdx.x);
-    dst[rank] = DfPart{m_r, a_r, S_r, T_r};
+    dst[rank] = s_mine;
   }
   cl.sync();
   // The combine, by one thread (the same arithmetic in every CTA).
@@ -315,20 +417,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     s_owner = -1;
     const bool ok = m > -INFINITY && m < INFINITY;
     if (ok && !greedy) {
-      const double M = (double)__fmul_rn(m, sc.hi);
+      float Mc = -INFINITY;
+      for (int r = 0; r < cs; ++r)
+        if (s_part[r].S > 0.0) Mc = fmaxf(Mc, s_part[r].M);
       double f[kDfMaxCluster];
       double S = 0.0, Tm = 0.0;
       for (int r = 0; r < cs; ++r) {
         f[r] = 0.0;
         if (s_part[r].S > 0.0) {
-          const float mr = s_part[r].m;
-          f[r] = exp2((double)__fmul_rn(mr, sc.hi) - M);
+          f[r] = pow2d(s_part[r].M - Mc);
           S += s_part[r].S * f[r];
-          Tm += (s_part[r].T + ((double)mr - (double)m) * s_part[r].S) * f[r];
+          Tm += (s_part[r].T + ((double)s_part[r].m - (double)m) * s_part[r].S) * f[r];
         }
       }
-      const double Mcm = (M - (double)m * (double)sc.hi) - (double)m * (double)sc.lo;
-      s_Lt = M + log2(S);
+      // Lt = Mc + log2 S; H = ln2 (Lt - c E[l]) with E[l] = m + Tm / S.
+      const double Mcm = ((double)Mc - (double)m * (double)sc.hi) - (double)m * (double)sc.lo;
+      s_Lt = (double)Mc + log2(S);
       s_H = kLn2 * (Mcm + log2(S) - sc.d * (Tm / S));
       const float u =
           spec_uniforms(A.seed, (uint32_t)A.seq_id[b], A.round, (uint32_t)A.pos[b], 0u).y;
@@ -362,7 +466,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
   if (rank != owner) return;
 
   // Owner: the tile (warp 0 prefixes the tile sums: a contiguous run per
-  // lane, then a scan over the lanes), then the element.
+  // lane, then a scan over the lanes), then the element, with the tile's own
+  // shift and the same rescaling as its sum.
   if (warp == 0) {
     const int per = (nt + 31) / 32;
     const int a0 = min(nt, lane * per), a1 = min(nt, a0 + per);
@@ -387,17 +492,21 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     const int tile = best < 0 ? 0 : best;
     const unsigned holder = __ballot_sync(0xffffffffu, cand == best && best >= 0);
     const double pre = holder ? __shfl_sync(0xffffffffu, c_cand, __ffs(holder) - 1) : 0.0;
-    const float Mr = __fmul_rn(s_part[owner].m, sc.hi);
-    const ProbCoef kr = make_coef((double)Mr, s_part[owner].m, sc);
-    float x[8], w[8];
-    smem8(xs, tile * kResTile + lane * 8, n, x);
+    const double ft = pow2d(tM[tile] - s_part[owner].M);
+    float2 xp[4];
+    lane_pairs(xs, tile * kResTile + lane * 8, n, xp);
+    float w[8];
+    {
+      const float2 chi2 = make_float2(sc.hi, sc.hi), clo2 = make_float2(sc.lo, sc.lo);
+      const float2 nM2 = make_float2(-tM[tile], -tM[tile]);
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float2 pr = prob2(make_float2(x[e], x[e + 1]), kr);
-      w[e] = pr.x;
-      w[e + 1] = pr.y;
+      for (int j = 0; j < 4; ++j) {
+        const float2 e = __ffma2_rn(xp[j], clo2, __ffma2_rn(xp[j], chi2, nM2));
+        w[2 * j] = ex2(e.x);
+        w[2 * j + 1] = ex2(e.y);
+      }
     }
-    const double ls = lane_sum8(w);
+    const double ls = lane_sum8(w) * ft;
     double li = ls;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -409,7 +518,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     if (start <= local) {
       double acc = start;
       for (int e = 0; e < 8; ++e) {
-        acc += (double)w[e];
+        acc += (double)w[e] * ft;
         if (acc > local && w[e] > 0.0f) { found = tile * kResTile + lane * 8 + e; break; }
       }
     }
@@ -444,7 +553,7 @@ static cudaError_t launch_draw(const DraftArgs& a, cudaStream_t st) {
 template <typename T>
 static cudaError_t launch_fused_draw(const DraftArgs& a, int cs, int tc, cudaStream_t st) {
   auto k = draft_fused_kernel<T>;
-  const size_t smem = (size_t)tc * kResTile * sizeof(T) + (size_t)tc * sizeof(double);
+  const size_t smem = (size_t)tc * kResTile * sizeof(T) + (size_t)tc * kDfTileBytes;
   const cudaError_t e = reserve_dyn_smem(k, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl_cluster(k, dim3(cs, a.B), dim3(kDecThreads), smem, st, (unsigned)cs, a, tc);
@@ -459,7 +568,7 @@ cudaError_t launch_draft_step(int dtype, const unsigned char* lg, long long ld_b
   const int esz = dtype == SPEC_BF16 ? 2 : 4, nrt = residual_tiles(V);
   for (int cs = 4; cs <= kDfMaxCluster; cs *= 2) {
     const int tc = (nrt + cs - 1) / cs;
-    if ((size_t)tc * kResTile * esz + (size_t)tc * sizeof(double) > (size_t)kDfSliceBytes) continue;
+    if ((size_t)tc * kResTile * esz > (size_t)kDfSliceBytes) continue;
     DraftArgs a{};
     a.B = B;
     a.V = V;
