@@ -217,9 +217,10 @@ __device__ __forceinline__ float lane_pairs(const float* xs, int i0, int n, floa
   }
   return m;
 }
-// 2^k for an integer-valued k (0 below the double range).
+// 2^k for an integer-valued k <= 0, built from its exponent bits (0 below
+// the normal double range, where a term is negligible beside the largest).
 __device__ __forceinline__ double pow2d(float k) {
-  return k < -1074.0f ? 0.0 : ldexp(1.0, (int)k);
+  return k < -1022.0f ? 0.0 : __longlong_as_double((long long)(1023 + (int)k) << 52);
 }
 
 template <typename T>
@@ -259,6 +260,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     return;
   }
   const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+  // The draw's uniform, formed now so that the combine does not wait for it.
+  __shared__ float s_u;
+  if (threadIdx.x == 0 && !greedy)
+    s_u = spec_uniforms(A.seed, (uint32_t)A.seq_id[b], A.round, (uint32_t)A.pos[b], 0u).y;
 
   // Stage the slice: bulk copies of its 16-byte part in chunks of whole
   // tiles, plain loads of the rest (fewer than 16 bytes, at the slice's end).
@@ -311,9 +316,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
     }
     float2 xp[4];
     const float tile_max = lane_pairs(xs, t * kResTile + lane * 8, n, xp);
-    float lm = tile_max;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+    float lm;  // the tile's largest logit in every lane: one warp reduction (sm_100a)
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(lm) : "f"(tile_max));
     float S = 0.0f, Tm = 0.0f, Mt = 0.0f;
     if (lm > -INFINITY && lm < INFINITY) {  // a finite element (the same in every lane)
       Mt = ceilf(lm * sc.hi);
@@ -432,11 +436,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_fused_kernel(DraftArgs A
       }
       // Lt = Mc + log2 S; H = ln2 (Lt - c E[l]) with E[l] = m + Tm / S.
       const double Mcm = ((double)Mc - (double)m * (double)sc.hi) - (double)m * (double)sc.lo;
-      s_Lt = (double)Mc + log2(S);
-      s_H = kLn2 * (Mcm + log2(S) - sc.d * (Tm / S));
-      const float u =
-          spec_uniforms(A.seed, (uint32_t)A.seq_id[b], A.round, (uint32_t)A.pos[b], 0u).y;
-      const double target = (double)u * S;
+      const double l2S = log2(S);
+      s_Lt = (double)Mc + l2S;
+      s_H = kLn2 * (Mcm + l2S - sc.d * (Tm / S));
+      const double target = (double)s_u * S;
       // The CTA whose slice holds the target: the first whose running total passes it.
       double cum = 0.0;
       for (int r = 0; r < cs; ++r) {
