@@ -246,7 +246,9 @@ int spec_commit_paged(int B, int block_size, int max_blocks,
  * (a + 1 rows kept per sequence: the accepted drafts and the drawn token),
  * in three launches instead of four: the row statistics; one cluster per
  * sequence for the check and the draw, whose last sequence to finish its
- * accept test plans the commit; the copy of the kept K/V and hidden rows.
+ * accept test plans the commit from per-sequence records; the copy of the
+ * kept K/V and hidden rows, which starts while the draws run, as soon as the
+ * plan is written.
  * Arguments: those of spec_verify_chain (the logits, drafts, temperatures,
  * Philox key, accept_len, out_tok, diag, workspace) and of spec_commit_paged
  * (tables, lengths, base_len, stack, pool, stage and hidden buffers), with
