@@ -27,6 +27,8 @@ def main():
     ap.add_argument("--B", type=int, default=32)
     ap.add_argument("--iters", type=int, default=6)
     ap.add_argument("--commit", action="store_true", help="also run the paged commit")
+    ap.add_argument("--fused", action="store_true",
+                    help="spec_verify_chain_commit on a small pool (4 layers, contexts 256-1024)")
     ap.add_argument("--no-verify", action="store_true", help="commit only (random accept lengths)")
     ap.add_argument("--outcome", type=int, default=-1,
                     help="run the outcome law with this many outcomes instead of verifying")
@@ -43,6 +45,9 @@ def main():
         prob = W.chain_batch(device=dev, B=B)
         ws = capi.workspace(B, K, V, torch.bfloat16, device=dev)
         out = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    if args.fused:
+        state, bufs = W.commit_setup(B, K, ctx_lo=256, ctx_hi=1024, layers=4, device=dev)
+        base = state.seq_lens.clone()
     if args.commit:
         state, bufs = W.commit_setup(B, K, device=dev)
         base = state.seq_lens.clone()
@@ -54,7 +59,15 @@ def main():
     times = []
     for i in range(args.iters):
         ev[0].record()
-        if not args.no_verify:
+        if args.fused:
+            capi.spec_verify_chain_commit(prob.tgt, prob.drf, prob.draft_tok, prob.temperature,
+                                          prob.seed, prob.seq_id, i, acc, out, state.tables,
+                                          state.seq_lens, base, state.free_stack,
+                                          state.free_top, st, ws, block_size=16,
+                                          kv_stage=bufs.kv_stage, kv_pool=bufs.kv_pool,
+                                          hid_stage=bufs.hid_stage, hid_out=bufs.hid_out,
+                                          hid_off=bufs.hid_off)
+        elif not args.no_verify:
             capi.spec_verify_chain(prob.tgt, prob.drf, prob.draft_tok, prob.temperature, prob.seed,
                                    prob.seq_id, i, acc, out, st, ws)
         elif args.commit:
