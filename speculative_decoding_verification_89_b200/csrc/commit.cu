@@ -72,7 +72,7 @@ cudaError_t launch_commit_copy_planned(const CommitArgs& a, const int32_t* plan_
   const size_t smem = (2 * (size_t)a.B + 1) * sizeof(int);
   cudaError_t e = reserve_dyn_smem(commit_copy_planned_kernel, smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(commit_copy_planned_kernel, dim3(sm_count() * kCopyCtasPerSm),
+  return launch_pdl(commit_copy_planned_kernel, dim3(sm_count() * kCopyCtasPerSmPlanned),
                     dim3(kCopyThreads), smem, st, a, plan_flag);
 }
 

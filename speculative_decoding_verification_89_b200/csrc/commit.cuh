@@ -12,6 +12,10 @@ namespace specv {
 constexpr int kPlanThreads = 1024;
 constexpr int kCopyThreads = 256;
 constexpr int kCopyCtasPerSm = 8;  // 64 warps per SM: one round of items for most calls
+// The copy launch that starts beside the decide launch finds room for few CTAs
+// until the decide CTAs leave; 4 per SM measured best there (8 after a plain
+// planner launch).
+constexpr int kCopyCtasPerSmPlanned = 4;
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
