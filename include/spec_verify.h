@@ -531,6 +531,17 @@ int spec_vp_pick(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_dr
  * device-wide setting: calls on other streams see it too. */
 int spec_test_set_wait_limit_ns(uint64_t ns);
 
+/* Test hook (no counterpart in the paper): the limit of the wait, in
+ * nanoseconds (2e9 by default), of spec_verify_chain_commit's copy launch for
+ * the plan word that its decide launch's planner sets. 0 makes the wait one
+ * poll, so copy CTAs that start before the plan is written run out: they
+ * record SPEC_ETIMEOUT in dev_status and copy nothing. The verification
+ * outputs stand; the plan is made in full, or not at all when the timeout is
+ * recorded before the planner reads the status word; kept rows may be left
+ * uncopied. Set it
+ * back to 2000000000 afterwards; a device-wide setting, as above. */
+int spec_test_set_copy_wait_limit_ns(uint64_t ns);
+
 /* Test hook of spec_verify_chain_noalloc (no counterpart in the paper):
  * forgets every kept scratch address and makes the next n address lookups
  * fail as a lookup inside a stream capture does (SPEC_ECUDA), so a test can

@@ -68,6 +68,7 @@ _SIGS = {
                           _p, _p, _p, _p, _sz, _p]),
     "spec_noalloc_test_fail_lookups": (_i, [_i]),
     "spec_test_set_wait_limit_ns": (_i, [_u64]),
+    "spec_test_set_copy_wait_limit_ns": (_i, [_u64]),
     "spec_draft_workspace_bytes": (_sz, [_i, _i, _i]),
     "spec_outcome_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spec_outcome_law": (_i, [_p, _i64, _p, _i64, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p,

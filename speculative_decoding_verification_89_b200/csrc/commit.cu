@@ -18,6 +18,11 @@
 
 namespace specv {
 
+// Limit of the planned copy launch's wait for the plan word: kWaitLimitNs
+// unless a test has set another with spec_test_set_copy_wait_limit_ns (0:
+// one poll, so a plan not yet written makes the wait run out).
+__device__ unsigned long long g_copy_wait_limit_ns = kWaitLimitNs;
+
 __global__ void __launch_bounds__(kPlanThreads) commit_plan_kernel(CommitArgs a) {
   pdl_begin();
   extern __shared__ int s_seq[];
@@ -46,13 +51,14 @@ __global__ void __launch_bounds__(kCopyThreads) commit_copy_planned_kernel(Commi
   if (threadIdx.x == 0) {
     int v = ld_relaxed(plan_flag);
     if (!v) {
+      const uint64_t limit = g_copy_wait_limit_ns;
       const uint64_t t0 = globaltimer_ns();
       unsigned ns = 64;
       for (;;) {
         __nanosleep(ns);
         if (ns < 256) ns <<= 1;
         v = ld_relaxed(plan_flag);
-        if (v || globaltimer_ns() - t0 > kWaitLimitNs) break;
+        if (v || globaltimer_ns() - t0 > limit) break;
       }
     }
     if (v) fence_acq_rel();  // the planner's writes are visible from here on
@@ -111,3 +117,12 @@ cudaError_t launch_philox(uint64_t seed, const uint32_t* ctr, int n, float* out,
 }
 
 }  // namespace specv
+
+#pragma GCC visibility push(default)
+extern "C" int spec_test_set_copy_wait_limit_ns(uint64_t ns) {
+  const unsigned long long v = ns;
+  const cudaError_t e = cudaMemcpyToSymbol(specv::g_copy_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return specv::record_cuda_status(e);
+  return SPEC_OK;
+}
+#pragma GCC visibility pop

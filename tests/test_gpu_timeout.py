@@ -35,3 +35,39 @@ def test_wait_timeout_records_status_and_commits_nothing():
     assert r2["status"] == 0
     _check_oracle(prob, state, bufs, r2, "after-timeout", tally)
     tally.check_share()
+
+
+def test_copy_wait_timeout_records_status():
+    """The verify-and-commit copy launch's bounded wait for the plan word,
+    run out on purpose (limit 0: one poll, while the decide launch has not yet
+    planned): SPEC_ETIMEOUT, the verification outputs as in a normal call, the
+    plan made in full or not at all (a timeout recorded before the planner
+    reads the status word stops it, as any earlier error does), and the next
+    normal call on the same stream matches the oracle."""
+    from speculative_decoding_verification_89_b200 import capi
+    prob = W.chain_batch(device="cuda")
+    state, bufs = W.commit_setup(64, 8, device="cuda")
+    state = W.PagedState(state.tables.cpu(), state.seq_lens.cpu(), state.free_stack.cpu(),
+                         state.free_top.cpu(), 16)
+    ref = _run(prob, state, bufs, True)
+    assert ref["status"] == 0
+    assert capi._lib.spec_test_set_copy_wait_limit_ns(0) == capi.SPEC_OK
+    try:
+        r = _run(prob, state, bufs, True)
+    finally:
+        assert capi._lib.spec_test_set_copy_wait_limit_ns(2_000_000_000) == capi.SPEC_OK
+    assert r["status"] == capi.SPEC_ETIMEOUT
+    for k in ("acc", "out"):
+        assert torch.equal(r[k], ref[k]), k
+    assert torch.equal(torch.nan_to_num(r["diag"], nan=-99.0),
+                       torch.nan_to_num(ref["diag"], nan=-99.0))
+    planned = torch.equal(r["tables"], ref["tables"])
+    before = dict(tables=state.tables, seq_lens=state.seq_lens, free_stack=state.free_stack,
+                  free_top=state.free_top)
+    for k in ("tables", "seq_lens", "free_stack", "free_top"):
+        assert torch.equal(r[k], ref[k] if planned else before[k]), (k, planned)
+    tally = Tally()
+    r2 = _run(prob, state, bufs, True)
+    assert r2["status"] == 0
+    _check_oracle(prob, state, bufs, r2, "after-copy-timeout", tally)
+    tally.check_share()
