@@ -845,10 +845,13 @@ def run_cfg_hier(dev, peak, kind, rounds):
 def run_cfg_engine(dev, rounds=256):
     """Engine loop: 64 sequences x 256 rounds, K = N_i = 4, V=32000 bf16,
     logits regenerated each round from a generator seeded by (4, round); each
-    round reserves the cycle's slots in the block tables, verifies, commits
-    the committed tokens and rolls the reservation back (block 16, pool of
-    65536 blocks, starts U[128, 2048]). Committed tokens per second of the
-    device work, with and without the round's logit generation."""
+    round reserves the cycle's slots in the block tables, drafts its K tokens
+    per sequence from the L_d rows with the library's draft step (the K rows
+    of each window gathered, one draw per row with the Philox counter
+    (sequence, round, slot)), verifies, commits the committed tokens and
+    rolls the reservation back (block 16, pool of 65536 blocks, starts
+    U[128, 2048]). Committed tokens per second of the device work, with and
+    without the round's logit generation."""
     from speculative_decoding_verification_89_b200 import capi
     from speculative_decoding_verification_89_b200 import workloads as W
     B, K, Ni, V = 64, 4, 4, 32000
@@ -862,6 +865,12 @@ def run_cfg_engine(dev, rounds=256):
     full = torch.full((B,), S, dtype=torch.int32, device=dev)
     loop = HierLoop(B, K, Ni, V, torch.bfloat16, dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
+    draft_rows = torch.empty((B * K, V), dtype=torch.bfloat16, device=dev)
+    draft_ws = capi.draft_workspace(B * K, V, torch.bfloat16, device=dev)
+    draft_sid = seq_id.repeat_interleave(K)
+    draft_T = torch.ones(B * K, device=dev)
+    draft_tok = torch.empty(B * K, dtype=torch.int32, device=dev)
+    kk = torch.arange(K, device=dev).view(1, K)
     ms_work = ms_all = 0.0
     total = 0
     for r in range(rounds):
@@ -873,8 +882,12 @@ def run_cfg_engine(dev, rounds=256):
         w0.record()
         capi.spec_commit_paged(state.tables, state.seq_lens, committed, full, 0,
                                state.free_stack, state.free_top, S, st, block_size=16)
-        drafts = W.window_drafts(loop.lg[0], loop.win_len, K, T, W.generator(40 + r, dev))
-        loop.call(drafts, T, 4, seq_id, r)
+        slots = loop.win_len.long().view(B, 1) + kk  # the window's next K slots
+        torch.gather(loop.lg[0], 1, slots.view(B, K, 1).expand(B, K, V),
+                     out=draft_rows.view(B, K, V))
+        capi.spec_draft_sample(draft_rows, draft_T, 40, draft_sid, r,
+                               slots.view(-1).to(torch.int32), draft_tok, st, draft_ws)
+        loop.call(draft_tok.view(B, K), T, 4, seq_id, r)
         capi.spec_commit_paged(state.tables, state.seq_lens, committed, loop.cn, 0,
                                state.free_stack, state.free_top, S, st, block_size=16)
         committed.copy_(state.seq_lens)
@@ -886,8 +899,9 @@ def run_cfg_engine(dev, rounds=256):
         total += int(loop.cn.sum().item())
     if int(st.item()) != 0 or int(loop.status.item()) != 0:
         raise RuntimeError("engine loop: device status")
-    return {"workload": "engine loop 64 sequences x 256 rounds, K=N_i=4, V=32000 bf16, paged "
-                        "commit/rollback every round (block 16, pool 65536)",
+    return {"workload": "engine loop 64 sequences x 256 rounds, K=N_i=4, V=32000 bf16, drafts "
+                        "by the draft step, paged commit/rollback every round (block 16, pool "
+                        "65536)",
             "rounds": rounds, "committed_tokens": total,
             "committed_tokens_per_s": total / (ms_work * 1e-3),
             "committed_tokens_per_s_with_logit_generation": total / (ms_all * 1e-3),
