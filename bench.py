@@ -762,9 +762,11 @@ def _timed(fn):
     return e0, e1
 
 
-def run_cfg_chain_small(dev):
+def run_cfg_chain_small(dev, dist):
     """Chain verification, B=1, K=4, V=1024 fp32, T=1, fresh logits every
-    round for 100 rounds: latency of one spec_verify_chain call."""
+    round for 100 rounds: latency of one spec_verify_chain call, as called
+    from Python (events around each call) and on the device alone (the 100
+    calls captured in a CUDA graph and replayed)."""
     from speculative_decoding_verification_89_b200 import capi
     from speculative_decoding_verification_89_b200 import workloads as W
     probs = [W.chain_small(rnd=r, device=dev) for r in range(100)]
@@ -784,11 +786,13 @@ def run_cfg_chain_small(dev):
     torch.cuda.synchronize()
     us = [a.elapsed_time(b) * 1e3 for a, b in ev]
     tokens = float((acc.cpu().numpy() + 1).sum())
+    us_graph = graph_us_per_call([lambda i=i: call(probs[i], i) for i in range(100)], 20, dist)
     if int(st.item()) != 0:
         raise RuntimeError("chain small: device status")
     return {"workload": "chain verification B=1, K=4, V=1024 fp32 (N(0,4) targets, drafts "
                         "+N(0,1), T=1), fresh logits each of 100 rounds",
             "us_per_round_median": statistics.median(us), "us_per_round_mean": statistics.mean(us),
+            "us_per_round_graph": us_graph,
             "tokens_per_s": tokens / (sum(us) * 1e-6), "rounds": 100,
             "bound": "latency (9 rows of 4 KB; two launches)", "gpu_launches_per_round": 2}
 
@@ -1090,7 +1094,7 @@ def run_configs(args, dev, dist, peak, head):
     the oracle's throughput on one host core and on all of them."""
     with_oracle = dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline
     out = {
-        "cfg1_chain_small": run_cfg_chain_small(dev),
+        "cfg1_chain_small": run_cfg_chain_small(dev, dist),
         "cfg2_hier_peaked": run_cfg_hier(dev, peak, "peaked", rounds=24),
         "cfg3_chain_commit": {"workload": "the headline step", "tokens_per_s": head["value"],
                               "ms_per_step": head["ms_per_step"], "hbm_gbs": head["hbm_gbs"],
