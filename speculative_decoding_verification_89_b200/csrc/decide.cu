@@ -15,8 +15,9 @@
 // The CTAs combine the tile partials of the sequence's rows (a warp per row)
 // into the leader CTA's shared memory (distributed shared memory), meet at a
 // cluster barrier, each run the accept test on all positions (a lane per
-// position, ballot for the first rejection), split the residual row pair
-// between them and write their tile sums into the leader, meet again, and the
+// position, ballot for the first rejection), take groups of residual tiles of
+// the row pair from a counter in the leader (so the CTAs that share an SM with
+// another take fewer) and write their tile sums into the leader, meet again, and the
 // leader prefixes the tile sums, finds the tile holding u' * Z, rescans that
 // one tile and writes the outputs. No spinning and no second launch; the
 // variant that also plans a paged commit (chain_decide_commit_kernel, at the
@@ -180,6 +181,8 @@ struct Outcome {
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecideArgs A) {
   pdl_begin();
+  __shared__ int s_claim;
+  if (threadIdx.x == 0) s_claim = 0;  // the leader's: residual groups claimed so far
   cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
@@ -236,9 +239,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
     qrow = o.a < K ? dp(o.a) : nullptr;
     kp = make_coef(lsh->M[o.a] + lsh->L[o.a], lsh->m[o.a], sc);
     kq = o.a < K ? make_coef(dl(o.a), lsh->m[K + 1 + o.a], sc) : make_coef(0.0, 0.0f, sc);
-    const int chunk = (nrt + kCluster - 1) / kCluster;
-    residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, (int)rank * chunk),
-                          min(nrt, ((int)rank + 1) * chunk), ltsum);
+    residual_tile_sums_claimed<T>(prow, qrow, V, kp, kq, nrt, ltsum,
+                                  cl.map_shared_rank(&s_claim, 0));
   }
   cl.sync();  // every tile sum is in the leader
   if (rank != 0) return;
@@ -485,9 +487,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) hier2_decide_kernel(HierDecide
 // Once its accept test is done the leader writes the kept count (a + 1) and
 // takes a ticket (one atomic, never awaited): the CTA that takes the B-th
 // ticket has seen every kept count and runs the commit planner (tables, free
-// stack, lengths, hidden offsets). The leader takes no residual tiles -- the
-// other kCluster - 1 CTAs sum them -- so the planner, which overlaps the
-// other sequences' draws, delays nothing but its own sequence's draw. The
+// stack, lengths, hidden offsets). The leader joins the residual tiles only
+// after its ticket (and the planner after the plan), taking groups from the
+// same counter as the other CTAs, so the planner, which overlaps the other
+// sequences' draws, delays nothing but its own sequence's draw. The
 // copy launch after this one moves the kept K/V and hidden rows: it starts
 // while this launch runs and waits for plan_flag, which the first CTA clears
 // before it lets that launch start and the planner sets when it is done.
@@ -502,12 +505,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
     __syncthreads();  // cleared before any thread of this CTA lets the copy launch start
   }
   grid_dependents_launch();
+  __shared__ int s_last, s_claim;
+  if (threadIdx.x == 0) s_claim = 0;  // the leader's: residual groups claimed so far
   cluster_arrive_relaxed();  // paired with the wait in cluster_rows
   cg::cluster_group cl = cg::this_cluster();
   const unsigned rank = cl.block_rank();
   __shared__ SeqShared sh;
   __shared__ Outcome s_out;
-  __shared__ int s_last;
   extern __shared__ double dyn[];  // leader: [nrt] tile sums, [nrt] prefixes; planner: 3B ints
   SeqShared* lsh = cl.map_shared_rank(&sh, 0);
   double* ltsum = cl.map_shared_rank(dyn, 0);
@@ -600,21 +604,18 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_commit_kernel(Fus
       }
     }
   }
-  // Residual tile sums of a sampled sequence, split over the CTAs but the leader.
+  // Residual tile sums of a sampled sequence: groups claimed by every CTA of the cluster.
   const bool draw = !o.bad && !greedy;
   const T* prow = nullptr;
   const T* qrow = nullptr;
   ProbCoef kp{}, kq{};
-  constexpr int kWorkers = kCluster - 1;
   if (draw) {
     prow = tp(a);
     qrow = a < K ? dp(a) : nullptr;
     kp = make_coef(lsh->M[a] + lsh->L[a], lsh->m[a], sc);
     kq = a < K ? make_coef(dl(a), lsh->m[K + 1 + a], sc) : make_coef(0.0, 0.0f, sc);
-    const int chunk = (nrt + kWorkers - 1) / kWorkers, wr = (int)rank - 1;
-    if (wr >= 0)
-      residual_tile_sums<T>(prow, qrow, V, kp, kq, min(nrt, wr * chunk),
-                            min(nrt, (wr + 1) * chunk), ltsum);
+    residual_tile_sums_claimed<T>(prow, qrow, V, kp, kq, nrt, ltsum,
+                                  cl.map_shared_rank(&s_claim, 0));
   }
   // The tile sums are in the leader once every CTA has arrived; only the
   // leader waits.

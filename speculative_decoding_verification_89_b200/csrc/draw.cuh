@@ -191,6 +191,57 @@ __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const Pr
   }
 }
 
+// Same, with the groups of kResGroup tiles claimed one at a time from a
+// counter (any shared memory of the cluster) by every warp that calls it.
+template <typename T>
+__device__ void residual_tile_sums_claimed(const T* prow, const T* qrow, int V,
+                                           const ProbCoef& kp, const ProbCoef& kq, int nrt,
+                                           double* out, int* claim) {
+  constexpr int G = kResGroup<T>;
+  const int lane = threadIdx.x & 31;
+  const bool hq = qrow != nullptr;
+  const int ngroups = (nrt + G - 1) / G;
+  for (;;) {
+    int g = 0;
+    if (lane == 0) g = atomicAdd(claim, 1);
+    g = __shfl_sync(0xffffffffu, g, 0);
+    if (g >= ngroups) break;
+    const int tb = g * G;
+    Raw8<T> rp[G], rq[G];
+    bool full[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      const int e0 = (tb + u) * kResTile + lane * 8;
+      full[u] = tb + u < nrt && e0 + 8 <= V;
+      rp[u] = raw8(prow, e0, full[u]);
+      rq[u] = raw8(hq ? qrow : prow, e0, full[u] && hq);
+    }
+    double s[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      const int t = tb + u, e0 = t * kResTile + lane * 8;
+      float w[8];
+      if (full[u]) {
+        float xp[8], xq[8];
+        unpack8(rp[u], xp);
+        unpack8(rq[u], xq);
+        weights_of(xp, xq, hq, kp, kq, w);
+      } else if (t < nrt && e0 < V) {
+        weights8<T>(prow, qrow, e0, V, kp, kq, w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = 0.0f;
+      }
+      s[u] = lane_sum8(w);
+    }
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      const double v = warp_sum_d(s[u]);
+      if (lane == 0 && tb + u < nrt) out[tb + u] = v;
+    }
+  }
+}
+
 // Leader: given all tile sums in shared memory (tsum), prefix them in a fixed
 // order, locate u * Z, rescan that tile and return the drawn token in every
 // thread (-1 if the weights have no mass). *Z_out gets Z. A caller that owns
