@@ -69,8 +69,8 @@ constexpr int kStackCache = 2048;  // stack entries popped from below the old to
 // planner runs (the verify-and-commit decide launch's leader of the sequence,
 // once its accept test is done): the table entries it holds, checked, its new
 // length and the first entries to be freed. The planner then reads one record
-// per sequence instead of the lengths and the whole table row.
-// (CommitRec, kernels.cuh)
+// per sequence instead of the lengths and the whole table row. The record's
+// layout, CommitRec, is declared with CommitArgs.
 
 // Whole CTA; old_len = seq_lens[b]. The checks are plan_body's, per sequence.
 static __device__ void commit_record(const CommitArgs& a, int b, int old_len, int kept,
