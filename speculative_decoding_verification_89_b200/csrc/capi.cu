@@ -358,9 +358,12 @@ const char* spec_status_string(int status) {
 }
 
 // Leading positions whose rows the row-statistics kernel streams last, so
-// the draw that follows finds them in L2: as many (at most 2) as fit in 60%
-// of the L2 with rows_per_pos rows per position and sequence.
-static int late_positions(int B, int V, int dtype, int rows_per_pos, int cap = 2) {
+// the draw that follows finds them in L2: as many (at most cap) as fit in 60%
+// of the L2 with rows_per_pos rows per position and sequence. At B=64, K=8,
+// V=128256 bf16 one position measured best: the verify-and-commit step
+// 82.4 us with one, 83.2 with two, 84.4 with three, 90.2 with none; the
+// outcome law 155.9 us with one, 158.4 with two, 163.0 with three.
+static int late_positions(int B, int V, int dtype, int rows_per_pos, int cap = 1) {
   static int l2s[kMaxDevs];  // bytes per device, looked up once per device (0: unknown)
   static bool known[kMaxDevs];
   const int dev = current_device();
@@ -396,10 +399,7 @@ int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64
   rows.ld_drf = ld_drf * es;
   rows.temperature = temperature;
   rows.K = K;
-  // The rows of the first position are streamed last (cap 1): at B=64, K=8,
-  // V=128256 bf16 the verify-and-commit step measured 82.4 us with one late
-  // position, 83.2 with two, 84.4 with three and 90.2 with none.
-  rows.late_pos = late_positions(B, V, dtype, 2, 1);
+  rows.late_pos = late_positions(B, V, dtype, 2);
   RsBuffers rb = rs_buffers(ws, ck.L);
   rb.zero = reinterpret_cast<int32_t*>((char*)ws + ck.L.ticket);  // for spec_chain_decide_commit
   return cuda_status(launch_row_stats(dtype, rows, B * (2 * K + 1), V, rb, dev_status,
