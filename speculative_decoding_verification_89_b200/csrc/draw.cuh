@@ -30,6 +30,11 @@ constexpr int kDecWarps = kDecThreads / 32;
 // lane and row).
 template <typename T>
 constexpr int kResGroup = sizeof(T) == 2 ? 4 : 2;
+// Groups claimed from a counter are smaller: the finer hand-out balances the
+// CTAs of a cluster better (B=64, K=8, V=128256 bf16 verify-and-commit step:
+// 80.4 us with 2 tiles per group, 81.3 with 1 or 3, 82.4 with 4).
+template <typename T>
+constexpr int kResClaimGroup = 2;
 
 // ---------------------------------------------------------------------------
 // Residual weights of 8 consecutive elements
@@ -191,13 +196,13 @@ __device__ void residual_tile_sums(const T* prow, const T* qrow, int V, const Pr
   }
 }
 
-// Same, with the groups of kResGroup tiles claimed one at a time from a
+// Same, with groups of kResClaimGroup tiles claimed one at a time from a
 // counter (any shared memory of the cluster) by every warp that calls it.
 template <typename T>
 __device__ void residual_tile_sums_claimed(const T* prow, const T* qrow, int V,
                                            const ProbCoef& kp, const ProbCoef& kq, int nrt,
                                            double* out, int* claim) {
-  constexpr int G = kResGroup<T>;
+  constexpr int G = kResClaimGroup<T>;
   const int lane = threadIdx.x & 31;
   const bool hq = qrow != nullptr;
   const int ngroups = (nrt + G - 1) / G;
