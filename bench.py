@@ -801,8 +801,11 @@ def run_cfg_hier(dev, peak, kind, rounds):
     """Two-stage verification as a rolling loop (the window carries from call
     to call): kind 'peaked' = B=8, V=32000 bf16, T=0.7 with one greedy
     sequence; kind 'mixed' = B=256, V=151936 fp32, T ~ U(0, 1.2] with 51
-    greedy sequences. Each call is timed alone (events around it); the row
-    redraw and the drafts are outside."""
+    greedy sequences. Each call is timed alone with events around it, the
+    row redraw and the drafts outside: us_per_call as called from Python
+    (a small call's pace is then set by its launches), us_per_call_device
+    the same rounds again with the call's launches queued behind a short
+    device sleep, so that the events see the device time alone."""
     from speculative_decoding_verification_89_b200 import workloads as W
     if kind == "peaked":
         base = W.hier_peaked(device=dev)
@@ -815,34 +818,51 @@ def run_cfg_hier(dev, peak, kind, rounds):
         dtype, desc = torch.float32, ("two-stage verification B=256, K=N_i=4, V=151936 fp32, "
                                       "T ~ U(0,1.2] with 51 greedy sequences")
     B, K, Ni, V = base.lg_f.shape[0], base.K, base.Ni, base.lg_f.shape[2]
-    loop = HierLoop(B, K, Ni, V, dtype, dev)
     T = base.temperature.to(dev)
     greedy = (base.temperature == 0).cpu().numpy()
     esz = torch.tensor([], dtype=dtype).element_size()
-    ms = 0.0
-    rows = committed = calls = 0
-    for r in range(rounds + 3):
-        fresh = [base.lg_d, base.lg_i, base.lg_f] if r == 0 else list(
-            W.hier_logits(B, loop.S, V, dtype, W.generator(9000 + r, dev), dev, **kw))
-        loop.logits(fresh)
-        w_before = loop.win_len.cpu().numpy()
-        drafts = W.window_drafts(loop.lg[0], loop.win_len, K, T, W.generator(40 + r, dev))
-        e0, e1 = _timed(lambda: loop.call(drafts, T, base.seed, base.seq_id, r))
-        torch.cuda.synchronize()
-        if r >= 3:  # the first rounds fill the windows
-            ms += e0.elapsed_time(e1)
-            rows += loop.rows_read(w_before, greedy)
-            committed += int(loop.cn.sum().item())
-            calls += 1
-    if int(loop.status.item()) != 0:
-        raise RuntimeError(f"two-stage {kind}: device status")
+
+    def rolling(ahead):
+        """The rounds from fresh windows; returns (ms, rows, committed, calls,
+        hashable outputs)."""
+        loop = HierLoop(B, K, Ni, V, dtype, dev)
+        ms = 0.0
+        rows = committed = calls = 0
+        outs = []
+        for r in range(rounds + 3):
+            fresh = [base.lg_d, base.lg_i, base.lg_f] if r == 0 else list(
+                W.hier_logits(B, loop.S, V, dtype, W.generator(9000 + r, dev), dev, **kw))
+            loop.logits(fresh)
+            w_before = loop.win_len.cpu().numpy()
+            drafts = W.window_drafts(loop.lg[0], loop.win_len, K, T, W.generator(40 + r, dev))
+            torch.cuda.synchronize()
+            if ahead:
+                torch.cuda._sleep(200_000)  # ~100 us: the host queues the call meanwhile
+            e0, e1 = _timed(lambda: loop.call(drafts, T, base.seed, base.seq_id, r))
+            torch.cuda.synchronize()
+            outs.append((loop.ctok.cpu().numpy().tobytes(), loop.cn.cpu().numpy().tobytes()))
+            if r >= 3:  # the first rounds fill the windows
+                ms += e0.elapsed_time(e1)
+                rows += loop.rows_read(w_before, greedy)
+                committed += int(loop.cn.sum().item())
+                calls += 1
+        if int(loop.status.item()) != 0:
+            raise RuntimeError(f"two-stage {kind}: device status")
+        return ms, rows, committed, calls, outs
+
+    ms, rows, committed, calls, outs = rolling(False)
+    ms_dev, _, _, _, outs_dev = rolling(True)
+    if outs_dev != outs:
+        raise RuntimeError(f"two-stage {kind}: the device-timed rounds differ")
     nbytes = rows * V * esz
     return {"workload": desc + ", rolling windows", "calls": calls,
-            "us_per_call": ms * 1e3 / calls,
+            "us_per_call": ms * 1e3 / calls, "us_per_call_device": ms_dev * 1e3 / calls,
             "committed_tokens_per_s": committed / (ms * 1e-3),
-            "algorithmic_bytes_per_call": nbytes / calls,
             "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
             "frac_of_peak_hbm": nbytes / (ms * 1e-3) / 1e9 / peak,
+            "achieved_gbs_device": nbytes / (ms_dev * 1e-3) / 1e9,
+            "frac_of_peak_hbm_device": nbytes / (ms_dev * 1e-3) / 1e9 / peak,
+            "algorithmic_bytes_per_call": nbytes / calls,
             "gpu_launches_per_call": 4}
 
 
