@@ -794,7 +794,7 @@ def run_cfg_chain_small(dev, dist):
             "us_per_round_median": statistics.median(us), "us_per_round_mean": statistics.mean(us),
             "us_per_round_graph": us_graph,
             "tokens_per_s": tokens / (sum(us) * 1e-6), "rounds": 100,
-            "bound": "latency (9 rows of 4 KB; two launches)", "gpu_launches_per_round": 2}
+            "bound": "latency (9 rows of 4 KB; one launch)", "gpu_launches_per_round": 1}
 
 
 def run_cfg_hier(dev, peak, kind, rounds):

@@ -91,6 +91,11 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 #define SPEC_VP_ROW_BYTES 32     /* one row record of a shard         */
 #define SPEC_VP_MASS_BYTES 16    /* one sequence's draw masses of a shard */
 
+/* spec_verify_chain is one launch when V <= SPEC_SMALL_V (one CTA per
+   sequence computes its rows' statistics itself, then checks and draws),
+   two launches otherwise (row statistics over all SMs, then the check). */
+#define SPEC_SMALL_V 4096
+
 /* Bytes of workspace a call needs (aligned to 256 bytes). Ni == 0 sizes a
  * chain call, Ni > 0 a two-stage call. Returns 0 for invalid sizes. */
 size_t spec_workspace_bytes(int B, int K, int V, int dtype, int Ni);
@@ -121,7 +126,11 @@ const char* spec_status_string(int status);
  *               bonus). NaN for greedy sequences.
  * ws, ws_bytes: workspace of at least spec_workspace_bytes(B, K, V, dtype, 0)
  *               bytes, 256-byte aligned. No initial contents are needed.
- * Equivalent to spec_chain_row_stats followed by spec_chain_decide.
+ * Equivalent to spec_chain_row_stats followed by spec_chain_decide. At
+ * V <= SPEC_SMALL_V it runs as one launch that forms each row's statistics
+ * in one pass per sequence instead (the sums are taken in another order, so
+ * bits may differ from the two-launch form within the verification
+ * tolerance); the workspace is checked but not written then.
  * ------------------------------------------------------------------------- */
 int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf,
                       int64_t ld_drf, int dtype, int B, int K, int V,

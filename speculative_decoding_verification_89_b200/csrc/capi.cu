@@ -11,6 +11,12 @@
 
 using namespace specv;
 
+namespace specv {
+// decide.cu: the chain check of V <= SPEC_SMALL_V in one launch, one CTA per
+// sequence forming its rows' statistics itself.
+cudaError_t launch_chain_small(const ChainDecideArgs& a, cudaStream_t st);
+}  // namespace specv
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -406,11 +412,14 @@ int spec_chain_row_stats(const void* tgt, int64_t ld_tgt, const void* drf, int64
                                       (cudaStream_t)stream));
 }
 
-int spec_chain_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
-                      int B, int K, int V, const int32_t* draft_tok, const float* temperature,
-                      uint64_t seed, const int32_t* seq_id, uint32_t round, int32_t* accept_len,
-                      int32_t* out_tok, double* diag, int32_t* dev_status, void* ws,
-                      size_t ws_bytes, void* stream) {
+// The check's launch arguments (spec_chain_decide, and the one-launch form
+// of spec_verify_chain). small: launch the one-launch form.
+static int chain_decide_call(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf,
+                             int dtype, int B, int K, int V, const int32_t* draft_tok,
+                             const float* temperature, uint64_t seed, const int32_t* seq_id,
+                             uint32_t round, int32_t* accept_len, int32_t* out_tok, double* diag,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, void* stream,
+                             bool small) {
   const ChainCheck ck = check_chain(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, ws,
                                     ws_bytes);
   if (ck.rc != SPEC_OK || B == 0) return ck.rc;
@@ -425,7 +434,18 @@ int spec_chain_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t 
   a.ld_drf = ld_drf * es;
   a.accept_len = accept_len;
   a.out_tok = out_tok;
-  return cuda_status(launch_chain_decide(a, (cudaStream_t)stream));
+  return cuda_status(small ? launch_chain_small(a, (cudaStream_t)stream)
+                           : launch_chain_decide(a, (cudaStream_t)stream));
+}
+
+int spec_chain_decide(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
+                      int B, int K, int V, const int32_t* draft_tok, const float* temperature,
+                      uint64_t seed, const int32_t* seq_id, uint32_t round, int32_t* accept_len,
+                      int32_t* out_tok, double* diag, int32_t* dev_status, void* ws,
+                      size_t ws_bytes, void* stream) {
+  return chain_decide_call(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok, temperature, seed,
+                           seq_id, round, accept_len, out_tok, diag, dev_status, ws, ws_bytes,
+                           stream, false);
 }
 
 int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t ld_drf, int dtype,
@@ -438,6 +458,10 @@ int spec_verify_chain(const void* tgt, int64_t ld_tgt, const void* drf, int64_t 
     if (layout(B, K, V, dtype, 0, &L) && B == 0) return SPEC_OK;
     return SPEC_EINVAL;
   }
+  if (V >= 1 && V <= SPEC_SMALL_V)
+    return chain_decide_call(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, draft_tok, temperature,
+                             seed, seq_id, round, accept_len, out_tok, diag, dev_status, ws,
+                             ws_bytes, stream, true);
   int rc = spec_chain_row_stats(tgt, ld_tgt, drf, ld_drf, dtype, B, K, V, temperature, dev_status,
                                 ws, ws_bytes, stream);
   if (rc != SPEC_OK) return rc;

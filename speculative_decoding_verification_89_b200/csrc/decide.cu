@@ -23,6 +23,7 @@
 // variant that also plans a paged commit (chain_decide_commit_kernel, at the
 // end of this file) adds one atomic ticket per sequence.
 #include "draw.cuh"
+#include "rowmath.cuh"
 #include "commit.cuh"
 
 namespace specv {
@@ -256,6 +257,189 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
   } else {
     const float u = o.u_draw;
     tok = leader_draw<T>(prow, qrow, V, kp, kq, dyn, dyn + nrt, u, &Z);
+  }
+  for (int j = threadIdx.x; j <= K; j += blockDim.x)
+    A.out_tok[(size_t)b * (K + 1) + j] = j < a ? drafts[j] : (j == a ? tok : -1);
+  if (threadIdx.x == 0) A.accept_len[b] = a;
+  if (diag) {
+    if (greedy) {
+      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
+    } else {
+      for (int j = threadIdx.x; j < per; j += blockDim.x) diag[j] = (sh.M[j] + sh.L[j]) * kLn2;
+      if (threadIdx.x == 0) diag[4 * K + 1] = Z;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Small chain checks (V <= kSmallV): one CTA per sequence computes its rows'
+// statistics itself, then runs the accept test and the draw, in one launch.
+// ---------------------------------------------------------------------------
+// Statistics of one row by one warp (valid in every lane): the largest logit
+// and its first index; for a sampled row (chi != 0) also the log2 partition
+// M + L of 2^(l c), M = fl(m chi), from the terms 2^(l c - M) formed in fp32
+// as the streaming statistics form them and summed per lane in fp64.
+// The EPV elements of a 16-byte vector of a row as floats.
+__device__ __forceinline__ void vec_elems(uint4 w, float x[8], __nv_bfloat16*) {
+  x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
+  x[4] = bf_lo(w.z); x[5] = bf_hi(w.z); x[6] = bf_lo(w.w); x[7] = bf_hi(w.w);
+}
+__device__ __forceinline__ void vec_elems(uint4 w, float x[4], float*) {
+  x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
+  x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
+}
+
+// Statistics of one row by one warp (valid in every lane): the largest logit
+// and its first index; for a sampled row (chi != 0) also the log2 partition
+// M + L of 2^(l c), M = fl(m chi), from the terms 2^(l c - M) formed in fp32
+// as the streaming statistics form them and summed per lane in fp64. The row
+// is read as 16-byte vectors (rows start on 16-byte boundaries), kSmallU
+// vectors per lane in flight, the last V mod EPV elements one by one; a lane
+// visits its elements in rising index order.
+constexpr int kSmallU = 4;
+template <typename T>
+__device__ RowFinal small_row(const T* row, int V, bool greedy, float chi, float clo, int lane) {
+  constexpr int EPV = 16 / (int)sizeof(T);
+  const int nv = V / EPV;
+  const uint4* rv = reinterpret_cast<const uint4*>(row);
+  float mv = -INFINITY;
+  int mi = 0x7fffffff;
+  for (int i0 = lane; i0 < nv; i0 += 32 * kSmallU) {
+    uint4 w[kSmallU];
+#pragma unroll
+    for (int u = 0; u < kSmallU; ++u) w[u] = i0 + 32 * u < nv ? __ldg(rv + i0 + 32 * u) : uint4{};
+#pragma unroll
+    for (int u = 0; u < kSmallU; ++u) {
+      if (i0 + 32 * u >= nv) break;
+      float x[EPV];
+      vec_elems(w[u], x, (T*)nullptr);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e)
+        if (x[e] > mv) {  // indices rise along the lane: ties keep the first
+          mv = x[e];
+          mi = (i0 + 32 * u) * EPV + e;
+        }
+    }
+  }
+  for (int e = nv * EPV + lane; e < V; e += 32) {
+    const float x = load_elem(row + e);
+    if (x > mv) {
+      mv = x;
+      mi = e;
+    }
+  }
+  warp_argmax(mv, mi);
+  RowFinal f{0.0, 0.0, mv, mi, 0, 0};
+  bool ok = (mv > -INFINITY && mv < INFINITY);
+  if (ok && !greedy) {
+    const float Mf = __fmul_rn(mv, chi);
+    const bool far = !(fabsf(Mf) < kFarShift);
+    const float rr = fmaf(mv, chi, -Mf) + mv * clo;
+    auto t = [&](float x) { return far ? term_far(x, mv, chi, clo, rr) : term(x, chi, clo, -Mf); };
+    double s = 0.0;
+    for (int i0 = lane; i0 < nv; i0 += 32 * kSmallU) {
+      uint4 w[kSmallU];
+#pragma unroll
+      for (int u = 0; u < kSmallU; ++u)
+        w[u] = i0 + 32 * u < nv ? __ldg(rv + i0 + 32 * u) : uint4{};
+#pragma unroll
+      for (int u = 0; u < kSmallU; ++u) {
+        if (i0 + 32 * u >= nv) break;
+        float x[EPV];
+        vec_elems(w[u], x, (T*)nullptr);
+        float v = 0.0f;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) v += t(x[e]);
+        s += (double)v;
+      }
+    }
+    for (int e = nv * EPV + lane; e < V; e += 32) s += (double)t(load_elem(row + e));
+    s = warp_sum_d(s);
+    ok = (s > 0.0 && s < INFINITY);
+    f.M = (double)Mf;
+    f.L = log2(s);
+  }
+  f.ok = ok;
+  return f;
+}
+
+constexpr int kSmallV = SPEC_SMALL_V;
+constexpr int kSmallTiles = (kSmallV + kResTile - 1) / kResTile;
+
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads) chain_small_kernel(ChainDecideArgs A) {
+  pdl_begin();
+  __shared__ SeqShared sh;
+  __shared__ Outcome s_out;
+  __shared__ double s_tsum[kSmallTiles], s_pre[kSmallTiles];
+  const DecideCommon& c = A.c;
+  const int b = blockIdx.x, K = c.K, V = c.V, per = 2 * K + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float Tb = c.temperature[b];
+  const bool tvalid = temp_valid(Tb), greedy = (Tb == 0.0f);
+  double* diag = c.diag ? c.diag + (size_t)b * (4 * K + 2) : nullptr;
+  auto fail = [&]() {
+    if (threadIdx.x == 0) {
+      set_status(c.status, SPEC_EDEVICE);
+      A.accept_len[b] = -1;
+    }
+    for (int j = threadIdx.x; j <= K; j += blockDim.x) A.out_tok[(size_t)b * (K + 1) + j] = -1;
+    if (diag)
+      for (int j = threadIdx.x; j < 4 * K + 2; j += blockDim.x) diag[j] = dnan();
+  };
+  if (!tvalid) {
+    fail();
+    return;
+  }
+  const Scale sc = greedy ? Scale{0.f, 0.f, 0.0} : make_scale(Tb);
+  const int32_t* drafts = c.draft_tok + (size_t)b * K;
+  auto tp = [&](int j) { return row_ptr<T>(A.tgt, A.ld_tgt, (long long)b * (K + 1) + j); };
+  auto dp = [&](int j) { return row_ptr<T>(A.drf, A.ld_drf, (long long)b * K + j); };
+  auto dl = [&](int j) { return sh.M[K + 1 + j] + sh.L[K + 1 + j]; };
+  const bool accept_warp = warp == kDecWarps - 1;
+  AcceptPre pre{-1, 0.f, 0.f};
+  if (accept_warp) pre = accept_prefetch<T>(K, V, greedy, drafts, tp, dp, c, b, 0, 1);
+  // Rows 0..K: target positions; K+1..2K: draft positions (sampled sequences only).
+  for (int r = warp; r < per && warp < kRowWarps; r += kRowWarps) {
+    RowFinal f{0.0, 0.0, 0.f, -1, 1, 0};
+    if (r <= K || !greedy)
+      f = small_row<T>(r <= K ? tp(r) : dp(r - K - 1), V, greedy, sc.hi, sc.lo, lane);
+    if (lane == 0) {
+      sh.m[r] = f.m;
+      sh.M[r] = f.M;
+      sh.L[r] = f.L;
+      sh.amax[r] = f.amax;
+      sh.ok[r] = f.ok;
+    }
+  }
+  __syncthreads();
+  if (accept_warp) {
+    int bad;
+    float ud;
+    const int a = accept_scan<T>(&sh, K, 0, 1, c, b, greedy, sc.d, drafts, tp, dp, dl,
+                                 diag && !greedy ? diag + 2 * K + 1 : nullptr,
+                                 diag && !greedy ? diag + 3 * K + 1 : nullptr, pre, &bad, &ud);
+    if (lane == 0) s_out = Outcome{a, bad || !rows_ok(&sh, per), ud};
+  }
+  __syncthreads();
+  const Outcome o = s_out;
+  if (o.bad) {
+    fail();
+    return;
+  }
+  const int a = o.a;
+  int tok;
+  double Z = dnan();
+  if (greedy) {
+    tok = sh.amax[a];
+  } else {
+    const T* prow = tp(a);
+    const T* qrow = a < K ? dp(a) : nullptr;
+    const ProbCoef kp = make_coef(sh.M[a] + sh.L[a], sh.m[a], sc);
+    const ProbCoef kq = a < K ? make_coef(dl(a), sh.m[K + 1 + a], sc) : make_coef(0.0, 0.0f, sc);
+    residual_tile_sums<T>(prow, qrow, V, kp, kq, 0, residual_tiles(V), s_tsum);
+    __syncthreads();
+    tok = leader_draw<T>(prow, qrow, V, kp, kq, s_tsum, s_pre, o.u_draw, &Z);
   }
   for (int j = threadIdx.x; j <= K; j += blockDim.x)
     A.out_tok[(size_t)b * (K + 1) + j] = j < a ? drafts[j] : (j == a ? tok : -1);
@@ -641,6 +825,14 @@ static cudaError_t launch_decide(Kern k, const Args& a, cudaStream_t st) {
   const cudaError_t e = reserve_dyn_smem(k, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl_cluster(k, dim3(kCluster, a.c.B), dim3(kDecThreads), smem, st, kCluster, a);
+}
+
+cudaError_t launch_chain_small(const ChainDecideArgs& a, cudaStream_t st) {
+  if (a.c.V > kSmallV || a.c.V < 1) return cudaErrorInvalidValue;
+  return a.c.dtype == SPEC_BF16
+             ? launch_pdl(chain_small_kernel<__nv_bfloat16>, dim3(a.c.B), dim3(kDecThreads), 0,
+                          st, a)
+             : launch_pdl(chain_small_kernel<float>, dim3(a.c.B), dim3(kDecThreads), 0, st, a);
 }
 
 cudaError_t launch_chain_decide(const ChainDecideArgs& a, cudaStream_t st) {

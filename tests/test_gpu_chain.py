@@ -52,8 +52,11 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("split", [False, True], ids=["verify", "two_calls"])
 @pytest.mark.parametrize("B,K,V,dtype,tspec", EDGE)
-def test_chain_edge_cases(B, K, V, dtype, tspec):
+def test_chain_edge_cases(B, K, V, dtype, tspec, split):
+    """spec_verify_chain (one launch at V <= SPEC_SMALL_V) and the two-call
+    form (row statistics, then the check) on the same inputs."""
     if tspec == "mixed":
         T = torch.tensor([0.0, 0.5, 1.0, 0.0, 2.0])[:B]
     else:
@@ -62,7 +65,7 @@ def test_chain_edge_cases(B, K, V, dtype, tspec):
     for r in range(3):
         prob = W.chain_problem(B, K, V, dtype, seed=11 + V, rnd=r, target_std=2.0,
                                draft_noise=1.0, temperature=T, philox_seed=5)
-        _compare(prob, f"B{B}K{K}V{V}r{r}", tally)
+        _compare(prob, f"B{B}K{K}V{V}r{r}", tally, split=split)
     tally.check_share()
 
 
@@ -75,7 +78,8 @@ def test_chain_equal_laws_accept_all():
     _compare(prob, "equal", tally)
 
 
-def test_chain_masked_tokens_never_drawn():
+@pytest.mark.parametrize("split", [False, True], ids=["verify", "two_calls"])
+def test_chain_masked_tokens_never_drawn(split):
     prob = W.chain_problem(6, 3, 2048, torch.float32, seed=4, temperature=1.0)
     prob.tgt[:, :, 100:1900] = float("-inf")
     prob.drf[:, :, 100:1000] = float("-inf")
@@ -83,12 +87,12 @@ def test_chain_masked_tokens_never_drawn():
     tally = Tally()
     for r in range(5):
         prob.rnd = r
-        acc, out, _, st = run_chain_gpu(prob)
+        acc, out, _, st = run_chain_gpu(prob, split=split)
         assert st == 0
         for b in range(6):
             y = int(out[b, acc[b]])
             assert not (100 <= y < 1900)
-        _compare(prob, f"masked{r}", tally)
+        _compare(prob, f"masked{r}", tally, split=split)
 
 
 def test_chain_greedy_ties_smallest_id():
@@ -106,11 +110,12 @@ def test_chain_greedy_ties_smallest_id():
     assert list(out[1]) == [4100, 4100, -1] and acc[1] == 1
 
 
-def test_chain_invalid_values_flag_only_their_sequence():
+@pytest.mark.parametrize("split", [False, True], ids=["verify", "two_calls"])
+def test_chain_invalid_values_flag_only_their_sequence(split):
     prob = W.chain_problem(4, 3, 1000, torch.float32, seed=6, temperature=1.0)
     prob.draft_tok[1, 2] = 1000          # out of range
     prob.temperature[2] = -1.0           # invalid temperature
-    acc, out, _, st = run_chain_gpu(prob)
+    acc, out, _, st = run_chain_gpu(prob, split=split)
     assert st == -6
     assert acc[1] == -1 and acc[2] == -1 and np.all(out[1] == -1) and np.all(out[2] == -1)
     ref = run_chain_oracle(prob, [0, 3])

@@ -1,6 +1,7 @@
 """Chain verification fused with the paged commit (spec_verify_chain_commit)
-against the oracle and against the two-call path (spec_verify_chain, then
-spec_commit_paged with keep = accept_len + 1) on the same inputs: accepted
+against the oracle and against the separate calls of the same kernels
+(spec_chain_row_stats and spec_chain_decide, then spec_commit_paged with
+keep = accept_len + 1) on the same inputs: accepted
 counts, tokens, probabilities, tables, lengths, free stack, moved K/V rows and
 the packed hidden rows. The two GPU paths must agree bit for bit; the oracle
 comparison follows the chain and commit acceptance rules."""
@@ -48,7 +49,8 @@ def _run(prob, state, bufs, fused, base=None, status0=0, persistent=False):
         fn(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, t, l, b_len, f, top, s, ws,
            block_size=state.block_size, diag=dg, **kw)
     else:
-        capi.spec_verify_chain(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, s, ws,
+        capi.spec_chain_row_stats(tgt, drf, T, s, ws)
+        capi.spec_chain_decide(tgt, drf, dt, T, prob.seed, sid, prob.rnd, acc, out, s, ws,
                                diag=dg)
         capi.spec_commit_paged(t, l, b_len, acc, 1, f, top, K + 1, s,
                                block_size=state.block_size, **kw)
