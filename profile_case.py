@@ -8,6 +8,7 @@ while the whole case stays well under a few GB of device memory.
     python profile_case.py --B 32
     python profile_case.py --B 64 --commit
     python profile_case.py --B 64 --vp 8
+    python profile_case.py --small        (B=1, K=4, V=1024 fp32: the one-launch check)
 """
 from __future__ import annotations
 
@@ -33,12 +34,16 @@ def main():
     ap.add_argument("--outcome", type=int, default=-1,
                     help="run the outcome law with this many outcomes instead of verifying")
     ap.add_argument("--draft", action="store_true", help="run the draft step instead of verifying")
+    ap.add_argument("--small", action="store_true",
+                    help="chain verification of B=1, K=4, V=1024 fp32 (fresh rows each call)")
     ap.add_argument("--vp", type=int, default=0,
                     help="run the vocabulary-parallel check over this many shards, the ranks "
                          "in turn on this GPU, instead of verifying")
     args = ap.parse_args()
     B, K, V = args.B, 8, W.LLAMA3_V
     dev = torch.device("cuda")
+    if args.small:
+        return small(args, dev)
     acc = torch.zeros(B, dtype=torch.int32, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     if not args.no_verify:
@@ -82,6 +87,22 @@ def main():
         torch.cuda.synchronize()
         times.append(ev[0].elapsed_time(ev[1]) * 1e3)
     print(f"B={B} status={int(st.item())} us/iter median={sorted(times)[len(times) // 2]:.1f}")
+    if int(st.item()) != 0:
+        raise SystemExit(1)
+
+
+def small(args, dev):
+    """B=1, K=4, V=1024 fp32 chain checks on fresh rows each call."""
+    probs = [W.chain_small(rnd=r, device=dev) for r in range(args.iters)]
+    ws = capi.workspace(1, 4, 1024, torch.float32, device=dev)
+    acc = torch.empty(1, dtype=torch.int32, device=dev)
+    out = torch.empty((1, 5), dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    for i, p in enumerate(probs):
+        capi.spec_verify_chain(p.tgt, p.drf, p.draft_tok, p.temperature, p.seed, p.seq_id, i, acc,
+                               out, st, ws)
+    torch.cuda.synchronize()
+    print(f"small: {len(probs)} calls, status={int(st.item())}")
     if int(st.item()) != 0:
         raise SystemExit(1)
 
