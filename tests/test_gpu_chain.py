@@ -69,6 +69,22 @@ def test_chain_edge_cases(B, K, V, dtype, tspec, split):
     tally.check_share()
 
 
+@pytest.mark.parametrize("split", [False, True], ids=["verify", "two_calls"])
+@pytest.mark.parametrize("V", [2000, 6000])
+def test_chain_far_shift(V, split):
+    """Temperature 2e-6 on logits of spread 60: the row maxima times 1/(T ln 2)
+    lie far above 2^26, where both paths form the exponentials relative to
+    the row maximum (V=2000 takes the one-launch path, V=6000 the row
+    statistics launch)."""
+    tally = Tally()
+    for r in range(3):
+        prob = W.chain_problem(3, 3, V, torch.float32, seed=21, rnd=r, target_std=60.0,
+                               draft_noise=1.0, temperature=2e-6, philox_seed=9)
+        assert float(prob.tgt.max()) / (2e-6 * 0.6931471805599453) > 2.0 ** 26
+        _compare(prob, f"far/V{V}/r{r}", tally, split=split)
+    tally.check_share()
+
+
 def test_chain_equal_laws_accept_all():
     prob = W.chain_problem(8, 6, 5000, torch.bfloat16, seed=3, temperature=0.9)
     prob.drf = prob.tgt[:, :6].clone()
