@@ -272,14 +272,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) chain_decide_kernel(ChainDecid
 }
 
 // ---------------------------------------------------------------------------
-// Small chain checks (V <= kSmallV): one CTA per sequence computes its rows'
-// statistics itself, then runs the accept test and the draw, in one launch.
+// Small chain checks (V <= SPEC_SMALL_V): one CTA per sequence computes its
+// rows' statistics itself, then runs the accept test and the draw, in one
+// launch.
 // ---------------------------------------------------------------------------
-// Statistics of one row by one warp (valid in every lane): the largest logit
-// and its first index; for a sampled row (chi != 0) also the log2 partition
-// M + L of 2^(l c), M = fl(m chi), from the terms 2^(l c - M) formed in fp32
-// as the streaming statistics form them and summed per lane in fp64.
-// The EPV elements of a 16-byte vector of a row as floats.
+// The elements of a 16-byte vector of a row as floats.
 __device__ __forceinline__ void vec_elems(uint4 w, float x[8], __nv_bfloat16*) {
   x[0] = bf_lo(w.x); x[1] = bf_hi(w.x); x[2] = bf_lo(w.y); x[3] = bf_hi(w.y);
   x[4] = bf_lo(w.z); x[5] = bf_hi(w.z); x[6] = bf_lo(w.w); x[7] = bf_hi(w.w);
