@@ -867,6 +867,20 @@ def run_cfg_hier(dev, peak, kind, rounds):
 
 
 def run_cfg_engine(dev, rounds=256):
+    """The engine loop from a fresh state, timed as called from Python and
+    again with each round's work queued behind a short device sleep (the
+    device time alone); the two passes must commit the same tokens."""
+    paced = _engine_loop(dev, rounds, ahead=False)
+    ahead = _engine_loop(dev, rounds, ahead=True)
+    if ahead["outputs"] != paced["outputs"]:
+        raise RuntimeError("engine loop: the device-timed pass differs")
+    out = {k: v for k, v in paced.items() if k != "outputs"}
+    out["ms_per_round_device"] = ahead["ms_per_round"]
+    out["committed_tokens_per_s_device"] = ahead["committed_tokens_per_s"]
+    return out
+
+
+def _engine_loop(dev, rounds, ahead):
     """Engine loop: 64 sequences x 256 rounds, K = N_i = 4, V=32000 bf16,
     logits regenerated each round from a generator seeded by (4, round); each
     round reserves the cycle's slots in the block tables, drafts its K tokens
@@ -875,7 +889,8 @@ def run_cfg_engine(dev, rounds=256):
     (sequence, round, slot)), verifies, commits the committed tokens and
     rolls the reservation back (block 16, pool of 65536 blocks, starts
     U[128, 2048]). Committed tokens per second of the device work, with and
-    without the round's logit generation."""
+    without the round's logit generation (ahead: the work queued behind a
+    device sleep, without the generation)."""
     from speculative_decoding_verification_89_b200 import capi
     from speculative_decoding_verification_89_b200 import workloads as W
     B, K, Ni, V = 64, 4, 4, 32000
@@ -895,20 +910,25 @@ def run_cfg_engine(dev, rounds=256):
     draft_T = torch.ones(B * K, device=dev)
     draft_tok = torch.empty(B * K, dtype=torch.int32, device=dev)
     kk = torch.arange(K, device=dev).view(1, K)
+    base_row = torch.arange(B, device=dev).view(B, 1) * S
     ms_work = ms_all = 0.0
     total = 0
+    h = hashlib.sha256()
     for r in range(rounds):
         a0 = torch.cuda.Event(enable_timing=True)
         a0.record()
         fresh, _ = W.engine_round_logits(B, S, V, r, dev)
         loop.logits(fresh)
+        if ahead:
+            torch.cuda.synchronize()
+            torch.cuda._sleep(400_000)  # ~200 us: the host queues the round meanwhile
         w0 = torch.cuda.Event(enable_timing=True)
         w0.record()
         capi.spec_commit_paged(state.tables, state.seq_lens, committed, full, 0,
                                state.free_stack, state.free_top, S, st, block_size=16)
         slots = loop.win_len.long().view(B, 1) + kk  # the window's next K slots
-        torch.gather(loop.lg[0], 1, slots.view(B, K, 1).expand(B, K, V),
-                     out=draft_rows.view(B, K, V))
+        torch.index_select(loop.lg[0].view(B * S, V), 0, (base_row + slots).view(-1),
+                           out=draft_rows)  # whole rows: (b, slot) -> b * S + slot
         capi.spec_draft_sample(draft_rows, draft_T, 40, draft_sid, r,
                                slots.view(-1).to(torch.int32), draft_tok, st, draft_ws)
         loop.call(draft_tok.view(B, K), T, 4, seq_id, r)
@@ -921,6 +941,8 @@ def run_cfg_engine(dev, rounds=256):
         ms_work += w0.elapsed_time(w1)
         ms_all += a0.elapsed_time(w1)
         total += int(loop.cn.sum().item())
+        h.update(loop.ctok.cpu().numpy().tobytes())
+    h.update(state.tables.cpu().numpy().tobytes())
     if int(st.item()) != 0 or int(loop.status.item()) != 0:
         raise RuntimeError("engine loop: device status")
     return {"workload": "engine loop 64 sequences x 256 rounds, K=N_i=4, V=32000 bf16, drafts "
@@ -929,7 +951,8 @@ def run_cfg_engine(dev, rounds=256):
             "rounds": rounds, "committed_tokens": total,
             "committed_tokens_per_s": total / (ms_work * 1e-3),
             "committed_tokens_per_s_with_logit_generation": total / (ms_all * 1e-3),
-            "ms_per_round": ms_work / rounds, "ms_per_round_with_logit_generation": ms_all / rounds}
+            "ms_per_round": ms_work / rounds, "ms_per_round_with_logit_generation": ms_all / rounds,
+            "outputs": h.hexdigest()}
 
 
 # ----------------------------------------------------------------------------

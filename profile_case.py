@@ -9,6 +9,7 @@ while the whole case stays well under a few GB of device memory.
     python profile_case.py --B 64 --commit
     python profile_case.py --B 64 --vp 8
     python profile_case.py --small        (B=1, K=4, V=1024 fp32: the one-launch check)
+    python profile_case.py --engine --iters 8   (rounds of the benchmark's engine loop)
 """
 from __future__ import annotations
 
@@ -34,6 +35,8 @@ def main():
     ap.add_argument("--outcome", type=int, default=-1,
                     help="run the outcome law with this many outcomes instead of verifying")
     ap.add_argument("--draft", action="store_true", help="run the draft step instead of verifying")
+    ap.add_argument("--engine", action="store_true",
+                    help="--iters rounds of the engine loop (64 sequences, V=32000 bf16)")
     ap.add_argument("--small", action="store_true",
                     help="chain verification of B=1, K=4, V=1024 fp32 (fresh rows each call)")
     ap.add_argument("--vp", type=int, default=0,
@@ -44,6 +47,11 @@ def main():
     dev = torch.device("cuda")
     if args.small:
         return small(args, dev)
+    if args.engine:
+        import bench
+        r = bench.run_cfg_engine(dev, rounds=args.iters)
+        print(f"engine: {args.iters} rounds, {r['ms_per_round_device'] * 1e3:.1f} us per round")
+        return None
     acc = torch.zeros(B, dtype=torch.int32, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     if not args.no_verify:
