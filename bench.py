@@ -909,8 +909,8 @@ def _engine_loop(dev, rounds, ahead):
     draft_sid = seq_id.repeat_interleave(K)
     draft_T = torch.ones(B * K, device=dev)
     draft_tok = torch.empty(B * K, dtype=torch.int32, device=dev)
-    kk = torch.arange(K, device=dev).view(1, K)
-    base_row = torch.arange(B, device=dev).view(B, 1) * S
+    kk = torch.arange(K, dtype=torch.int32, device=dev).view(1, K)
+    base_row = torch.arange(B, device=dev).view(B, 1) * S  # int64: the flat row index
     ms_work = ms_all = 0.0
     total = 0
     h = hashlib.sha256()
@@ -926,11 +926,11 @@ def _engine_loop(dev, rounds, ahead):
         w0.record()
         capi.spec_commit_paged(state.tables, state.seq_lens, committed, full, 0,
                                state.free_stack, state.free_top, S, st, block_size=16)
-        slots = loop.win_len.long().view(B, 1) + kk  # the window's next K slots
+        slots = loop.win_len.view(B, 1) + kk  # the window's next K slots (int32)
         torch.index_select(loop.lg[0].view(B * S, V), 0, (base_row + slots).view(-1),
                            out=draft_rows)  # whole rows: (b, slot) -> b * S + slot
-        capi.spec_draft_sample(draft_rows, draft_T, 40, draft_sid, r,
-                               slots.view(-1).to(torch.int32), draft_tok, st, draft_ws)
+        capi.spec_draft_sample(draft_rows, draft_T, 40, draft_sid, r, slots.view(-1), draft_tok,
+                               st, draft_ws)
         loop.call(draft_tok.view(B, K), T, 4, seq_id, r)
         capi.spec_commit_paged(state.tables, state.seq_lens, committed, loop.cn, 0,
                                state.free_stack, state.free_top, S, st, block_size=16)
