@@ -9,8 +9,8 @@
 // mind-verse.de, SVIP paragraphs), from which a draft-length policy decides
 // whether to keep drafting.
 //
-// One launch when a cluster of 4 (or 8) CTAs can hold a row in shared memory
-// (draft_fused_kernel: every logit read from HBM once, statistics and draw
+// One launch when a cluster of up to 8 CTAs can hold a row in shared memory
+// (draft_fused_kernel, 1 to 8 CTAs per row as launch_draft_step chooses: every logit read from HBM once, statistics and draw
 // from shared memory). Larger rows take two launches: the row-statistics
 // kernel over the B rows (DraftRows, which also gathers the first moment sum
 // 2^(l*c - M) * (l - m)), then one thread-block cluster per sequence that
@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) draft_draw_kernel(DraftArgs A)
 // the token.
 constexpr int kDfMaxCluster = 8;
 constexpr int kDfSliceBytes = 100 * 1024;  // staged slice per CTA, at most
+constexpr int kDfSmallSlice = 16;           // tiles: a slice this short is not split further
 constexpr uint32_t kDfChunk = 32768;        // bytes per bulk copy (whole tiles)
 constexpr int kDfMaxChunks = (kDfSliceBytes + (int)kDfChunk - 1) / (int)kDfChunk;
 // Per tile of the slice: the scaled sum (double), then m_t, M_t, S_t, T_t.
@@ -567,11 +568,18 @@ cudaError_t launch_draft_step(int dtype, const unsigned char* lg, long long ld_b
                               uint32_t round, const int32_t* pos, Partial* part, double* mom,
                               int32_t* out_tok, double* out_logq, double* out_entropy,
                               int32_t* status, cudaStream_t st) {
-  // One launch when a cluster of 4 (or 8) CTAs holds the row in shared memory.
+  // One launch when a cluster of up to 8 CTAs holds the row in shared memory:
+  // clusters of 1 or 2 CTAs when that slice fits and either the grid still
+  // gives every SM a CTA or the slice is at most kDfSmallSlice tiles, else the
+  // smallest of 4 and 8 that fits. (B200, bf16 rows: 256 x 32000 takes 14.2 us
+  // per call with clusters of 1, 18.1 with 2, 26.2 with 4; 64 x 32000 10.3,
+  // 8.2 and 7.6; 8 x 4096 6.0, 6.2 and 6.4; the same tokens at every size.)
   const int esz = dtype == SPEC_BF16 ? 2 : 4, nrt = residual_tiles(V);
-  for (int cs = 4; cs <= kDfMaxCluster; cs *= 2) {
+  const int sms = sm_count();
+  for (int cs = 1; cs <= kDfMaxCluster; cs *= 2) {
     const int tc = (nrt + cs - 1) / cs;
     if ((size_t)tc * kResTile * esz > (size_t)kDfSliceBytes) continue;
+    if (cs < 4 && !((long long)B * cs >= sms || tc <= kDfSmallSlice)) continue;
     DraftArgs a{};
     a.B = B;
     a.V = V;
