@@ -41,6 +41,8 @@ EDGE = [
     (3, 0, 1000, torch.float32, 1.0),          # no drafts: plain draw from p
     (2, 1, 1, torch.float32, 1.0),             # single-token vocabulary
     (2, 2, 7, torch.bfloat16, 0.9),            # row shorter than one vector
+    (3, 4, 4096, torch.bfloat16, 0.6),         # the largest one-launch vocabulary
+    (3, 4, 4096, torch.float32, 1.7),          # the same in fp32
     (4, 3, 4097, torch.bfloat16, 0.8),         # ragged: one bf16 tile + 1
     (4, 3, 8191, torch.float32, 1.3),          # ragged fp32 tiles, odd tail
     (5, 2, 12345, torch.bfloat16, "mixed"),    # greedy and sampled in a batch
